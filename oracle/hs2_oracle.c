@@ -1,0 +1,288 @@
+/*
+ * hs2_oracle.c -- plain, slow, fp64 CPU oracle for HySparse2's Cross-Decoder
+ * attention hot path.  TEST INFRASTRUCTURE ONLY: the product path (the CUDA
+ * library and its Python binding) never links, loads or calls this file.
+ * Only the tests, the smoke check and the benchmark's CPU-baseline leg use it.
+ *
+ * What it computes, per query token ("row") at absolute position t of one
+ * sequence, following the HySparse2 pages:
+ *   - "KV Reuse" (xiawanshe.com report, section "两级KV共享", second level):
+ *     one full-attention layer of the Cross-Decoder produces the KV cache AND
+ *     a token-selection result; several following sparse-attention layers
+ *     reuse both.
+ *   - "Token-level selection" (same report, section "Token级选择"): tokens are
+ *     picked one by one; the most recent 128 tokens are always kept and 1024
+ *     tokens are picked from the older context; local and global attention
+ *     share one KV cache.  The davidyin.dev video notes (section "HySparse2
+ *     的解法") add that no extra indexer is trained.
+ *
+ * Where the pages are silent this file takes the readings below (each one is
+ * the plainest reading the pages support):
+ *   - softmax scale 1/sqrt(D), causal row j in [0, t], natural-log LSE;
+ *   - heads map to KV groups contiguously: g = h / G, G = H_q / H_kv;
+ *   - window(t) = [max(0, t-W+1), t] (W tokens including t itself);
+ *     candidates are j in [0, t-W], n_cand = max(0, t-W+1);
+ *   - selection score of candidate j for group g = sum over the G heads of the
+ *     group of the causal softmax probability p_{h,t,j} (normalised over the
+ *     whole causal row, window included);
+ *   - the selection takes the min(K, n_cand) candidates first in the order
+ *     (score descending, j ascending) -- ties go to the lower index -- and is
+ *     emitted sorted ascending by j, padded with -1;
+ *   - a sparse layer attends, per head, to the set idx_g(t) U window(t) with
+ *     its own query, same K/V, same 1/sqrt(D) scale.
+ *
+ * Every quantity is computed in double precision from the bf16 inputs widened
+ * exactly (bf16 bits << 16 is an exact fp32, and fp32 -> fp64 is exact).
+ * No blocking, no online softmax, no fusion: each step is the textbook
+ * definition written out.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define HS2O_OK 0
+#define HS2O_EINVAL 1
+#define HS2O_ENOMEM 2
+#define HS2O_EIDX 3
+
+static double bf16_to_double(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+typedef struct {
+    double score;
+    int64_t j;
+} cand_t;
+
+/* Order "first is better": larger score first, then smaller j. */
+static int cand_cmp(const void* a, const void* b) {
+    const cand_t* x = (const cand_t*)a;
+    const cand_t* y = (const cand_t*)b;
+    if (x->score > y->score) return -1;
+    if (x->score < y->score) return 1;
+    if (x->j < y->j) return -1;
+    if (x->j > y->j) return 1;
+    return 0;
+}
+
+static int i32_cmp(const void* a, const void* b) {
+    int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+    return (x > y) - (x < y);
+}
+
+/* s[j] = scale * <q_h, k_{g,j}> for j in [0, n). */
+static void dot_scores(const uint16_t* qh, const uint16_t* kg, int64_t n, int d,
+                       double scale, double* s) {
+    double qd[512];
+    for (int e = 0; e < d; ++e) qd[e] = bf16_to_double(qh[e]);
+    for (int64_t j = 0; j < n; ++j) {
+        const uint16_t* kj = kg + j * (int64_t)d;
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += qd[e] * bf16_to_double(kj[e]);
+        s[j] = acc * scale;
+    }
+}
+
+/*
+ * Full causal attention + selection for n_rows query tokens of ONE sequence.
+ *
+ * q      [n_rows, h_q, d]        bf16 bits, the full-attention layer's queries
+ * t      [n_rows]                absolute position of each query (0 <= t < kv_len)
+ * k, v   [h_kv, kv_stride, d]    bf16 bits, the shared cache of the sequence
+ * out    [n_rows, h_q, d]        softmax(s) . v, fp64
+ * lse    [n_rows, h_q]           ln sum_j exp(s_j), fp64
+ * idx    [n_rows, h_kv, topk]    selection, ascending, -1 padded
+ * kth    [n_rows, h_kv]          score of the last selected candidate in rank
+ *                                order (NAN when nothing is selected)
+ * next   [n_rows, h_kv]          score of the best unselected candidate
+ *                                (-1 when every candidate is selected)
+ * scores [n_rows, h_kv, score_stride] or NULL: score of every candidate
+ *                                j in [0, t-window] (entries beyond n_cand untouched)
+ */
+int hs2o_full_select(int h_q, int h_kv, int d, int window, int topk, double scale,
+                     int64_t n_rows, const int64_t* t, const uint16_t* q,
+                     const uint16_t* k, const uint16_t* v, int64_t kv_len, int64_t kv_stride,
+                     double* out, double* lse, int32_t* idx, double* kth, double* next,
+                     double* scores, int64_t score_stride, int n_threads) {
+    if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0 || d <= 0 || d > 512 || window < 1 ||
+        topk < 0 || n_rows < 0 || kv_len > kv_stride)
+        return HS2O_EINVAL;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (t[r] < 0 || t[r] >= kv_len) return HS2O_EINVAL;
+    const int G = h_q / h_kv;
+    int err = HS2O_OK;
+    const int64_t n_work = n_rows * h_kv;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t w = 0; w < n_work; ++w) {
+        const int64_t r = w / h_kv;
+        const int g = (int)(w % h_kv);
+        const int64_t tr = t[r];
+        const int64_t n_causal = tr + 1;
+        const int64_t n_cand = tr - window + 1 > 0 ? tr - window + 1 : 0;
+        double* s = (double*)malloc(sizeof(double) * (size_t)n_causal);
+        double* grp = (double*)calloc((size_t)(n_cand > 0 ? n_cand : 1), sizeof(double));
+        cand_t* cand = (cand_t*)malloc(sizeof(cand_t) * (size_t)(n_cand > 0 ? n_cand : 1));
+        if (!s || !grp || !cand) {
+            free(s); free(grp); free(cand);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = HS2O_ENOMEM;
+            continue;
+        }
+        const uint16_t* kg = k + (int64_t)g * kv_stride * d;
+        const uint16_t* vg = v + (int64_t)g * kv_stride * d;
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            const uint16_t* qh = q + (r * h_q + h) * (int64_t)d;
+            /* step 1: scaled dot products over the causal row */
+            dot_scores(qh, kg, n_causal, d, scale, s);
+            /* step 2: lse = m + ln sum exp(s - m) */
+            double m = -INFINITY;
+            for (int64_t j = 0; j < n_causal; ++j) m = s[j] > m ? s[j] : m;
+            double z = 0.0;
+            for (int64_t j = 0; j < n_causal; ++j) z += exp(s[j] - m);
+            const double l = m + log(z);
+            lse[r * h_q + h] = l;
+            /* out_h = sum_j exp(s_j - lse) v_j */
+            double* o = out + (r * h_q + h) * (int64_t)d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (int64_t j = 0; j < n_causal; ++j) {
+                const double p = exp(s[j] - l);
+                const uint16_t* vj = vg + j * (int64_t)d;
+                for (int e = 0; e < d; ++e) o[e] += p * bf16_to_double(vj[e]);
+            }
+            /* step 3: group score = sum over the group's heads of p_{h,j} */
+            for (int64_t j = 0; j < n_cand; ++j) grp[j] += exp(s[j] - l);
+        }
+        /* step 4: rank candidates by (score desc, j asc), keep the first n */
+        for (int64_t j = 0; j < n_cand; ++j) {
+            cand[j].score = grp[j];
+            cand[j].j = j;
+        }
+        if (scores)
+            for (int64_t j = 0; j < n_cand; ++j) scores[(r * h_kv + g) * score_stride + j] = grp[j];
+        qsort(cand, (size_t)n_cand, sizeof(cand_t), cand_cmp);
+        const int64_t n_sel = n_cand < topk ? n_cand : topk;
+        int32_t* row_idx = idx + (r * h_kv + g) * (int64_t)topk;
+        for (int64_t i = 0; i < n_sel; ++i) row_idx[i] = (int32_t)cand[i].j;
+        qsort(row_idx, (size_t)n_sel, sizeof(int32_t), i32_cmp);
+        for (int64_t i = n_sel; i < topk; ++i) row_idx[i] = -1;
+        kth[r * h_kv + g] = n_sel > 0 ? cand[n_sel - 1].score : NAN;
+        next[r * h_kv + g] = n_sel < n_cand ? cand[n_sel].score : -1.0;
+        free(s);
+        free(grp);
+        free(cand);
+    }
+    return err;
+}
+
+/*
+ * One sparse (KV-reuse) layer for n_rows query tokens of ONE sequence:
+ * per head h, softmax attention of the layer's own query over the set
+ * idx_{g}(t) U window(t), g = h / G.
+ *
+ * idx [n_rows, h_kv, topk]: entries are -1 (unused) or a candidate index in
+ * [0, t-window]; duplicates are rejected (HS2O_EIDX).
+ */
+int hs2o_sparse(int h_q, int h_kv, int d, int window, int topk, double scale,
+                int64_t n_rows, const int64_t* t, const uint16_t* q,
+                const uint16_t* k, const uint16_t* v, int64_t kv_len, int64_t kv_stride,
+                const int32_t* idx, double* out, int n_threads) {
+    if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0 || d <= 0 || d > 512 || window < 1 ||
+        topk < 0 || n_rows < 0 || kv_len > kv_stride)
+        return HS2O_EINVAL;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (t[r] < 0 || t[r] >= kv_len) return HS2O_EINVAL;
+    const int G = h_q / h_kv;
+    int err = HS2O_OK;
+    const int64_t n_work = n_rows * h_kv;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t w = 0; w < n_work; ++w) {
+        const int64_t r = w / h_kv;
+        const int g = (int)(w % h_kv);
+        const int64_t tr = t[r];
+        const int64_t w0 = tr - window + 1 > 0 ? tr - window + 1 : 0;
+        /* the attended set: selected candidates, then the window */
+        int64_t* set = (int64_t*)malloc(sizeof(int64_t) * (size_t)(topk + window));
+        double* s = (double*)malloc(sizeof(double) * (size_t)(topk + window));
+        if (!set || !s) {
+            free(set); free(s);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = HS2O_ENOMEM;
+            continue;
+        }
+        int64_t n = 0;
+        int bad = 0;
+        const int32_t* ir = idx + (r * h_kv + g) * (int64_t)topk;
+        for (int i = 0; i < topk; ++i) {
+            const int64_t j = ir[i];
+            if (j == -1) continue;
+            if (j < 0 || j > tr - window) { bad = 1; break; }
+            for (int64_t u = 0; u < n; ++u)
+                if (set[u] == j) { bad = 1; break; }
+            if (bad) break;
+            set[n++] = j;
+        }
+        if (bad) {
+            free(set); free(s);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = HS2O_EIDX;
+            continue;
+        }
+        for (int64_t j = w0; j <= tr; ++j) set[n++] = j;
+        const uint16_t* kg = k + (int64_t)g * kv_stride * d;
+        const uint16_t* vg = v + (int64_t)g * kv_stride * d;
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            const uint16_t* qh = q + (r * h_q + h) * (int64_t)d;
+            double qd[512];
+            for (int e = 0; e < d; ++e) qd[e] = bf16_to_double(qh[e]);
+            double m = -INFINITY;
+            for (int64_t u = 0; u < n; ++u) {
+                const uint16_t* kj = kg + set[u] * (int64_t)d;
+                double acc = 0.0;
+                for (int e = 0; e < d; ++e) acc += qd[e] * bf16_to_double(kj[e]);
+                s[u] = acc * scale;
+                m = s[u] > m ? s[u] : m;
+            }
+            double z = 0.0;
+            for (int64_t u = 0; u < n; ++u) z += exp(s[u] - m);
+            double* o = out + (r * h_q + h) * (int64_t)d;
+            for (int e = 0; e < d; ++e) o[e] = 0.0;
+            for (int64_t u = 0; u < n; ++u) {
+                const double p = exp(s[u] - m) / z;
+                const uint16_t* vj = vg + set[u] * (int64_t)d;
+                for (int e = 0; e < d; ++e) o[e] += p * bf16_to_double(vj[e]);
+            }
+        }
+        free(set);
+        free(s);
+    }
+    return err;
+}
+
+int hs2o_max_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
