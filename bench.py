@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Throughput of the HySparse2 Cross-Decoder attention hot path on B200.
+
+One step = the full-attention + selection layer (hs2_full_attn_select, or
+hs2_decode for decode workloads) followed by every sparse KV-reuse layer
+(hs2_sparse_attn / hs2_decode_sparse, one call per layer, each with its own
+query), over one batch of seeded synthetic input already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...    # the fp64 CPU oracle, same workload
+
+Prints ONE JSON line on rank 0.  Metric: query tokens/s through the whole
+step.  With N > 1 (torchrun), every rank runs an independent replica of the
+workload (its own sequences: weak scaling, no data-path collective); value =
+all ranks' query tokens / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_flash_b200 import native as nv  # noqa: E402
+from long_context_sparse_flash_b200 import workloads as wl  # noqa: E402
+
+METRIC = "query tokens/s (full-attn+select + sparse-reuse layers) and % of TC/HBM roofline"
+UNIT = "query tokens/s"
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return dict(hbm=float(d["hbm_gbs"]), tc=float(d["bf16_tflops"]),
+                    tc_sustained=float(d["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, tc=1590.0, tc_sustained=1400.0, src="fallback")
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per kernel (per call of the entry point, all sequences)
+
+
+def kernel_work(w: wl.Workload):
+    f = wl.flops_and_bytes(w)
+    D, Hq, Hk = w.head_dim, w.h_q, w.h_kv
+    n_rows = w.batch * w.n_q
+    cand = f["cand"]  # sum over (sequence, query, KV head) of candidate counts
+    return {
+        # dense causal contraction: QK^T and PV over the causal pairs
+        "full_attn": dict(bound="tensor", flops=f["full_flops"]),
+        "fused_attn_select": dict(bound="tensor", flops=f["full_flops"] + f["select_qk_flops"]),
+        "decode_attn": dict(bound="hbm", bytes=f["kv_bytes"] + 2 * f["q_bytes"] + 4 * n_rows * Hq),
+        # QK^T recompute over the candidates of every query
+        "select_score": dict(bound="tensor", flops=f["select_qk_flops"]),
+        # read every stored score once, write idx
+        "select_topk": dict(bound="hbm", bytes=4.0 * cand + f["idx_bytes"]),
+        # gathered K/V rows + q + out + idx, per layer
+        "sparse_attn": dict(bound="hbm", bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
+    }
+
+
+def source_sha(path: str) -> str:
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+KERNEL_SOURCE = {
+    "full_attn": "k1_full_attn.cu", "select_score": "k2_select.cu", "select_topk": "k2_select.cu",
+    "sparse_attn": "k3_sparse_attn.cu",
+}
+
+
+def dram_traffic(kernel: str, workload: str):
+    """Per-launch DRAM bytes from the committed ncu summary, if it was taken on
+    the current source of that kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    src = KERNEL_SOURCE.get(kernel)
+    if not src or not os.path.exists(path):
+        return None
+    cur = source_sha(os.path.join(ROOT, "long_context_sparse_flash_b200", "csrc", src))
+    for line in open(path):
+        parts = line.split()
+        if len(parts) >= 4 and not line.startswith("#") and parts[0] == kernel and parts[1] == workload:
+            if parts[2] == cur:
+                return float(parts[3])
+    return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+
+
+class ClockSampler:
+    FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.proc = None
+        self.uuid = None
+        try:
+            u = str(torch.cuda.get_device_properties(device).uuid)
+            self.uuid = u if u.startswith("GPU-") else "GPU-" + u
+        except Exception:
+            pass
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
+        if self.uuid:
+            mine = [r for r in rows if r[0] == self.uuid]
+            rows = mine or rows
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                for name, val in zip(names, r[4:8]):
+                    if val.strip().lower() == "active":
+                        reasons.add(name)
+            except (ValueError, IndexError):
+                continue
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+
+
+class Step:
+    """Buffers and the C-ABI calls of one step."""
+
+    def __init__(self, w: wl.Workload, inp: dict, device):
+        self.w = w
+        self.q, self.k, self.v = inp["q"], inp["k"], inp["v"]
+        self.qs = inp["q_sparse"]
+        B, Hq, nq, D = self.q.shape
+        self.shape = nv.shape_of(self.q, self.k, window=w.window, topk=w.topk,
+                                 q_pos0=(w.kv_len - 1) if w.decode else w.q_pos0)
+        entry = nv.HS2_ENTRY_DECODE if w.decode else nv.HS2_ENTRY_FULL_SELECT
+        self.ws = nv.alloc_workspace(self.shape, entry, device)
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty(B, Hq, nq, dtype=torch.float32, device=device)
+        self.idx = torch.empty(B, w.h_kv, nq, w.topk, dtype=torch.int32, device=device)
+        self.sp_out = [torch.empty_like(self.q) for _ in self.qs]
+
+    def __call__(self):
+        if self.w.decode:
+            nv.hs2_decode(self.shape, None, self.q, self.k, self.v, self.out, self.lse, self.idx, self.ws)
+            for qs, o in zip(self.qs, self.sp_out):
+                nv.hs2_decode_sparse(self.shape, None, qs, self.k, self.v, self.idx, o, None)
+        else:
+            nv.hs2_full_attn_select(self.shape, self.q, self.k, self.v, self.out, self.lse, self.idx, self.ws)
+            for qs, o in zip(self.qs, self.sp_out):
+                nv.hs2_sparse_attn(self.shape, qs, self.k, self.v, self.idx, o, None)
+
+    def inputs(self):
+        return [self.q, self.k, self.v, *self.qs]
+
+    def outputs(self):
+        return [self.out, self.lse, self.idx, *self.sp_out]
+
+
+def dist_setup(n_gpus: int):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def time_steps(step, K: int, flush_buf: torch.Tensor, ws: int):
+    """K steps, L2 flushed (outside the timed events) before each."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for a, b in evs:
+        flush_buf.zero_()
+        a.record()
+        step()
+        b.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    return [a.elapsed_time(b) for a, b in evs]
+
+
+def time_e2e(step: Step, K: int, ws: int):
+    """Same metric end to end: pinned host inputs copied in, the C-ABI calls, results copied out."""
+    h_in = [t.cpu().pin_memory() for t in step.inputs()]
+    h_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in step.outputs()]
+    d_in = step.inputs()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(ws)
+    torch.cuda.synchronize()
+    for a, b in evs:
+        a.record()
+        for h, d in zip(h_in, d_in):
+            d.copy_(h, non_blocking=True)
+        step()
+        for h, d in zip(h_out, step.outputs()):
+            h.copy_(d, non_blocking=True)
+        b.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = [a.elapsed_time(b) for a, b in evs]
+    bi = sum(t.numel() * t.element_size() for t in h_in)
+    bo = sum(t.numel() * t.element_size() for t in h_out)
+    return ms, bi, bo
+
+
+def cpu_baseline(w: wl.Workload, inp: dict, n_rows: int, seed: int = 2024) -> dict:
+    """The oracle, as it stands, on a bounded seeded sample of the workload's
+    query rows (full attention + selection + every sparse layer per row)."""
+    import oracle
+    cores = len(os.sched_getaffinity(0))
+    rng = np.random.default_rng(seed)
+    if w.decode:
+        seqs = rng.choice(w.batch, size=min(n_rows, w.batch), replace=False)
+        picks = [(int(b), np.array([0]), np.array([w.kv_len - 1])) for b in seqs]
+    else:
+        rows = np.sort(rng.choice(w.n_q, size=min(n_rows, w.n_q), replace=False))
+        picks = [(0, rows, w.q_pos0 + rows)]
+    prepared = []
+    for b, rows, ts in picks:
+        rt = torch.as_tensor(rows, device=inp["q"].device)
+        kb, vb = wl.bf16_bits(inp["k"][b]), wl.bf16_bits(inp["v"][b])
+        qb = np.ascontiguousarray(wl.bf16_bits(inp["q"][b][:, rt]).transpose(1, 0, 2))
+        qsb = [np.ascontiguousarray(wl.bf16_bits(qs[b][:, rt]).transpose(1, 0, 2)) for qs in inp["q_sparse"]]
+        prepared.append((ts, qb, qsb, kb, vb))
+    t0 = time.perf_counter()
+    n = 0
+    for ts, qb, qsb, kb, vb in prepared:
+        res = oracle.full_select(qb, ts, kb, vb, window=w.window, topk=w.topk, n_threads=cores)
+        for q2 in qsb:
+            oracle.sparse(q2, ts, kb, vb, res["idx"], window=w.window, n_threads=cores)
+        n += len(ts)
+    dt = time.perf_counter() - t0
+    mean_t = float(np.mean(np.concatenate([p[0] for p in prepared]))) + 1
+    return {"value": n / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} seeded random query rows of {w.name} (mean context {mean_t:.0f} tokens), "
+                      f"full-attn+select and {w.n_sparse} sparse layers each, {dt:.2f} s",
+            "_rows": n, "_seconds": dt}
+
+
+def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
+    work = kernel_work(w)
+    per = {}
+    for name, (ms, launches) in prof.items():
+        if name not in work or ms <= 0:
+            continue
+        wk = work[name]
+        calls = K * (w.n_sparse if name == "sparse_attn" else 1)
+        if wk["bound"] == "tensor":
+            achieved = wk["flops"] * calls / (ms / 1e3) / 1e12
+            peak, unit = pk["tc_sustained"], "TFLOP/s"
+        else:
+            achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
+            peak, unit = pk["hbm"], "GB/s"
+        per[name] = dict(ms=ms / K, launches=launches // K if K else launches, bound=wk["bound"],
+                         achieved=round(achieved, 2), peak=peak, unit=unit, frac=round(achieved / peak, 4))
+    if not per:
+        return None, per
+    top = max(per, key=lambda n: per[n]["ms"])
+    p = per[top]
+    launches_total = prof[top][1]
+    traffic = dram_traffic(top, w.name)
+    rf = {"kernel": top, "bound": "hbm" if p["bound"] == "hbm" else "tensor", "achieved": p["achieved"],
+          "peak": p["peak"], "unit": p["unit"], "frac": p["frac"],
+          "peak_source": pk["src"] + (" (sustained bf16)" if p["bound"] == "tensor" else " (copy GB/s)"),
+          "launches_per_step": launches_total / K, "traffic": traffic,
+          "share_of_step": None}
+    return rf, per
+
+
+def run_ours(args):
+    ws, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.WORKLOADS[args.workload]
+    nv.load()
+    inp = wl.make_inputs(w, dev, seed=w.seed + 1000 * rank)  # independent replica per rank
+    step = Step(w, inp, dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, info = nv.hs2_get_device_status(step.ws)
+    if st != 0:
+        raise RuntimeError(f"device error word after warm-up: {st} {info}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    l0 = nv.hs2_launch_count()
+    nv.hs2_profile_start()
+    ms = time_steps(step, args.steps, flush, ws)
+    prof = nv.hs2_profile_stop()
+    launches = nv.hs2_launch_count() - l0
+    clk = clocks.stop()
+    total_ms = max_over_ranks(float(sum(ms)), ws)
+    ms_per_step = total_ms / args.steps
+    tokens = w.query_tokens * ws * args.steps
+    value = tokens / (total_ms / 1e3)
+
+    e2e = None
+    if not args.no_e2e:
+        ems, bi, bo = time_e2e(step, args.steps, ws)
+        e_total = max_over_ranks(float(sum(ems)), ws)
+        e2e = {"value": round(tokens / (e_total / 1e3), 2), "unit": UNIT, "h2d_bytes_per_step": bi,
+               "d2h_bytes_per_step": bo, "ms_per_step": round(e_total / args.steps, 3)}
+
+    pk = peaks()
+    rf, per_kernel = roofline(w, prof, args.steps, pk)
+    if rf is not None:
+        rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp, args.cpu_rows)
+        cpu.pop("_rows"), cpu.pop("_seconds")
+        cpu["value"] = round(cpu["value"], 4)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded, shapes and value distributions of the workload; no dataset)",
+            "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "q_pos0": w.q_pos0,
+                       "kv_len": w.kv_len, "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim,
+                       "window": w.window, "topk": w.topk, "sparse_layers": w.n_sparse,
+                       "parallelism": f"replicas x{ws} (independent sequences per GPU)",
+                       "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write, outside the events)"},
+            "per_kernel": per_kernel,
+            "roofline": rf,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+            "step_ms": {"median": round(statistics.median(ms), 4), "min": round(min(ms), 4),
+                        "max": round(max(ms), 4)},
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.destroy_process_group()
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle as it stands, on a bounded sample
+    of the same workload per step (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    w = wl.WORKLOADS[args.workload]
+    inp = wl.make_inputs(w, "cpu")
+    rows_per_step = max(1, args.ref_rows)
+    samples, cores = [], None
+    total_rows, total_s = 0, 0.0
+    for s in range(args.warmup + args.steps):
+        c = cpu_baseline(w, inp, rows_per_step, seed=3000 + s)
+        if s >= args.warmup:
+            samples.append(c["sample"])
+            cores = c["cores"]
+            total_rows += c["_rows"]
+            total_s += c["_seconds"]
+    value = total_rows / total_s
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_s / args.steps, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded, shapes and value distributions of the workload; no dataset)",
+        "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "q_pos0": w.q_pos0, "kv_len": w.kv_len,
+                   "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim, "window": w.window, "topk": w.topk,
+                   "sparse_layers": w.n_sparse, "parallelism": "host cores (OpenMP over rows)"},
+        "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows_per_step} seeded random query rows per step; " + samples[-1]},
+        "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="prefill_32k", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=64, help="query rows in the oracle baseline sample")
+    ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference-arm step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("note: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

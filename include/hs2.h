@@ -1,0 +1,179 @@
+/*
+ * hs2.h -- C ABI of libhs2: HySparse2 Cross-Decoder attention on one B200.
+ *
+ * The method (HySparse2 pages):
+ *   - xiawanshe.com report, section "两级KV共享" (second level, "KV Reuse"):
+ *     inside the Cross-Decoder one full-attention layer produces the KV cache
+ *     and a token-selection result, and several following sparse-attention
+ *     layers reuse both.
+ *   - same report, section "Token级选择": selection is per token, anywhere in
+ *     the context; the separate SWA branch is dropped; the most recent 128
+ *     tokens are always attended and 1024 tokens are selected from the older
+ *     context; local and global attention share one KV cache.
+ *   - davidyin.dev video notes, section "HySparse2 的解法": no extra indexer
+ *     is trained for the selection.
+ *
+ * Definitions used by every entry point (t = absolute position of a query):
+ *   s_{h,j}   = softmax_scale * <q_h, k_{g,j}>, g = h / G, G = h_q / h_kv, j in [0, t]
+ *   lse_h     = ln sum_{j<=t} exp(s_{h,j})            (natural log, fp32)
+ *   out_h     = sum_{j<=t} exp(s_{h,j} - lse_h) v_{g,j}
+ *   window(t) = [max(0, t-window+1), t]               (window tokens incl. t)
+ *   score_{g,j} = sum_{h in g} exp(s_{h,j} - lse_h),   j in [0, t-window]
+ *   idx_g(t)  = the min(topk, max(0, t-window+1)) candidates first in the order
+ *               (score descending, j ascending), stored ascending by j, then
+ *               -1 padding up to topk entries.
+ *   sparse layer: out'_h = softmax over S = idx_g(t) U window(t) of
+ *               softmax_scale * <q'_h, k_{g,j}>, applied to v_{g,j}.
+ *
+ * Layouts (all row-major, contiguous, device memory, 16-byte aligned):
+ *   q, q'  [batch, h_q, n_q, head_dim]      bf16
+ *   k, v   [batch, h_kv, kv_len, head_dim]  bf16   (the shared cache)
+ *   out    [batch, h_q, n_q, head_dim]      bf16
+ *   lse    [batch, h_q, n_q]                fp32
+ *   idx    [batch, h_kv, n_q, topk]         int32
+ * Query i of a call sits at t = q_pos0 + i; kv_len >= q_pos0 + n_q.
+ *
+ * Ownership: the caller allocates and owns every buffer, including the
+ * workspace; the library allocates no device memory and keeps no per-call
+ * state.  Execution: every entry point validates its arguments on the host,
+ * returns an error status without launching anything if a check fails, and
+ * otherwise enqueues its kernels on `stream` and returns at once (no host
+ * synchronisation), except hs2_get_device_status which synchronises `stream`.
+ * A call whose sizes make the work empty (batch == 0 or n_q == 0) returns
+ * HS2_OK without launching.
+ */
+#ifndef HS2_H
+#define HS2_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Binary compatible with cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* hs2_stream_t;
+
+typedef enum {
+    HS2_OK = 0,
+    HS2_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misaligned pointer      */
+    HS2_ERR_UNSUPPORTED = 2,   /* valid but outside the built kernels' range      */
+    HS2_ERR_WORKSPACE = 3,     /* ws_bytes below hs2_workspace_size()             */
+    HS2_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed            */
+    HS2_ERR_DEVICE_CHECK = 5,  /* a kernel found an invalid input (error word)    */
+    HS2_ERR_TIMEOUT = 6        /* a bounded device-side wait gave up (error word) */
+} hs2_status;
+
+/* Problem description shared by all entry points.
+ *   head_dim in {64, 128}; h_q % h_kv == 0 with G = h_q / h_kv in {1, 2, 4, 8};
+ *   1 <= window <= 1024; 0 <= topk <= 2048; q_pos0 >= 0;
+ *   q_pos0 + n_q <= kv_len <= 2^31 - 1; softmax_scale == 0 selects 1/sqrt(head_dim),
+ *   otherwise it must be finite and > 0; reserved must be 0. */
+typedef struct {
+    int32_t batch;
+    int32_t n_q;
+    int32_t h_q;
+    int32_t h_kv;
+    int32_t head_dim;
+    int32_t window;
+    int32_t topk;
+    int32_t reserved;
+    int64_t q_pos0;
+    int64_t kv_len;
+    float softmax_scale;
+} hs2_shape;
+
+enum {
+    HS2_ENTRY_FULL_SELECT = 0,
+    HS2_ENTRY_SPARSE = 1,
+    HS2_ENTRY_PREFILL = 2,
+    HS2_ENTRY_DECODE = 3
+};
+
+/* Bytes of workspace the entry point `entry` needs for `shape` (0 if the shape
+ * is invalid).  The first 256 bytes of every workspace hold the device error
+ * word; hs2_workspace_init() must zero them once before first use. */
+size_t hs2_workspace_size(const hs2_shape* shape, int entry);
+
+/* Zero the workspace header (error word) on `stream`.  Asynchronous. */
+hs2_status hs2_workspace_init(void* ws, size_t ws_bytes, hs2_stream_t stream);
+
+/* Full-attention layer of the Cross-Decoder with token selection
+ * (xiawanshe.com report, "两级KV共享" KV Reuse + "Token级选择").
+ * Reads q, k, v; writes out, lse and idx for every query of the call.  Runs the
+ * full-attention pass, then the selection pass that recomputes the scores
+ * from the written LSE (two separate kernels).  ws: hs2_workspace_size(shape,
+ * HS2_ENTRY_FULL_SELECT) bytes, contents are scratch except the header. */
+hs2_status hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k,
+                                const void* v, void* out, float* lse, int32_t* idx,
+                                void* ws, size_t ws_bytes, hs2_stream_t stream);
+
+/* One sparse KV-reuse layer (xiawanshe.com report, "两级KV共享": the following
+ * sparse layers reuse the full layer's cache and selection; "Token级选择": they
+ * attend to the selected tokens plus the forced recent window).  q is this
+ * layer's own query; k, v and idx are those of the full-attention layer.
+ * idx rows must be as hs2_full_attn_select writes them (ascending valid
+ * entries in [0, t-window], then -1); the checked build reports violations
+ * through the error word.  ws may be NULL with ws_bytes == 0. */
+hs2_status hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v,
+                           const int32_t* idx, void* out, void* ws, size_t ws_bytes,
+                           hs2_stream_t stream);
+
+/* Prefill-chunk entry: the full-attention + selection layer for a chunk of
+ * n_q new tokens appended to a cache of kv_len tokens (q_pos0 = kv_len - n_q
+ * for an append; any q_pos0 with q_pos0 + n_q <= kv_len is accepted).  Same
+ * arguments, workspace rule and outputs as hs2_full_attn_select. */
+hs2_status hs2_prefill_chunk(const hs2_shape* shape, const void* q, const void* k,
+                             const void* v, void* out, float* lse, int32_t* idx, void* ws,
+                             size_t ws_bytes, hs2_stream_t stream);
+
+/* Decode entry: one new token per sequence (n_q == 1).  kv_len_per_seq is a
+ * device array of `batch` int64 lengths (1 <= len <= kv_len; the query of
+ * sequence b sits at t = len_b - 1 and its own K/V row is already in the
+ * cache), or NULL for len_b = kv_len for every b (q_pos0 is then ignored).
+ * The selection pass splits every sequence's candidates over many CTAs.
+ * Out-of-range lengths are clamped and reported through the error word. */
+hs2_status hs2_decode(const hs2_shape* shape, const int64_t* kv_len_per_seq, const void* q,
+                      const void* k, const void* v, void* out, float* lse, int32_t* idx,
+                      void* ws, size_t ws_bytes, hs2_stream_t stream);
+
+/* One sparse KV-reuse layer for decode-shaped calls (n_q == 1) whose sequences
+ * have their own cache lengths: the query of sequence b sits at
+ * t = kv_len_per_seq[b] - 1 (device int64 array; NULL means kv_len for every
+ * b).  Otherwise identical to hs2_sparse_attn; idx is what hs2_decode wrote. */
+hs2_status hs2_decode_sparse(const hs2_shape* shape, const int64_t* kv_len_per_seq, const void* q,
+                             const void* k, const void* v, const int32_t* idx, void* out, void* ws,
+                             size_t ws_bytes, hs2_stream_t stream);
+
+/* Synchronise `stream`, read and clear the workspace error word.  Returns
+ * HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA).  If
+ * `info` is non-NULL it receives 4 words: code, kernel id, and two values
+ * describing the first failure. */
+hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info);
+
+/* Static description of a status code. */
+const char* hs2_status_string(hs2_status status);
+
+/* Number of kernels this library has launched in this process (all threads). */
+uint64_t hs2_launch_count(void);
+
+/* Measurement aid: from hs2_profile_start() on, the library records a CUDA
+ * event pair on the launching stream around every kernel it launches (event
+ * objects only, no device memory).  hs2_profile_stop() ends the recording,
+ * waits for the recorded events, and writes, for every kernel id u < n_kinds,
+ * the summed event time in ms (total_ms[u]) and the launch count
+ * (launches[u]); either array may be NULL.  Kernel ids: 1 full attention,
+ * 2 selection scores, 3 top-k select, 4 sparse attention, 5 decode attention
+ * partials, 6 decode combine, 7 fused attention + selection. */
+hs2_status hs2_profile_start(void);
+hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
+
+/* 1 when the library was built with device-side input checks (HS2_CHECKED). */
+int hs2_is_checked_build(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HS2_H */

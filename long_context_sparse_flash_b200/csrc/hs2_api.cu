@@ -1,0 +1,321 @@
+// hs2_api.cu -- the extern "C" boundary of libhs2: argument validation,
+// workspace layout, dispatch of the kernels onto the caller's stream.
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "hs2_kernels.h"
+
+namespace hs2 {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch(int n) { g_launches.fetch_add((uint64_t)n, std::memory_order_relaxed); }
+
+// ---------------------------------------------------------------------------
+// per-kernel event timing (measurement aid; off unless hs2_profile_start ran)
+
+namespace {
+struct ProfRec {
+    uint32_t kid;
+    cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<bool> g_prof_on{false};
+std::vector<ProfRec> g_prof_recs;      // recorded, not yet collected
+std::vector<cudaEvent_t> g_prof_pool;  // free events
+thread_local uint32_t t_prof_kid = 0;
+thread_local cudaEvent_t t_prof_a = nullptr;
+
+cudaEvent_t prof_event() {
+    cudaEvent_t e = nullptr;
+    if (!g_prof_pool.empty()) {
+        e = g_prof_pool.back();
+        g_prof_pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+        e = nullptr;
+    }
+    return e;
+}
+}  // namespace
+
+void prof_begin(uint32_t kid, cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    t_prof_kid = kid;
+    t_prof_a = prof_event();
+    if (t_prof_a) cudaEventRecord(t_prof_a, st);
+}
+
+void prof_end(cudaStream_t st) {
+    if (!g_prof_on.load(std::memory_order_relaxed) || t_prof_a == nullptr) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = prof_event();
+    if (b) {
+        cudaEventRecord(b, st);
+        g_prof_recs.push_back({t_prof_kid, t_prof_a, b});
+    } else {
+        g_prof_pool.push_back(t_prof_a);
+    }
+    t_prof_a = nullptr;
+}
+
+namespace {
+
+constexpr size_t kHeader = sizeof(WsHeader);
+constexpr size_t kScoreBudget = size_t(1) << 30;  // bytes of stored scores per chunk of queries
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+// Host validation of the shape; fills `p` on success.
+hs2_status check_shape(const hs2_shape* s, Problem* p) {
+    if (s == nullptr) return HS2_ERR_INVALID_ARG;
+    if (s->reserved != 0) return HS2_ERR_INVALID_ARG;
+    if (s->batch < 0 || s->n_q < 0 || s->h_q <= 0 || s->h_kv <= 0 || s->head_dim <= 0) return HS2_ERR_INVALID_ARG;
+    if (s->h_q % s->h_kv != 0) return HS2_ERR_INVALID_ARG;
+    if (s->window < 1 || s->topk < 0 || s->q_pos0 < 0 || s->kv_len < 0) return HS2_ERR_INVALID_ARG;
+    if (s->q_pos0 + (int64_t)s->n_q > s->kv_len) return HS2_ERR_INVALID_ARG;
+    const float sc = s->softmax_scale;
+    if (!(sc == 0.f || (std::isfinite(sc) && sc > 0.f))) return HS2_ERR_INVALID_ARG;
+    const int G = s->h_q / s->h_kv;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return HS2_ERR_UNSUPPORTED;
+    if (s->head_dim != 64 && s->head_dim != 128) return HS2_ERR_UNSUPPORTED;
+    if (s->window > 1024 || s->topk > 2048) return HS2_ERR_UNSUPPORTED;
+    if (s->kv_len > INT32_MAX || s->batch > 65535 || s->h_q > 65535) return HS2_ERR_UNSUPPORTED;
+    p->B = s->batch;
+    p->nq = s->n_q;
+    p->hq = s->h_q;
+    p->hkv = s->h_kv;
+    p->D = s->head_dim;
+    p->window = s->window;
+    p->topk = s->topk;
+    p->q_pos0 = s->q_pos0;
+    p->kv_len = s->kv_len;
+    const float scale = sc == 0.f ? 1.0f / std::sqrt((float)s->head_dim) : sc;
+    p->scale_log2 = scale * kLog2e;
+    p->seq_len = nullptr;
+    p->err = nullptr;
+    return HS2_OK;
+}
+
+// Stored-score layout of the selection pass: queries are processed in chunks
+// of `chunk` rows; each (sequence, group, query) row holds `sstride` floats.
+struct ScorePlan {
+    int64_t sstride = 0;
+    int chunk = 0;
+    size_t bytes = 0;
+};
+
+ScorePlan score_plan(const Problem& p, bool decode) {
+    ScorePlan sp;
+    const int64_t t_hi = decode ? p.kv_len - 1 : p.q_pos0 + p.nq - 1;
+    const int64_t cand = t_hi - p.window + 1;
+    if (cand <= p.topk || p.nq == 0 || p.B == 0 || p.topk == 0) return sp;  // every row takes all candidates
+    sp.sstride = (cand + 3) / 4 * 4;
+    const size_t per_q = (size_t)p.B * p.hkv * sp.sstride * 4;
+    int64_t chunk = (int64_t)(kScoreBudget / per_q);
+    if (chunk >= 256) chunk = chunk / 128 * 128;
+    if (chunk < 1) chunk = 1;
+    if (chunk > p.nq) chunk = p.nq;
+    sp.chunk = (int)chunk;
+    sp.bytes = (size_t)chunk * per_q;
+    return sp;
+}
+
+hs2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA; }
+
+hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool decode, const void* q,
+                           const void* k, const void* v, void* out, float* lse, int32_t* idx, void* ws,
+                           size_t ws_bytes, hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (decode && p.nq != 1 && p.nq != 0) return HS2_ERR_INVALID_ARG;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k || !v || !out || !lse || !ws) return HS2_ERR_INVALID_ARG;
+    if (p.topk > 0 && !idx) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(idx, 4) || !aligned(ws, 256) || (seq_len && !aligned(seq_len, 8)))
+        return HS2_ERR_INVALID_ARG;
+    const ScorePlan sp = score_plan(p, decode);
+    if (ws_bytes < kHeader + sp.bytes) return HS2_ERR_WORKSPACE;
+    p.seq_len = seq_len;
+    p.err = reinterpret_cast<WsHeader*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = launch_full(p, q, k, v, out, lse, st);
+    if (e != cudaSuccess) return HS2_ERR_CUDA;
+    if (p.topk == 0) return HS2_OK;
+    float* scores = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kHeader);
+    const int chunk = sp.chunk > 0 ? sp.chunk : p.nq;
+    for (int i0 = 0; i0 < p.nq; i0 += chunk) {
+        const int cnt = p.nq - i0 < chunk ? p.nq - i0 : chunk;
+        if (sp.sstride > 0) {
+            e = launch_score(p, q, k, lse, scores, i0, cnt, sp.sstride, st);
+            if (e != cudaSuccess) return HS2_ERR_CUDA;
+        }
+        e = launch_topk(p, scores, sp.sstride, idx, i0, cnt, st);
+        if (e != cudaSuccess) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
+}  // namespace
+}  // namespace hs2
+
+using namespace hs2;
+
+extern "C" {
+
+size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
+    Problem p;
+    if (check_shape(shape, &p) != HS2_OK) return 0;
+    switch (entry) {
+        case HS2_ENTRY_SPARSE: return kHeader;
+        case HS2_ENTRY_FULL_SELECT:
+        case HS2_ENTRY_PREFILL: return kHeader + score_plan(p, false).bytes;
+        case HS2_ENTRY_DECODE: return kHeader + score_plan(p, true).bytes;
+        default: return 0;
+    }
+}
+
+hs2_status hs2_workspace_init(void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    if (ws == nullptr || ws_bytes < kHeader || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
+    return cuda_status(cudaMemsetAsync(ws, 0, kHeader, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v, void* out,
+                                float* lse, int32_t* idx, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    return run_full_select(shape, nullptr, false, q, k, v, out, lse, idx, ws, ws_bytes, stream);
+}
+
+hs2_status hs2_prefill_chunk(const hs2_shape* shape, const void* q, const void* k, const void* v, void* out,
+                             float* lse, int32_t* idx, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    return run_full_select(shape, nullptr, false, q, k, v, out, lse, idx, ws, ws_bytes, stream);
+}
+
+hs2_status hs2_decode(const hs2_shape* shape, const int64_t* kv_len_per_seq, const void* q, const void* k,
+                      const void* v, void* out, float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                      hs2_stream_t stream) {
+    if (shape == nullptr) return HS2_ERR_INVALID_ARG;
+    hs2_shape s = *shape;
+    if (s.n_q != 1 && s.n_q != 0) return HS2_ERR_INVALID_ARG;
+    if (s.kv_len < 1 && s.n_q == 1) return HS2_ERR_INVALID_ARG;
+    s.q_pos0 = s.kv_len > 0 ? s.kv_len - 1 : 0;  // sequences without a length array end at kv_len - 1
+    return run_full_select(&s, kv_len_per_seq, true, q, k, v, out, lse, idx, ws, ws_bytes, stream);
+}
+
+namespace hs2 {
+namespace {
+hs2_status run_sparse(const hs2_shape* shape, const int64_t* seq_len, const void* q, const void* k, const void* v,
+                      const int32_t* idx, void* out, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (seq_len && !aligned(seq_len, 8)) return HS2_ERR_INVALID_ARG;
+    p.seq_len = seq_len;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k || !v || !out || (p.topk > 0 && !idx)) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(idx, 4))
+        return HS2_ERR_INVALID_ARG;
+    if (ws != nullptr) {
+        if (ws_bytes < kHeader || !aligned(ws, 256)) return HS2_ERR_WORKSPACE;
+        p.err = reinterpret_cast<WsHeader*>(ws);
+    } else if (ws_bytes != 0) {
+        return HS2_ERR_INVALID_ARG;
+    }
+    return cuda_status(launch_sparse(p, q, k, v, idx, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+}  // namespace
+}  // namespace hs2
+
+hs2_status hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
+                           void* out, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    return run_sparse(shape, nullptr, q, k, v, idx, out, ws, ws_bytes, stream);
+}
+
+hs2_status hs2_decode_sparse(const hs2_shape* shape, const int64_t* kv_len_per_seq, const void* q, const void* k,
+                             const void* v, const int32_t* idx, void* out, void* ws, size_t ws_bytes,
+                             hs2_stream_t stream) {
+    if (shape == nullptr) return HS2_ERR_INVALID_ARG;
+    hs2_shape s = *shape;
+    if (s.n_q != 1 && s.n_q != 0) return HS2_ERR_INVALID_ARG;
+    if (s.kv_len < 1 && s.n_q == 1) return HS2_ERR_INVALID_ARG;
+    s.q_pos0 = s.kv_len > 0 ? s.kv_len - 1 : 0;
+    return run_sparse(&s, kv_len_per_seq, q, k, v, idx, out, ws, ws_bytes, stream);
+}
+
+hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info) {
+    if (ws == nullptr || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint32_t h[4] = {0, 0, 0, 0};
+    if (cudaStreamSynchronize(st) != cudaSuccess) return HS2_ERR_CUDA;
+    if (cudaMemcpy(h, ws, sizeof h, cudaMemcpyDeviceToHost) != cudaSuccess) return HS2_ERR_CUDA;
+    if (h[0] != 0) {
+        if (cudaMemset(ws, 0, sizeof h) != cudaSuccess) return HS2_ERR_CUDA;
+    }
+    if (info) {
+        for (int u = 0; u < 4; ++u) info[u] = h[u];
+    }
+    if (h[0] == HS2_ERR_DEVICE_CHECK) return HS2_ERR_DEVICE_CHECK;
+    if (h[0] == HS2_ERR_TIMEOUT) return HS2_ERR_TIMEOUT;
+    return h[0] == 0 ? HS2_OK : HS2_ERR_DEVICE_CHECK;
+}
+
+const char* hs2_status_string(hs2_status status) {
+    switch (status) {
+        case HS2_OK: return "ok";
+        case HS2_ERR_INVALID_ARG: return "invalid argument";
+        case HS2_ERR_UNSUPPORTED: return "unsupported shape";
+        case HS2_ERR_WORKSPACE: return "workspace too small";
+        case HS2_ERR_CUDA: return "CUDA error";
+        case HS2_ERR_DEVICE_CHECK: return "device-side input check failed";
+        case HS2_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+uint64_t hs2_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+hs2_status hs2_profile_start(void) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (auto& r : g_prof_recs) {
+        g_prof_pool.push_back(r.a);
+        g_prof_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+    g_prof_on.store(true);
+    return HS2_OK;
+}
+
+hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches) {
+    g_prof_on.store(false);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    for (uint32_t u = 0; u < n_kinds; ++u) {
+        if (total_ms) total_ms[u] = 0.f;
+        if (launches) launches[u] = 0;
+    }
+    hs2_status st = HS2_OK;
+    for (auto& r : g_prof_recs) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess)
+            st = HS2_ERR_CUDA;
+        if (r.kid < n_kinds) {
+            if (total_ms) total_ms[r.kid] += ms;
+            if (launches) launches[r.kid] += 1;
+        }
+        g_prof_pool.push_back(r.a);
+        g_prof_pool.push_back(r.b);
+    }
+    g_prof_recs.clear();
+    return st;
+}
+
+int hs2_is_checked_build(void) {
+#ifdef HS2_CHECKED
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+}  // extern "C"

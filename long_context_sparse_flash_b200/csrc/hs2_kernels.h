@@ -1,0 +1,58 @@
+// hs2_kernels.h -- host-side launchers of the libhs2 kernels (internal).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "hs2_common.cuh"
+
+namespace hs2 {
+
+// A validated problem, as the kernels see it.
+struct Problem {
+    int B, nq, hq, hkv, D, window, topk;
+    int64_t q_pos0, kv_len;   // kv_len is also the row stride of k/v per (b, g)
+    float scale_log2;         // softmax_scale * log2(e)
+    const int64_t* seq_len;   // decode: per-sequence cache lengths (device) or nullptr
+    WsHeader* err;            // device error word or nullptr
+};
+
+// count of kernel launches issued by the library
+void count_launch(int n = 1);
+
+// Per-kernel timing (enabled by hs2_profile_start): an event pair recorded on
+// the launching stream around every launch.  Bracket each launch with
+// prof_begin / prof_end; both are no-ops while profiling is off.
+void prof_begin(uint32_t kid, cudaStream_t st);
+void prof_end(cudaStream_t st);
+
+// K1: causal full attention + LSE for every query of the call.
+cudaError_t launch_full(const Problem& p, const void* q, const void* k, const void* v, void* out,
+                        float* lse, cudaStream_t st);
+
+// K2 part 1: selection scores of queries [i_begin, i_begin + i_count) into
+// scores[((b * hkv + g) * i_count + (i - i_begin)) * sstride + j], j <= t - window.
+cudaError_t launch_score(const Problem& p, const void* q, const void* k, const float* lse,
+                         float* scores, int i_begin, int i_count, int64_t sstride,
+                         cudaStream_t st);
+
+// K2 part 2: exact top-k per (query, KV head) over the stored scores.
+cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, int32_t* idx,
+                        int i_begin, int i_count, cudaStream_t st);
+
+// K3: one sparse KV-reuse layer.
+cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v,
+                          const int32_t* idx, void* out, cudaStream_t st);
+
+// Query position of query 0 of sequence b: q_pos0, or seq_len[b] - nq for decode
+// (clamped into [0, kv_len - nq]; a clamp is reported through the error word).
+__device__ __forceinline__ int64_t seq_pos0(const Problem& p, int b, uint32_t kid) {
+    if (p.seq_len == nullptr) return p.q_pos0;
+    int64_t len = p.seq_len[b];
+    if (len < p.nq || len > p.kv_len) {
+        if (threadIdx.x == 0) report_error(p.err, HS2_ERR_DEVICE_CHECK, kid, (uint32_t)b, (uint32_t)len);
+        len = len < p.nq ? p.nq : p.kv_len;
+    }
+    return len - p.nq;
+}
+
+}  // namespace hs2

@@ -1,0 +1,337 @@
+// k2_select.cu -- K2: token-level selection of HySparse2 (xiawanshe.com report,
+// section "Token级选择": per-token choice of 1024 older tokens beside the forced
+// 128-token window; davidyin.dev notes, "HySparse2 的解法": no trained indexer,
+// so the score comes from the full-attention layer itself).
+//
+// Score of candidate j for KV group g at query t:
+//     score = sum_{h in g} 2^(s2_{h,j} - lse2_h),  s2 = scale*log2(e)*<q_h,k_j>,
+// recomputed from the LSE that K1 wrote.  Part 1 (k2_score_kernel) computes the
+// scores with mma.sync in the transposed form S^T = K Q^T, so one 16-key x
+// 8-column tile holds one query's 8 heads (G = 8) in one row of the fragment and
+// the group sum is two in-thread adds plus two quad shuffles.  Part 2
+// (k2_topk_kernel) selects the top-k of each (query, group) row exactly: a
+// 4-pass, 8-bit radix select on the fp32 bit patterns (non-negative floats order
+// like their bits) finds the k-th key, then one ordered pass keeps every key
+// above it plus the lowest-index keys equal to it, writing indices ascending.
+#include "hs2_kernels.h"
+
+namespace hs2 {
+
+namespace {
+
+constexpr int SC_WARPS = 8;
+constexpr int SC_BN = 64;  // keys per staged tile
+
+template <int D, int G>
+__global__ void __launch_bounds__(SC_WARPS * 32) k2_score_kernel(Problem p, const __nv_bfloat16* __restrict__ q,
+                                                                  const __nv_bfloat16* __restrict__ k,
+                                                                  const float* __restrict__ lse,
+                                                                  float* __restrict__ scores, int i_begin,
+                                                                  int i_count, int64_t sstride,
+                                                                  int64_t keys_per_split, int splits) {
+    constexpr int CH = D / 8;
+    constexpr int QPN = 8 / G;                   // queries per 8-column n-tile
+    constexpr int QPC = SC_WARPS * 2 * QPN;      // queries per CTA
+    constexpr int T_BYTES = SC_BN * D * 2;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = blockIdx.y;
+    const int b = blockIdx.z / splits, split = blockIdx.z % splits;
+    const int64_t pos0 = seq_pos0(p, b, KID_SCORE);
+    const int qc0 = blockIdx.x * QPC;            // first query of the CTA, relative to i_begin
+    const int q_end = min(qc0 + QPC, i_count);   // exclusive
+    if (qc0 >= q_end) return;
+    const int64_t t_hi = pos0 + i_begin + q_end - 1;
+    const int64_t cand_end = t_hi - p.window + 1;  // candidates are j < cand_end
+    const int64_t j_lo = (int64_t)split * keys_per_split;
+    const int64_t j_hi = min(j_lo + keys_per_split, cand_end);
+    if (j_lo >= j_hi) return;
+    const int n_tiles = (int)((j_hi - j_lo + SC_BN - 1) / SC_BN);
+
+    const __nv_bfloat16* kg = k + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
+    const uint32_t s_t = smem_u32(smem);
+    auto load_tile = [&](int kt, int stage) {
+        const uint32_t sk = s_t + stage * T_BYTES;
+        for (int c = tid; c < SC_BN * CH; c += SC_WARPS * 32) {
+            const int r = c / CH, ch = c % CH;
+            const int64_t j = j_lo + (int64_t)kt * SC_BN + r;
+            const bool ok = j < j_hi;
+            cp_async16(sk + swz<CH>(r, ch), kg + (ok ? j : 0) * D + ch * 8, ok ? 16 : 0);
+        }
+    };
+    load_tile(0, 0);
+    cp_async_commit();
+
+    // B fragments (Q^T) of this warp's two n-tiles: column c = query (c / G), head (c % G)
+    uint32_t qb[2][D / 16][2];
+    float l2[2][2];          // lse * log2(e) of this thread's two columns per n-tile
+    int64_t t_col[2][2];     // absolute position of the column's query (-1: none)
+    int row_col[2][2];       // score row of the column's query
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        {
+            const int c = lane >> 2;  // column this thread feeds to the B fragment
+            const int qi = qc0 + (warp * 2 + nt) * QPN + c / G;
+            const int hh = c % G;
+            const bool ok = qi < q_end;
+            const int i = i_begin + (ok ? qi : qc0);
+            const __nv_bfloat16* qrow = q + ((int64_t)(b * p.hq + g * G + hh) * p.nq + i) * D;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                const int d0 = ks * 16 + 2 * (lane & 3);
+                qb[nt][ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+                qb[nt][ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int c = 2 * (lane & 3) + e;  // column of accumulator element e
+            const int qi = qc0 + (warp * 2 + nt) * QPN + c / G;
+            const int hh = c % G;
+            const bool ok = qi < q_end;
+            const int i = i_begin + (ok ? qi : qc0);
+            l2[nt][e] = ok ? lse[(int64_t)(b * p.hq + g * G + hh) * p.nq + i] * kLog2e : INFINITY;
+            t_col[nt][e] = ok ? pos0 + i : -1;
+            row_col[nt][e] = qi;
+        }
+    }
+
+    for (int kt = 0; kt < n_tiles; ++kt) {
+        if (kt + 1 < n_tiles) {
+            load_tile(kt + 1, (kt + 1) & 1);
+            cp_async_commit();
+            cp_async_wait<1>();
+        } else {
+            cp_async_wait<0>();
+        }
+        __syncthreads();
+        const uint32_t sk = s_t + (kt & 1) * T_BYTES;
+        const int64_t j_tile = j_lo + (int64_t)kt * SC_BN;
+#pragma unroll
+        for (int mt = 0; mt < SC_BN / 16; ++mt) {
+            float c[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+                uint32_t a[4];
+                const int mi = lane >> 3;
+                ldsm_x4(a, sk + swz<CH>(mt * 16 + (mi & 1) * 8 + (lane & 7), 2 * ks + (mi >> 1)));
+                mma16816(c[0], a, qb[0][ks]);
+                mma16816(c[1], a, qb[1][ks]);
+            }
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                float pe[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) pe[e] = ex2(c[nt][e] * p.scale_log2 - l2[nt][e & 1]);
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {  // key rows lane/4 and lane/4 + 8
+                    const int64_t j = j_tile + mt * 16 + (lane >> 2) + 8 * r;
+                    float v0 = pe[2 * r], v1 = pe[2 * r + 1];
+                    if (G == 8) {
+                        float sum = v0 + v1;
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+                        if ((lane & 3) == 0 && j <= t_col[nt][0] - p.window && j < j_hi)
+                            scores[((int64_t)(b * p.hkv + g) * i_count + row_col[nt][0]) * sstride + j] = sum;
+                    } else if (G == 4) {
+                        float sum = v0 + v1;
+                        sum += __shfl_xor_sync(0xffffffffu, sum, 1);
+                        if ((lane & 1) == 0 && j <= t_col[nt][0] - p.window && j < j_hi)
+                            scores[((int64_t)(b * p.hkv + g) * i_count + row_col[nt][0]) * sstride + j] = sum;
+                    } else if (G == 2) {
+                        const float sum = v0 + v1;
+                        if (j <= t_col[nt][0] - p.window && j < j_hi)
+                            scores[((int64_t)(b * p.hkv + g) * i_count + row_col[nt][0]) * sstride + j] = sum;
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const float val = e ? v1 : v0;
+                            if (j <= t_col[nt][e] - p.window && j < j_hi)
+                                scores[((int64_t)(b * p.hkv + g) * i_count + row_col[nt][e]) * sstride + j] = val;
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// ---------------------------------------------------------------------------
+
+constexpr int TK_THREADS = 256;
+
+struct TopkSmem {
+    uint32_t hist[256];
+    uint32_t warp_tot[TK_THREADS / 32];
+    uint32_t warp_tot2[TK_THREADS / 32];
+    uint32_t digit, k_rem;
+};
+
+// exclusive prefix of `flag` over the block; returns the prefix, writes the block total
+__device__ __forceinline__ uint32_t block_excl_scan(bool flag, uint32_t* warp_tot, uint32_t& total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
+    const uint32_t in_warp = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(bal);
+    __syncthreads();
+    uint32_t before = 0, tot = 0;
+#pragma unroll
+    for (int w = 0; w < TK_THREADS / 32; ++w) {
+        const uint32_t x = warp_tot[w];
+        before += (w < warp) ? x : 0u;
+        tot += x;
+    }
+    total = tot;
+    return before + in_warp;
+}
+
+__global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const float* __restrict__ scores,
+                                                             int64_t sstride, int32_t* __restrict__ idx,
+                                                             int i_begin, int i_count) {
+    __shared__ TopkSmem sm;
+    const int tid = threadIdx.x;
+    const int qi = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int i = i_begin + qi;
+    const int64_t pos0 = seq_pos0(p, b, KID_TOPK);
+    const int64_t t = pos0 + i;
+    const int64_t n64 = t - p.window + 1;
+    const int n = n64 > 0 ? (int)n64 : 0;
+    int32_t* orow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
+    if (n <= p.topk) {
+        for (int r = tid; r < p.topk; r += TK_THREADS) orow[r] = r < n ? r : -1;
+        return;
+    }
+    const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + ((int64_t)(b * p.hkv + g) * i_count + qi) * sstride);
+
+    // radix select: find the key value of the topk-th largest
+    uint32_t prefix = 0, pmask = 0;
+    uint32_t k_rem = (uint32_t)p.topk;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        sm.hist[tid] = 0;
+        __syncthreads();
+        for (int j = tid; j < n; j += TK_THREADS) {
+            const uint32_t x = key[j];
+            if ((x & pmask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 255u], 1u);
+        }
+        __syncthreads();
+        if (tid < 32) {
+            // lane l owns bins 8*(31-l) .. 8*(31-l)+7, so lane order is descending digit
+            uint32_t bins[8], s = 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                bins[u] = sm.hist[8 * (31 - tid) + u];
+                s += bins[u];
+            }
+            uint32_t incl = s;  // inclusive prefix over lanes 0..tid (descending digits)
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (tid >= o) incl += y;
+            }
+            const uint32_t excl = incl - s;
+            if (excl < k_rem && k_rem <= incl) {
+                uint32_t above = excl;
+#pragma unroll
+                for (int u = 7; u >= 0; --u) {
+                    if (above + bins[u] >= k_rem) {
+                        sm.digit = 8 * (31 - tid) + u;
+                        sm.k_rem = k_rem - above;
+                        break;
+                    }
+                    above += bins[u];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sm.digit << shift;
+        pmask |= 255u << shift;
+        k_rem = sm.k_rem;
+        __syncthreads();
+    }
+    const uint32_t kth = prefix;
+    const uint32_t need_eq = k_rem;  // how many keys equal to kth are taken (lowest j first)
+
+    // ordered pass: keep keys > kth and the first need_eq keys == kth, ascending j
+    uint32_t eq_seen = 0, written = 0;
+    for (int base = 0; base < n; base += TK_THREADS) {
+        const int j = base + tid;
+        const uint32_t x = j < n ? key[j] : 0u;
+        const bool gt = j < n && x > kth;
+        const bool eq = j < n && x == kth;
+        uint32_t eq_tot;
+        const uint32_t eq_rank = block_excl_scan(eq, sm.warp_tot, eq_tot);
+        const bool take = gt || (eq && eq_seen + eq_rank < need_eq);
+        __syncthreads();
+        uint32_t take_tot;
+        const uint32_t pos = block_excl_scan(take, sm.warp_tot2, take_tot);
+        if (take) orow[written + pos] = j;
+        eq_seen += eq_tot;
+        written += take_tot;
+        __syncthreads();
+    }
+}
+
+template <int D, int G>
+cudaError_t launch_score_dg(const Problem& p, const void* q, const void* k, const float* lse, float* scores,
+                            int i_begin, int i_count, int64_t sstride, cudaStream_t st) {
+    constexpr int QPC = SC_WARPS * 2 * (8 / G);
+    constexpr int SMEM = 2 * SC_BN * D * 2;
+    auto kern = k2_score_kernel<D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    // split the key range so that every (query block, group, sequence) gets
+    // enough CTAs to fill the machine even for one query (decode)
+    const int qblocks = (i_count + QPC - 1) / QPC;
+    const int64_t t_hi = p.seq_len ? p.kv_len - 1 : p.q_pos0 + i_begin + i_count - 1;
+    const int64_t cand = t_hi - p.window + 1;
+    if (cand <= 0) return cudaSuccess;
+    const int64_t work_ctas = (int64_t)qblocks * p.hkv * p.B;
+    int64_t splits = (4 * 148 + work_ctas - 1) / work_ctas;
+    const int64_t max_splits = (cand + 4 * SC_BN - 1) / (4 * SC_BN);
+    if (splits > max_splits) splits = max_splits;
+    if (splits < 1) splits = 1;
+    if (splits > 65535 / p.B) splits = 65535 / p.B;
+    int64_t kps = (cand + splits - 1) / splits;
+    kps = (kps + SC_BN - 1) / SC_BN * SC_BN;
+    dim3 grid(qblocks, p.hkv, (unsigned)(p.B * splits));
+    prof_begin(KID_SCORE, st);
+    kern<<<grid, SC_WARPS * 32, SMEM, st>>>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, lse, scores,
+                                            i_begin, i_count, sstride, kps, (int)splits);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_score_d(const Problem& p, const void* q, const void* k, const float* lse, float* scores,
+                           int i_begin, int i_count, int64_t sstride, cudaStream_t st) {
+    switch (p.hq / p.hkv) {
+        case 1: return launch_score_dg<D, 1>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+        case 2: return launch_score_dg<D, 2>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+        case 4: return launch_score_dg<D, 4>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+        default: return launch_score_dg<D, 8>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_score(const Problem& p, const void* q, const void* k, const float* lse, float* scores,
+                         int i_begin, int i_count, int64_t sstride, cudaStream_t st) {
+    if (p.D == 64) return launch_score_d<64>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+    return launch_score_d<128>(p, q, k, lse, scores, i_begin, i_count, sstride, st);
+}
+
+cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, int32_t* idx, int i_begin,
+                        int i_count, cudaStream_t st) {
+    dim3 grid(i_count, p.hkv, p.B);
+    prof_begin(KID_TOPK, st);
+    k2_topk_kernel<<<grid, TK_THREADS, 0, st>>>(p, scores, sstride, idx, i_begin, i_count);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace hs2

@@ -1,0 +1,267 @@
+// k3_sparse_attn.cu -- K3: one sparse KV-reuse layer of HySparse2's
+// Cross-Decoder (xiawanshe.com report, section "两级KV共享": the following
+// sparse layers reuse the full layer's cache and token selection; section
+// "Token级选择": each attends to the selected older tokens plus the forced
+// most-recent window, all from the one shared cache).
+//
+// One CTA = one (sequence, query, KV group); its G heads share every gathered
+// K/V row.  The attended rows S = idx U window are listed in shared memory,
+// split over 4 warps in 16-row tiles, and gathered with 16-byte cp.async into
+// per-warp double-buffered, swizzled staging.  Per tile:
+//   S^T (16 keys x 8 heads) = K_tile Q^T      mma.sync m16n8k16, A = K rows
+//   P^T = 2^(S^T - m) per head column, online softmax over the warp's tiles
+//   O^T (D x 8 heads) += V_tile^T P^T         A = V^T via ldmatrix.trans,
+//                                             B = P^T via movmatrix.trans
+// The group's heads sit in the MMA's N = 8 columns (padded when G < 8), so no
+// tensor-core work is spent on padding rows of M.  The 4 warps' partial
+// (max, sum, O) are merged exactly at the end.
+#include "hs2_kernels.h"
+
+namespace hs2 {
+
+namespace {
+
+constexpr int SP_WARPS = 4;
+
+template <int D>
+struct K3Cfg {
+    static constexpr int CH = D / 8;
+    static constexpr int TILE_BYTES = 16 * D * 2;                 // one 16-row K (or V) tile
+    static constexpr int WARP_BYTES = 2 * 2 * TILE_BYTES;         // 2 stages x (K, V)
+    static constexpr int STAGE_BYTES = SP_WARPS * WARP_BYTES;
+    static constexpr int COMB_BYTES = SP_WARPS * (D * 8 + 16) * 4;  // per warp: O^T, m, l
+    static constexpr int FIXED = STAGE_BYTES > COMB_BYTES ? STAGE_BYTES : COMB_BYTES;
+};
+
+template <int D, int G>
+__global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, const __nv_bfloat16* __restrict__ q,
+                                                                   const __nv_bfloat16* __restrict__ k,
+                                                                   const __nv_bfloat16* __restrict__ v,
+                                                                   const int32_t* __restrict__ idx,
+                                                                   __nv_bfloat16* __restrict__ out) {
+    using C = K3Cfg<D>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    int32_t* list = reinterpret_cast<int32_t*>(smem + C::FIXED);
+    __shared__ int s_nsel;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int64_t pos0 = seq_pos0(p, b, KID_SPARSE);
+    const int64_t t = pos0 + i;
+    const int64_t w0 = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
+    const int nwin = (int)(t - w0 + 1);
+
+    // attended list: the selection's valid prefix, then the window
+    if (tid == 0) s_nsel = 0;
+    __syncthreads();
+    const int32_t* irow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
+    int cnt = 0;
+    for (int r = tid; r < p.topk; r += SP_WARPS * 32) {
+        const int32_t j = irow[r];
+        list[r] = j;
+        cnt += j >= 0;
+#ifdef HS2_CHECKED
+        const bool bad_range = j < -1 || (int64_t)j > t - p.window;
+        const bool bad_order = r > 0 && j >= 0 && (irow[r - 1] < 0 || irow[r - 1] >= j);
+        if (bad_range || bad_order) report_error(p.err, HS2_ERR_DEVICE_CHECK, KID_SPARSE, (uint32_t)i, (uint32_t)r);
+#endif
+    }
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 16);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 8);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
+    cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
+    if (lane == 0) atomicAdd(&s_nsel, cnt);
+    __syncthreads();
+    const int nsel = s_nsel;
+    for (int r = tid; r < nwin; r += SP_WARPS * 32) list[nsel + r] = (int32_t)(w0 + r);
+    __syncthreads();
+    const int n = nsel + nwin;
+    const int n_mt = (n + 15) / 16;
+
+    // Q^T B fragments: column = head (lane / 4) of the group, zero beyond G
+    uint32_t qb[D / 16][2];
+    {
+        const int hh = lane >> 2;
+        const bool ok = hh < G;
+        const __nv_bfloat16* qrow = q + ((int64_t)(b * p.hq + g * G + (ok ? hh : 0)) * p.nq + i) * D;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            const int d0 = ks * 16 + 2 * (lane & 3);
+            qb[ks][0] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0) : 0u;
+            qb[ks][1] = ok ? *reinterpret_cast<const uint32_t*>(qrow + d0 + 8) : 0u;
+        }
+    }
+
+    const __nv_bfloat16* kg = k + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
+    const __nv_bfloat16* vg = v + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
+    const uint32_t s_w = smem_u32(smem) + warp * C::WARP_BYTES;
+    auto load_tile = [&](int mt, int stage) {
+        const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES, sv = sk + C::TILE_BYTES;
+#pragma unroll
+        for (int it = 0; it < 16 * C::CH / 32; ++it) {
+            const int c = it * 32 + lane;
+            const int r = c / C::CH, ch = c % C::CH;
+            const int li = mt * 16 + r;
+            const int32_t j = li < n ? list[li] : -1;
+            const bool ok = j >= 0 && (int64_t)j <= t;
+            const int64_t off = (int64_t)(ok ? j : 0) * D + ch * 8;
+            cp_async16(sk + swz<C::CH>(r, ch), kg + off, ok ? 16 : 0);
+            cp_async16(sv + swz<C::CH>(r, ch), vg + off, ok ? 16 : 0);
+        }
+    };
+
+    float acc[D / 16][4];
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
+    float m_c[2] = {-INFINITY, -INFINITY}, l_c[2] = {0.f, 0.f};
+
+    int mt = warp, stage = 0;
+    if (mt < n_mt) load_tile(mt, 0);
+    cp_async_commit();
+    for (; mt < n_mt; mt += SP_WARPS, stage ^= 1) {
+        if (mt + SP_WARPS < n_mt) load_tile(mt + SP_WARPS, stage ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncwarp();
+        const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES, sv = sk + C::TILE_BYTES;
+
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+            uint32_t a[4];
+            const int mi = lane >> 3;
+            ldsm_x4(a, sk + swz<C::CH>((mi & 1) * 8 + (lane & 7), 2 * ks + (mi >> 1)));
+            mma16816(c, a, qb[ks]);
+        }
+        // rows lane/4 and lane/4 + 8 of the tile; columns 2*(lane%4) + {0, 1}
+        bool row_ok[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int li = mt * 16 + (lane >> 2) + 8 * r;
+            const int32_t j = li < n ? list[li] : -1;
+            row_ok[r] = j >= 0 && (int64_t)j <= t;
+        }
+        float s[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s[e] = row_ok[e >> 1] ? c[e] * p.scale_log2 : -INFINITY;
+        float alpha[2], m_use[2];
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            float mx = fmaxf(s[cc], s[cc + 2]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            const float m_new = fmaxf(m_c[cc], mx);
+            m_use[cc] = m_new == -INFINITY ? 0.f : m_new;
+            alpha[cc] = ex2(m_c[cc] - m_use[cc]);
+            m_c[cc] = m_new;
+            l_c[cc] *= alpha[cc];
+        }
+        float pr[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            pr[e] = ex2(s[e] - m_use[e & 1]);
+            l_c[e & 1] += pr[e];
+        }
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+            acc[dt][0] *= alpha[0];
+            acc[dt][1] *= alpha[1];
+            acc[dt][2] *= alpha[0];
+            acc[dt][3] *= alpha[1];
+        }
+        uint32_t pb[2];
+        pb[0] = movm_t(pack_bf16(pr[0], pr[1]));
+        pb[1] = movm_t(pack_bf16(pr[2], pr[3]));
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt) {
+            uint32_t a[4];
+            const int mi = lane >> 3;
+            ldsm_x4_t(a, sv + swz<C::CH>((mi >> 1) * 8 + (lane & 7), 2 * dt + (mi & 1)));
+            mma16816(acc[dt], a, pb);
+        }
+        __syncwarp();
+    }
+    cp_async_wait<0>();
+
+    // per-warp column sums, then the exact merge of the warps' partial states
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {
+        l_c[cc] += __shfl_xor_sync(0xffffffffu, l_c[cc], 4);
+        l_c[cc] += __shfl_xor_sync(0xffffffffu, l_c[cc], 8);
+        l_c[cc] += __shfl_xor_sync(0xffffffffu, l_c[cc], 16);
+    }
+    __syncthreads();  // staging is reused for the merge
+    float* comb = reinterpret_cast<float*>(smem);
+    float* ot = comb + warp * (D * 8 + 16);  // [D][8] then m[8], l[8]
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int d = dt * 16 + (lane >> 2) + 8 * (e >> 1);
+            const int col = 2 * (lane & 3) + (e & 1);
+            ot[d * 8 + col] = acc[dt][e];
+        }
+    }
+    if ((lane >> 2) == 0) {
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+            ot[D * 8 + 2 * lane + cc] = m_c[cc];
+            ot[D * 8 + 8 + 2 * lane + cc] = l_c[cc];
+        }
+    }
+    __syncthreads();
+    for (int u = tid; u < G * D; u += SP_WARPS * 32) {
+        const int hh = u / D, d = u % D;
+        float mm = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < SP_WARPS; ++w) mm = fmaxf(mm, comb[w * (D * 8 + 16) + D * 8 + hh]);
+        float num = 0.f, den = 0.f;
+#pragma unroll
+        for (int w = 0; w < SP_WARPS; ++w) {
+            const float* wb = comb + w * (D * 8 + 16);
+            const float sc = ex2(wb[D * 8 + hh] - mm);
+            num += sc * wb[d * 8 + hh];
+            den += sc * wb[D * 8 + 8 + hh];
+        }
+        out[((int64_t)(b * p.hq + g * G + hh) * p.nq + i) * D + d] = __float2bfloat16_rn(num / den);
+    }
+}
+
+template <int D, int G>
+cudaError_t launch_sparse_dg(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
+                             void* out, cudaStream_t st) {
+    using C = K3Cfg<D>;
+    const int smem = C::FIXED + (p.topk + p.window) * 4;
+    auto kern = k3_sparse_kernel<D, G>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    dim3 grid(p.nq, p.hkv, p.B);
+    prof_begin(KID_SPARSE, st);
+    kern<<<grid, SP_WARPS * 32, smem, st>>>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                           (const __nv_bfloat16*)v, idx, (__nv_bfloat16*)out);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_sparse_d(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
+                            void* out, cudaStream_t st) {
+    switch (p.hq / p.hkv) {
+        case 1: return launch_sparse_dg<D, 1>(p, q, k, v, idx, out, st);
+        case 2: return launch_sparse_dg<D, 2>(p, q, k, v, idx, out, st);
+        case 4: return launch_sparse_dg<D, 4>(p, q, k, v, idx, out, st);
+        default: return launch_sparse_dg<D, 8>(p, q, k, v, idx, out, st);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
+                          void* out, cudaStream_t st) {
+    if (p.D == 64) return launch_sparse_d<64>(p, q, k, v, idx, out, st);
+    return launch_sparse_d<128>(p, q, k, v, idx, out, st);
+}
+
+}  // namespace hs2

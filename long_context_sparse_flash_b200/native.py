@@ -1,0 +1,263 @@
+"""Thin ctypes binding of libhs2 (include/hs2.h), same names as the C ABI.
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are passed as device pointers (``tensor.data_ptr()``) and the
+current torch CUDA stream is passed as the library's stream unless one is given.
+There is no fallback: if ``libhs2.so`` is missing or a call fails, an exception
+is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Sequence
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+
+HS2_OK = 0
+STATUS = {0: "HS2_OK", 1: "HS2_ERR_INVALID_ARG", 2: "HS2_ERR_UNSUPPORTED", 3: "HS2_ERR_WORKSPACE",
+          4: "HS2_ERR_CUDA", 5: "HS2_ERR_DEVICE_CHECK", 6: "HS2_ERR_TIMEOUT"}
+HS2_ENTRY_FULL_SELECT, HS2_ENTRY_SPARSE, HS2_ENTRY_PREFILL, HS2_ENTRY_DECODE = 0, 1, 2, 3
+
+# every symbol include/hs2.h declares
+EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_sparse_attn",
+           "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
+           "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop")
+
+KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
+                6: "decode_combine", 7: "fused_attn_select"}
+
+
+class HS2Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class hs2_shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q", ctypes.c_int32), ("h_q", ctypes.c_int32),
+                ("h_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("topk", ctypes.c_int32), ("reserved", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
+                ("kv_len", ctypes.c_int64), ("softmax_scale", ctypes.c_float)]
+
+
+_libs = {}
+
+
+def lib_path(checked: bool = False) -> str:
+    return os.path.join(_PKG, "libhs2_checked.so" if checked else "libhs2.so")
+
+
+def load(checked: bool = False) -> ctypes.CDLL:
+    """Load (once) libhs2.so or libhs2_checked.so from the package directory."""
+    if checked in _libs:
+        return _libs[checked]
+    path = lib_path(checked)
+    if not os.path.exists(path):
+        raise RuntimeError(f"{os.path.basename(path)} is not built; run "
+                           "`python -m long_context_sparse_flash_b200.build`")
+    lib = ctypes.CDLL(path)
+    P, S, U64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint64
+    sh = ctypes.POINTER(hs2_shape)
+    lib.hs2_workspace_size.argtypes = [sh, ctypes.c_int]
+    lib.hs2_workspace_size.restype = S
+    lib.hs2_workspace_init.argtypes = [P, S, P]
+    lib.hs2_full_attn_select.argtypes = [sh, P, P, P, P, P, P, P, S, P]
+    lib.hs2_prefill_chunk.argtypes = [sh, P, P, P, P, P, P, P, S, P]
+    lib.hs2_decode.argtypes = [sh, P, P, P, P, P, P, P, P, S, P]
+    lib.hs2_sparse_attn.argtypes = [sh, P, P, P, P, P, P, S, P]
+    lib.hs2_decode_sparse.argtypes = [sh, P, P, P, P, P, P, P, S, P]
+    lib.hs2_get_device_status.argtypes = [P, P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.hs2_status_string.argtypes = [ctypes.c_int]
+    lib.hs2_status_string.restype = ctypes.c_char_p
+    lib.hs2_launch_count.argtypes = []
+    lib.hs2_launch_count.restype = U64
+    lib.hs2_is_checked_build.argtypes = []
+    lib.hs2_profile_start.argtypes = []
+    lib.hs2_profile_stop.argtypes = [ctypes.c_uint32, P, P]
+    for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
+                 "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
+                 "hs2_profile_start", "hs2_profile_stop"):
+        getattr(lib, name).restype = ctypes.c_int
+    _libs[checked] = lib
+    return lib
+
+
+def make_shape(batch, n_q, h_q, h_kv, head_dim, window, topk, q_pos0, kv_len,
+               softmax_scale: float = 0.0) -> hs2_shape:
+    return hs2_shape(int(batch), int(n_q), int(h_q), int(h_kv), int(head_dim), int(window), int(topk), 0,
+                     int(q_pos0), int(kv_len), float(softmax_scale))
+
+
+def shape_of(q: torch.Tensor, k: torch.Tensor, *, window: int, topk: int, q_pos0: int,
+             softmax_scale: float = 0.0) -> hs2_shape:
+    B, Hq, nq, D = q.shape
+    Bk, Hkv, N, Dk = k.shape
+    if (B, D) != (Bk, Dk):
+        raise ValueError("q and k disagree on batch or head_dim")
+    return make_shape(B, nq, Hq, Hkv, D, window, topk, q_pos0, N, softmax_scale)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhs2 takes device tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhs2 takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != HS2_OK:
+        raise HS2Error(rc, where)
+
+
+def hs2_workspace_size(shape: hs2_shape, entry: int, checked: bool = False) -> int:
+    return int(load(checked).hs2_workspace_size(ctypes.byref(shape), int(entry)))
+
+
+def alloc_workspace(shape: hs2_shape, entry: int, device="cuda", checked: bool = False,
+                    stream=None) -> torch.Tensor:
+    """Allocate (with torch) and initialise a workspace for `entry`."""
+    n = hs2_workspace_size(shape, entry, checked)
+    if n == 0:
+        raise HS2Error(1, "hs2_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    hs2_workspace_init(ws, stream=stream, checked=checked)
+    return ws
+
+
+def hs2_workspace_init(ws: torch.Tensor, stream=None, checked: bool = False) -> None:
+    _check(load(checked).hs2_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "hs2_workspace_init")
+
+
+def _ws(ws):
+    return (None, 0) if ws is None else (_ptr(ws), ws.numel() * ws.element_size())
+
+
+def hs2_full_attn_select(shape, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                              _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
+           "hs2_full_attn_select")
+
+
+def hs2_prefill_chunk(shape, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_prefill_chunk(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                           _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
+           "hs2_prefill_chunk")
+
+
+def hs2_decode(shape, kv_len_per_seq, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_decode(ctypes.byref(shape), _ptr(kv_len_per_seq), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(out), _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
+           "hs2_decode")
+
+
+def hs2_sparse_attn(shape, q, k, v, idx, out, ws=None, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_sparse_attn(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                         _ptr(out), wp, wn, _stream(stream)),
+           "hs2_sparse_attn")
+
+
+def hs2_decode_sparse(shape, kv_len_per_seq, q, k, v, idx, out, ws=None, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_decode_sparse(ctypes.byref(shape), _ptr(kv_len_per_seq), _ptr(q), _ptr(k), _ptr(v),
+                                           _ptr(idx), _ptr(out), wp, wn, _stream(stream)),
+           "hs2_decode_sparse")
+
+
+def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):
+    """Returns (status, [code, kernel, a, b]); synchronises the stream."""
+    info = (ctypes.c_uint32 * 4)()
+    rc = load(checked).hs2_get_device_status(_ptr(ws), _stream(stream), info)
+    return int(rc), list(info)
+
+
+def hs2_status_string(status: int, checked=False) -> str:
+    return load(checked).hs2_status_string(int(status)).decode()
+
+
+def hs2_launch_count(checked=False) -> int:
+    return int(load(checked).hs2_launch_count())
+
+
+def hs2_profile_start(checked=False) -> None:
+    _check(load(checked).hs2_profile_start(), "hs2_profile_start")
+
+
+def hs2_profile_stop(checked=False) -> dict:
+    """{kernel name: (total ms, launches)} recorded since hs2_profile_start."""
+    n = 8
+    ms = (ctypes.c_float * n)()
+    cnt = (ctypes.c_uint64 * n)()
+    _check(load(checked).hs2_profile_stop(n, ms, cnt), "hs2_profile_stop")
+    return {KERNEL_NAMES[u]: (float(ms[u]), int(cnt[u])) for u in range(1, n) if cnt[u]}
+
+
+def hs2_is_checked_build(checked=False) -> bool:
+    return bool(load(checked).hs2_is_checked_build())
+
+
+# ---------------------------------------------------------------------------
+# convenience: allocate outputs and run one layer (still one C-ABI call each)
+
+
+def full_attn_select(q, k, v, *, window: int, topk: int, q_pos0: int = 0, ws=None, stream=None,
+                     entry: str = "full", checked: bool = False):
+    """Allocate out/lse/idx and run hs2_full_attn_select (or hs2_prefill_chunk)."""
+    shape = shape_of(q, k, window=window, topk=topk, q_pos0=q_pos0)
+    e = HS2_ENTRY_PREFILL if entry == "prefill" else HS2_ENTRY_FULL_SELECT
+    if ws is None:
+        ws = alloc_workspace(shape, e, q.device, checked, stream)
+    out = torch.empty_like(q)
+    B, Hq, nq, D = q.shape
+    lse = torch.empty(B, Hq, nq, dtype=torch.float32, device=q.device)
+    idx = torch.empty(B, k.shape[1], nq, topk, dtype=torch.int32, device=q.device)
+    fn = hs2_prefill_chunk if entry == "prefill" else hs2_full_attn_select
+    fn(shape, q, k, v, out, lse, idx, ws, stream, checked)
+    return out, lse, idx
+
+
+def decode(q, k, v, *, window: int, topk: int, kv_len_per_seq=None, ws=None, stream=None,
+           checked: bool = False):
+    shape = shape_of(q, k, window=window, topk=topk, q_pos0=k.shape[2] - 1)
+    if ws is None:
+        ws = alloc_workspace(shape, HS2_ENTRY_DECODE, q.device, checked, stream)
+    out = torch.empty_like(q)
+    B, Hq, nq, D = q.shape
+    lse = torch.empty(B, Hq, nq, dtype=torch.float32, device=q.device)
+    idx = torch.empty(B, k.shape[1], nq, topk, dtype=torch.int32, device=q.device)
+    hs2_decode(shape, kv_len_per_seq, q, k, v, out, lse, idx, ws, stream, checked)
+    return out, lse, idx
+
+
+def sparse_attn(q, k, v, idx, *, window: int, q_pos0: int = 0, stream=None, ws=None,
+                checked: bool = False):
+    """Run one sparse KV-reuse layer (queries at q_pos0 + i)."""
+    shape = shape_of(q, k, window=window, topk=idx.shape[-1], q_pos0=q_pos0)
+    out = torch.empty_like(q)
+    hs2_sparse_attn(shape, q, k, v, idx, out, ws, stream, checked)
+    return out
+
+
+def decode_sparse(q, k, v, idx, *, window: int, kv_len_per_seq=None, stream=None, ws=None,
+                  checked: bool = False):
+    """Run one sparse KV-reuse layer for a decode step (one query per sequence)."""
+    shape = shape_of(q, k, window=window, topk=idx.shape[-1], q_pos0=k.shape[2] - 1)
+    out = torch.empty_like(q)
+    hs2_decode_sparse(shape, kv_len_per_seq, q, k, v, idx, out, ws, stream, checked)
+    return out

@@ -1,0 +1,128 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every symbol include/hs2.h declares, sizes workspaces, and rejects invalid
+arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sparse_flash_b200 import native as nv
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hs2.h")
+
+# a fake, 256-byte-aligned device address: never dereferenced by host validation
+FAKE = ctypes.c_void_p(1 << 40)
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hs2_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module", params=[False, True], ids=["release", "checked"])
+def lib(request):
+    return request.param, nv.load(request.param)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    checked, L = lib
+    syms = declared_symbols()
+    assert len(syms) >= 10
+    for s in syms:
+        assert hasattr(L, s), s
+    assert set(syms) == set(nv.EXPORTS)
+    assert nv.hs2_is_checked_build(checked) == checked
+
+
+def shape(**kw):
+    base = dict(batch=1, n_q=256, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024, q_pos0=0,
+                kv_len=256)
+    base.update(kw)
+    return nv.make_shape(**base)
+
+
+def test_workspace_size_rules():
+    assert nv.hs2_workspace_size(shape(), nv.HS2_ENTRY_SPARSE) == 256
+    # no row has more than topk candidates: header only
+    assert nv.hs2_workspace_size(shape(), nv.HS2_ENTRY_FULL_SELECT) == 256
+    s = shape(n_q=4096, kv_len=4096)
+    n = nv.hs2_workspace_size(s, nv.HS2_ENTRY_FULL_SELECT)
+    cand = 4096 - 128
+    assert n == 256 + 4096 * 4 * ((cand + 3) // 4 * 4) * 4
+    # invalid shapes size to 0
+    assert nv.hs2_workspace_size(shape(h_q=30), nv.HS2_ENTRY_FULL_SELECT) == 0
+    assert nv.hs2_workspace_size(shape(q_pos0=1), nv.HS2_ENTRY_FULL_SELECT) == 0
+    assert nv.hs2_workspace_size(shape(), 99) == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(h_q=30), 1),                                      # h_q % h_kv != 0
+    (dict(h_q=48, h_kv=4), 2),                              # G = 12 unsupported
+    (dict(head_dim=96), 2),
+    (dict(window=0), 1),
+    (dict(window=2048), 2),
+    (dict(topk=-1), 1),
+    (dict(topk=4096), 2),
+    (dict(q_pos0=10), 1),                                   # q_pos0 + n_q > kv_len
+    (dict(n_q=-1), 1),
+    (dict(batch=70000), 2),
+])
+def test_invalid_shapes_rejected_without_launch(kw, status):
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    s = shape(**kw)
+    rc = L.hs2_full_attn_select(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1 << 30, None)
+    assert rc == status
+    rc = L.hs2_sparse_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None)
+    assert rc == status
+    assert nv.hs2_launch_count() == before
+
+
+def test_pointer_and_workspace_checks():
+    L = nv.load()
+    s = shape(n_q=4096, kv_len=4096)
+    need = nv.hs2_workspace_size(s, nv.HS2_ENTRY_FULL_SELECT)
+    args = [FAKE] * 7
+    assert L.hs2_full_attn_select(None, *args, need, None) == 1
+    assert L.hs2_full_attn_select(ctypes.byref(s), None, *args[1:], need, None) == 1
+    assert L.hs2_full_attn_select(ctypes.byref(s), *args, need - 1, None) == 3
+    mis = ctypes.c_void_p((1 << 40) + 8)
+    assert L.hs2_full_attn_select(ctypes.byref(s), mis, *args[1:], need, None) == 1
+    bad = shape()
+    bad.reserved = 1
+    assert L.hs2_full_attn_select(ctypes.byref(bad), *args, need, None) == 1
+    # decode needs n_q == 1
+    assert L.hs2_decode(ctypes.byref(s), None, *args, need, None) == 1
+    # sparse: ws_bytes without ws
+    assert L.hs2_sparse_attn(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, None, 64, None) == 1
+    # nan scale
+    s2 = shape(n_q=4096, kv_len=4096, softmax_scale=float("nan"))
+    assert L.hs2_full_attn_select(ctypes.byref(s2), *args, need, None) == 1
+
+
+def test_empty_calls_are_noops():
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    for kw in (dict(batch=0), dict(n_q=0)):
+        s = shape(**kw)
+        assert L.hs2_full_attn_select(ctypes.byref(s), None, None, None, None, None, None, None, 0, None) == 0
+        assert L.hs2_sparse_attn(ctypes.byref(s), None, None, None, None, None, None, 0, None) == 0
+        d = shape(**kw, **({} if "n_q" in kw else {"n_q": 1}))
+        assert L.hs2_decode(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None) == 0
+    assert nv.hs2_launch_count() == before
+
+
+def test_status_strings():
+    for code in range(7):
+        assert nv.hs2_status_string(code) != "unknown status"
+    assert nv.hs2_status_string(42) == "unknown status"
+
+
+def test_binding_refuses_host_tensors():
+    import torch
+    q = torch.zeros(1, 8, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        nv.sparse_attn(q, q[:, :2], q[:, :2], torch.zeros(1, 2, 4, 1, dtype=torch.int32), window=2)

@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded bf16 inputs.  Small cases are checked on every row; the full-size
+workloads on stratified samples (window / top-k boundary rows plus seeded
+random rows) and on properties that hold for every row."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from long_context_sparse_flash_b200 import native as nv
+from long_context_sparse_flash_b200 import workloads as wl
+from tests import parity as P
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from long_context_sparse_flash_b200 import build
+    build.build()
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    nv.load()
+    nv.load(True)
+
+
+def test_tiny_every_row():
+    w = wl.WORKLOADS["tiny"]
+    inp = wl.make_inputs(w, "cuda")
+    before = nv.hs2_launch_count()
+    gpu = P.run_gpu(w, inp)
+    assert nv.hs2_launch_count() > before  # the CUDA kernels ran
+    res = P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+    print("tiny", {k: v for k, v in res.items() if k != "oracle"})
+
+
+def test_prefill_entry_matches_full_select():
+    w = wl.WORKLOADS["tiny"]
+    inp = wl.make_inputs(w, "cuda", with_sparse=False)
+    a = nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk, entry="full")
+    b = nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk, entry="prefill")
+    torch.cuda.synchronize()
+    assert torch.equal(a[2], b[2])
+    P.assert_close(P.to_f64(a[0]), P.to_f64(b[0]), "prefill vs full out")
+
+
+RAGGED = [
+    # name, kwargs for workloads.custom
+    ("g8_d128_tail", dict(n_q=200, h_q=16, h_kv=2, head_dim=128, window=128, topk=64)),
+    ("g4_d64_chunk", dict(n_q=333, q_pos0=700, h_q=8, h_kv=2, head_dim=64, window=32, topk=100)),
+    ("g2_d64_extra_cache", dict(n_q=130, q_pos0=50, kv_len=400, h_q=4, h_kv=2, head_dim=64, window=16, topk=20)),
+    ("g1_d128", dict(n_q=257, h_q=2, h_kv=2, head_dim=128, window=8, topk=33)),
+    ("window1_topk_large", dict(n_q=190, h_q=8, h_kv=1, head_dim=64, window=1, topk=300)),
+    ("topk0", dict(n_q=160, h_q=8, h_kv=1, head_dim=128, window=40, topk=0)),
+    ("batch3", dict(batch=3, n_q=150, q_pos0=100, h_q=8, h_kv=1, head_dim=64, window=64, topk=48)),
+    ("topk_2048", dict(n_q=64, q_pos0=3000, h_q=16, h_kv=2, head_dim=64, window=128, topk=2048)),
+    ("window1024", dict(n_q=96, q_pos0=1500, h_q=8, h_kv=1, head_dim=128, window=1024, topk=256)),
+]
+
+
+@pytest.mark.parametrize("name,kw", RAGGED, ids=[r[0] for r in RAGGED])
+def test_ragged_shapes_every_row(name, kw):
+    w = wl.custom(name, n_sparse=2, seed=7, **kw)
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    for b in range(w.batch):
+        P.compare_rows(w, inp, gpu, b, np.arange(w.n_q))
+
+
+def test_sparse_kernel_with_oracle_selection():
+    """K3 alone, fed the oracle's idx row by row (one-query calls)."""
+    w = wl.custom("k3_oracle_idx", n_q=700, h_q=16, h_kv=2, head_dim=128, window=128, topk=128, seed=3)
+    inp = wl.make_inputs(w, "cuda")
+    rows = np.array([0, 127, 128, 129, 255, 256, 257, 400, 699])
+    kb, vb = P.bits(inp["k"][0]), P.bits(inp["v"][0])
+    qb = np.ascontiguousarray(P.bits(inp["q"][0][:, rows]).transpose(1, 0, 2))
+    ores = oracle.full_select(qb, rows, kb, vb, window=w.window, topk=w.topk)
+    qs = inp["q_sparse"][0]
+    qsb = np.ascontiguousarray(P.bits(qs[0][:, rows]).transpose(1, 0, 2))
+    ref = oracle.sparse(qsb, rows, kb, vb, ores["idx"], window=w.window)
+    for r, i in enumerate(rows):
+        q1 = qs[:, :, i:i + 1].contiguous()
+        idx1 = torch.as_tensor(ores["idx"][r][None, :, None, :], device="cuda").contiguous()
+        o = nv.sparse_attn(q1, inp["k"], inp["v"], idx1, window=w.window, q_pos0=int(i))
+        P.assert_close(P.to_f64(o[0, :, 0]), ref[r], f"K3 row {i}")
+
+
+def test_prefill_32k_sampled():
+    w = wl.WORKLOADS["prefill_32k"]
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    rows = wl.stratified_rows(w, 12)
+    res = P.compare_rows(w, inp, gpu, 0, rows)
+    print("32k", res["idx"], res["out_err"], res["sparse_err"])
+    _row_properties(gpu["idx"], w)
+
+
+def _row_properties(idx: torch.Tensor, w: wl.Workload, seq_len=None):
+    """Every row of a full-size call: size min(K, t-W+1), strictly ascending,
+    inside [0, t-W], -1 padded (checked on the device)."""
+    B, Hkv, nq, K = idx.shape
+    if seq_len is None:
+        t = torch.arange(w.q_pos0, w.q_pos0 + nq, device=idx.device).view(1, 1, nq, 1).expand(B, 1, nq, 1)
+    else:
+        t = (seq_len - 1).view(B, 1, 1, 1)
+    n_sel = torch.clamp(t - w.window + 1, min=0).clamp(max=K)
+    pos = torch.arange(K, device=idx.device).view(1, 1, 1, K)
+    valid = pos < n_sel
+    assert torch.all(torch.where(valid, idx >= 0, idx == -1))
+    assert torch.all(torch.where(valid, idx <= t - w.window, True))
+    if K > 1:
+        d = idx[..., 1:] - idx[..., :-1]
+        assert torch.all(torch.where(valid[..., 1:], d > 0, True))
+
+
+def test_chunk_256k_sampled():
+    w = wl.WORKLOADS["chunk_256k"]
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    rows = wl.stratified_rows(w, 8)
+    res = P.compare_rows(w, inp, gpu, 0, rows)
+    print("256k", res["idx"], res["out_err"], res["sparse_err"])
+    _row_properties(gpu["idx"], w)
+
+
+def test_decode_128k_sampled():
+    w = wl.WORKLOADS["decode_128k"]
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    t = np.array([w.kv_len - 1])
+    for b in (0, 1, 17, 40, 63):
+        P.compare_rows(w, inp, gpu, b, np.array([0]), ts=t)
+    _row_properties(gpu["idx"], w)
+
+
+def test_decode_ragged_lengths():
+    w = wl.custom("decode_ragged", batch=5, n_q=1, q_pos0=4999, kv_len=5000, h_q=32, h_kv=4, head_dim=128,
+                  window=128, topk=1024, n_sparse=2, decode=True, seed=9)
+    inp = wl.make_inputs(w, "cuda")
+    lens = torch.tensor([5000, 1, 128, 1153, 3001], dtype=torch.int64, device="cuda")
+    gpu = P.run_gpu(w, inp, seq_len=lens)
+    for b, ln in enumerate(lens.tolist()):
+        P.compare_rows(w, inp, gpu, b, np.array([0]), ts=np.array([ln - 1]))
+    _row_properties(gpu["idx"], w, seq_len=lens)
+
+
+def test_chunk_1m_sampled():
+    w = wl.WORKLOADS["chunk_1m"]
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    rows = wl.stratified_rows(w, 4)
+    res = P.compare_rows(w, inp, gpu, 0, rows)
+    print("1m chunk", res["idx"], res["out_err"], res["sparse_err"])
+    _row_properties(gpu["idx"], w)
+
+
+def test_decode_1m_every_sequence():
+    w = wl.WORKLOADS["decode_1m"]
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    t = np.array([w.kv_len - 1])
+    for b in range(w.batch):
+        P.compare_rows(w, inp, gpu, b, np.array([0]), ts=t)
+    _row_properties(gpu["idx"], w)
+
+
+def test_checked_build_reports_invalid_selection():
+    """A selection row that breaks the contract (an index inside the window) is
+    reported through the error word; the kernel skips nothing out of bounds."""
+    w = wl.custom("bad_idx", n_q=64, q_pos0=500, h_q=8, h_kv=1, head_dim=64, window=32, topk=16, seed=2)
+    inp = wl.make_inputs(w, "cuda")
+    _, _, idx = nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk,
+                                    q_pos0=w.q_pos0, checked=True)
+    shape = nv.shape_of(inp["q"], inp["k"], window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_SPARSE, checked=True)
+    out = torch.empty_like(inp["q"])
+    nv.hs2_sparse_attn(shape, inp["q"], inp["k"], inp["v"], idx, out, ws, checked=True)
+    rc, info = nv.hs2_get_device_status(ws, checked=True)
+    assert rc == nv.HS2_OK, (rc, info)
+    bad = idx.clone()
+    bad[0, 0, 5, 3] = w.q_pos0 + 5  # the query itself: inside the window
+    nv.hs2_sparse_attn(shape, inp["q"], inp["k"], inp["v"], bad, out, ws, checked=True)
+    rc, info = nv.hs2_get_device_status(ws, checked=True)
+    assert rc == 5 and info[1] == 4, (rc, info)  # HS2_ERR_DEVICE_CHECK from the sparse kernel
+    rc, info = nv.hs2_get_device_status(ws, checked=True)
+    assert rc == nv.HS2_OK  # reading clears the word
+
+
+def test_empty_call_launches_nothing():
+    q = torch.zeros(1, 8, 0, 64, dtype=torch.bfloat16, device="cuda")
+    k = torch.zeros(1, 2, 16, 64, dtype=torch.bfloat16, device="cuda")
+    before = nv.hs2_launch_count()
+    out, lse, idx = nv.full_attn_select(q, k, k, window=4, topk=4, q_pos0=0)
+    assert nv.hs2_launch_count() == before
