@@ -25,6 +25,10 @@ void count_launch(int n = 1);
 void prof_begin(uint32_t kid, cudaStream_t st);
 void prof_end(cudaStream_t st);
 
+// K1 on tcgen05/TMEM/TMA (prefill-shaped calls: 128-row query tiles).
+cudaError_t launch_full_tc(const Problem& p, const void* q, const void* k, const void* v, void* out,
+                           float* lse, cudaStream_t st);
+
 // K1: causal full attention + LSE for every query of the call.
 cudaError_t launch_full(const Problem& p, const void* q, const void* k, const void* v, void* out,
                         float* lse, cudaStream_t st);

@@ -54,7 +54,8 @@ enum : int {
     B_SEMPTY = B_SFULL + 2,
     B_PFULL = B_SEMPTY + 2,
     B_ODONE = B_PFULL + 1,
-    B_COUNT = B_ODONE + 1,
+    B_DRAIN = B_ODONE + 1,     // the MMA thread's final commit
+    B_COUNT = B_DRAIN + 1,
 };
 
 template <int D>
@@ -120,9 +121,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k1_full_tc_kernel(const __grid_
             }
             // drain: every issued load has landed before the CTA can exit
             if (ab->flag) {
+                tc::Abort none{0};
+                tc::mbar_wait(bar(B_Q), 0, &none, nullptr, 0, 0);
                 for (int j = (issued > TC_NS ? issued - TC_NS : 0); j < issued; ++j) {
                     const int s = j % TC_NS;
-                    tc::Abort none{0};
                     tc::mbar_wait(bar(B_KFULL + s), (j / TC_NS) & 1, &none, nullptr, 0, 0);
                     tc::mbar_wait(bar(B_VFULL + s), (j / TC_NS) & 1, &none, nullptr, 0, 0);
                 }
@@ -167,8 +169,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k1_full_tc_kernel(const __grid_
                 }
             }
             // every issued MMA completes before TMEM is released
+            tc::mma_commit(bar(B_DRAIN));
             tc::Abort none{0};
-            tc::mma_commit(bar(B_COUNT - 1 + 0));  // B_ODONE is the last slot; one more arrival is harmless
+            tc::mbar_wait(bar(B_DRAIN), 0, &none, nullptr, 0, 0);
         }
     } else {
         // ------------------------------------------------------------ softmax (warps 0-3)
@@ -291,11 +294,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k1_full_tc_kernel(const __grid_
     tc::fence_before_sync();
     __syncthreads();
     if (warp == 5) {
-        // the MMA thread's last commit: wait for it (bounded) before freeing TMEM
-        if (!ab->flag) {
-            tc::Abort none{0};
-            // completion of the final commit is observed through B_ODONE's phase
-        }
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TC_TMEM_COLS);
     }
