@@ -146,6 +146,40 @@ hs2_status hs2_decode_sparse(const hs2_shape* shape, const int64_t* kv_len_per_s
                              const void* k, const void* v, const int32_t* idx, void* out, void* ws,
                              size_t ws_bytes, hs2_stream_t stream);
 
+/* Bytes of the static scratch array behind hs2_full_attn_select_static. */
+#define HS2_STATIC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* hs2_full_attn_select for callers that cannot allocate device memory at the
+ * point where they run the layer: a process whose device memory is a
+ * pre-sized pool it may not grow, a host runtime or plugin that hands over
+ * only the input and output buffers, or a step that must not synchronise the
+ * device (cudaMalloc and cudaFree may).  The HySparse2 pages have no
+ * counterpart for it: it is a deployment convenience, not part of the method.
+ *
+ * Arguments and outputs are those of hs2_full_attn_select without the
+ * workspace.  Instead of a caller workspace it uses one static device array
+ * of HS2_STATIC_SCRATCH_BYTES inside the library; every GPU that loads the
+ * library holds that array until the process exits.  Calls no allocation
+ * routine.  Shapes whose workspace (hs2_workspace_size(shape,
+ * HS2_ENTRY_FULL_SELECT)) exceeds HS2_STATIC_SCRATCH_BYTES are rejected with
+ * HS2_ERR_WORKSPACE before anything is launched; invalid shapes get the
+ * status hs2_full_attn_select would give.
+ *
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call clears the error-word header of the
+ * array on `stream` (the array keeps the previous call's contents), so a
+ * device-side check failure of this entry point cannot be read back.  All
+ * calls on a device share the one array: calls that overlap on the GPU (other
+ * streams, or other host threads without ordering) race on it and corrupt
+ * each other's selections; order them on one stream or serialise them. */
+hs2_status hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const void* k,
+                                       const void* v, void* out, float* lse, int32_t* idx,
+                                       hs2_stream_t stream);
+
+/* HS2_STATIC_SCRATCH_BYTES, for callers that load the library dynamically. */
+size_t hs2_static_scratch_bytes(void);
+
 /* Synchronise `stream`, read and clear the workspace error word.  Returns
  * HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA).  If
  * `info` is non-NULL it receives 4 words: code, kernel id, and two values

@@ -25,7 +25,8 @@ HS2_ENTRY_FULL_SELECT, HS2_ENTRY_SPARSE, HS2_ENTRY_PREFILL, HS2_ENTRY_DECODE = 0
 # every symbol include/hs2.h declares
 EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_sparse_attn",
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
-           "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop")
+           "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
+           "hs2_full_attn_select_static", "hs2_static_scratch_bytes")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select"}
@@ -78,9 +79,12 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_is_checked_build.argtypes = []
     lib.hs2_profile_start.argtypes = []
     lib.hs2_profile_stop.argtypes = [ctypes.c_uint32, P, P]
+    lib.hs2_full_attn_select_static.argtypes = [sh, P, P, P, P, P, P, P]
+    lib.hs2_static_scratch_bytes.argtypes = []
+    lib.hs2_static_scratch_bytes.restype = S
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
-                 "hs2_profile_start", "hs2_profile_stop"):
+                 "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -178,6 +182,13 @@ def hs2_decode_sparse(shape, kv_len_per_seq, q, k, v, idx, out, ws=None, stream=
     _check(load(checked).hs2_decode_sparse(ctypes.byref(shape), _ptr(kv_len_per_seq), _ptr(q), _ptr(k), _ptr(v),
                                            _ptr(idx), _ptr(out), wp, wn, _stream(stream)),
            "hs2_decode_sparse")
+
+
+def hs2_full_attn_select_static(shape, q, k, v, out, lse, idx, stream=None, checked=False) -> None:
+    """hs2_full_attn_select without a workspace (library-internal static scratch)."""
+    _check(load(checked).hs2_full_attn_select_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                                     _ptr(lse), _ptr(idx), _stream(stream)),
+           "hs2_full_attn_select_static")
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):
