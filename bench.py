@@ -54,22 +54,26 @@ def peaks():
 
 
 def kernel_work(w: wl.Workload):
+    """Algorithmic work of each kernel per call (all sequences of the call)."""
     f = wl.flops_and_bytes(w)
-    D, Hq, Hk = w.head_dim, w.h_q, w.h_kv
+    Hq = w.h_q
     n_rows = w.batch * w.n_q
     cand = f["cand"]  # sum over (sequence, query, KV head) of candidate counts
-    return {
+    work = {
         # dense causal contraction: QK^T and PV over the causal pairs
         "full_attn": dict(bound="tensor", flops=f["full_flops"]),
-        "fused_attn_select": dict(bound="tensor", flops=f["full_flops"] + f["select_qk_flops"]),
         "decode_attn": dict(bound="hbm", bytes=f["kv_bytes"] + 2 * f["q_bytes"] + 4 * n_rows * Hq),
-        # QK^T recompute over the candidates of every query
-        "select_score": dict(bound="tensor", flops=f["select_qk_flops"]),
-        # read every stored score once, write idx
-        "select_topk": dict(bound="hbm", bytes=4.0 * cand + f["idx_bytes"]),
         # gathered K/V rows + q + out + idx, per layer
         "sparse_attn": dict(bound="hbm", bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
     }
+    if w.decode:
+        # decode: every candidate's score is computed (QK^T) and stored, then a radix top-k reads it
+        work["select_score"] = dict(bound="tensor", flops=f["select_qk_flops"])
+        work["select_topk"] = dict(bound="hbm", bytes=4.0 * cand + f["idx_bytes"])
+    else:
+        # prefill: the filtered sweep recomputes QK^T over every candidate of every query
+        work["select_filter"] = dict(bound="tensor", flops=f["select_qk_flops"])
+    return work
 
 
 def source_sha(path: str) -> str:
@@ -77,8 +81,8 @@ def source_sha(path: str) -> str:
 
 
 KERNEL_SOURCE = {
-    "full_attn": "k1_full_attn.cu", "select_score": "k2_select.cu", "select_topk": "k2_select.cu",
-    "sparse_attn": "k3_sparse_attn.cu",
+    "full_attn": "k1_full_tc.cu", "select_score": "k2_select.cu", "select_topk": "k2_select.cu",
+    "select_filter": "k2_select_tc.cu", "sparse_attn": "k3_sparse_attn.cu",
 }
 
 
@@ -296,6 +300,7 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
     per = {}
     for name, (ms, launches) in prof.items():
         if name not in work or ms <= 0:
+            per[name] = dict(ms=ms / K, launches=launches // K if K else launches)
             continue
         wk = work[name]
         calls = K * (w.n_sparse if name == "sparse_attn" else 1)
@@ -309,7 +314,7 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
                          achieved=round(achieved, 2), peak=peak, unit=unit, frac=round(achieved / peak, 4))
     if not per:
         return None, per
-    top = max(per, key=lambda n: per[n]["ms"])
+    top = max((n for n in per if "bound" in per[n]), key=lambda n: per[n]["ms"])
     p = per[top]
     launches_total = prof[top][1]
     traffic = dram_traffic(top, w.name)

@@ -199,7 +199,8 @@ uint64_t hs2_launch_count(void);
  * the summed event time in ms (total_ms[u]) and the launch count
  * (launches[u]); either array may be NULL.  Kernel ids: 1 full attention,
  * 2 selection scores, 3 top-k select, 4 sparse attention, 5 decode attention
- * partials, 6 decode combine, 7 fused attention + selection. */
+ * partials, 6 decode combine, 7 fused attention + selection, 8 selection
+ * threshold estimate, 9 filtered selection sweep, 10 selection retry. */
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 

@@ -98,19 +98,36 @@ hs2_status check_shape(const hs2_shape* s, Problem* p) {
     return HS2_OK;
 }
 
-// Stored-score layout of the selection pass: queries are processed in chunks
-// of `chunk` rows; each (sequence, group, query) row holds `sstride` floats.
+// Selection pass plan.  Prefill-shaped calls run the tcgen05 selection
+// (sample, threshold, filtered sweep, retry) over chunks of `chunk` queries;
+// decode-shaped calls store every candidate's score (sstride floats per row)
+// and run the radix top-k over them.
 struct ScorePlan {
+    bool tc = false;
     int64_t sstride = 0;
+    int64_t n_cand_max = 0;
     int chunk = 0;
     size_t bytes = 0;
 };
+
+constexpr size_t kSampleBudget = size_t(1) << 30;  // bytes of per-row selection state per chunk
 
 ScorePlan score_plan(const Problem& p, bool decode) {
     ScorePlan sp;
     const int64_t t_hi = decode ? p.kv_len - 1 : p.q_pos0 + p.nq - 1;
     const int64_t cand = t_hi - p.window + 1;
     if (cand <= p.topk || p.nq == 0 || p.B == 0 || p.topk == 0) return sp;  // every row takes all candidates
+    sp.n_cand_max = cand;
+    if (!decode && p.nq >= 16) {
+        sp.tc = true;
+        const size_t per_q = (size_t)p.B * p.hkv * (1024 * 4 + 12);
+        int64_t chunk = (int64_t)(kSampleBudget / per_q) / 32 * 32;
+        if (chunk < 32) chunk = 32;
+        if (chunk > p.nq) chunk = p.nq;
+        sp.chunk = (int)chunk;
+        sp.bytes = select_tc_scratch_bytes(p, sp.chunk, cand);
+        return sp;
+    }
     sp.sstride = (cand + 3) / 4 * 4;
     const size_t per_q = (size_t)p.B * p.hkv * sp.sstride * 4;
     int64_t chunk = (int64_t)(kScoreBudget / per_q);
@@ -149,6 +166,11 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
     const int chunk = sp.chunk > 0 ? sp.chunk : p.nq;
     for (int i0 = 0; i0 < p.nq; i0 += chunk) {
         const int cnt = p.nq - i0 < chunk ? p.nq - i0 : chunk;
+        if (sp.tc) {
+            e = launch_select_tc(p, q, k, lse, idx, scores, i0, cnt, sp.n_cand_max, st);
+            if (e != cudaSuccess) return HS2_ERR_CUDA;
+            continue;
+        }
         if (sp.sstride > 0) {
             e = launch_score(p, q, k, lse, scores, i0, cnt, sp.sstride, st);
             if (e != cudaSuccess) return HS2_ERR_CUDA;

@@ -30,6 +30,9 @@ enum KernelId : uint32_t {
     KID_DECODE = 5,
     KID_COMBINE = 6,
     KID_FUSED = 7,
+    KID_THRESH = 8,
+    KID_FILTER = 9,
+    KID_RETRY = 10,
 };
 
 __device__ __forceinline__ void report_error(WsHeader* h, uint32_t code, uint32_t kid, uint32_t a,

@@ -43,6 +43,12 @@ cudaError_t launch_score(const Problem& p, const void* q, const void* k, const f
 cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, int32_t* idx,
                         int i_begin, int i_count, cudaStream_t st);
 
+// K2 on tcgen05 for prefill-shaped calls: sampled threshold, filtered sweep
+// with on-chip survivor lists, exact final top-k, retry of underestimated rows.
+size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
+cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
+                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st);
+
 // K3: one sparse KV-reuse layer.
 cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* out, cudaStream_t st);

@@ -23,6 +23,35 @@
 
 namespace hs2 {
 
+// ---------------------------------------------------------------------------
+// host
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// [z][y][x] bf16 tensor, x contiguous (= D); box 64 x 128 x 1, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {x, y, z};
+    cuuint64_t strides[2] = {x * 2, x * y * 2};
+    cuuint32_t box[3] = {64, 128, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 namespace {
 
 constexpr int TC_BM = 128;   // query rows per CTA
@@ -297,35 +326,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1) k1_full_tc_kernel(const __grid_
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, TC_TMEM_COLS);
     }
-}
-
-// ---------------------------------------------------------------------------
-// host
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        cudaDriverEntryPointQueryResult q;
-        void* f = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }
-    return fn;
-}
-
-// [z][y][x] bf16 tensor, x contiguous (= D); box 64 x 128 x 1, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z) {
-    auto fn = encode_fn();
-    if (fn == nullptr) return false;
-    cuuint64_t dims[3] = {x, y, z};
-    cuuint64_t strides[2] = {x * 2, x * y * 2};
-    cuuint32_t box[3] = {64, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
 }
 
 template <int D>

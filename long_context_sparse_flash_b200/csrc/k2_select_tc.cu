@@ -1,0 +1,655 @@
+// k2_select_tc.cu -- K2 on the tensor cores: HySparse2's token-level
+// selection (xiawanshe.com report, section "Token级选择": per token, the 1024
+// best older tokens beside the forced 128-token window; davidyin.dev notes,
+// section "HySparse2 的解法": no separate indexer, so the score comes from the
+// full-attention layer's own probabilities).
+//
+//   score_{g,j}(t) = sum_{h in g} 2^(s2_{h,j} - lse2_h),  s2 = scale*log2(e)*<q_h, k_j>
+//
+// One CTA = one KV group x 32 consecutive queries (N = 32*G columns ordered
+// (query, head)); it sweeps the candidate keys in 128-key tiles:
+//   S^T (TMEM, 128 keys x N, double buffered) = K_tile Q^T    tcgen05.mma
+// and the epilogue thread that owns TMEM lane r (= key j) forms the group sum
+// for each of the 32 queries inside one thread.  Three passes keep the work
+// on chip and exact:
+//   SAMPLE  8 evenly spaced tiles per CTA -> 1024 sample scores per row
+//   (k2_thresh_kernel) per row, an estimate tau of a score that about 2 K
+//           candidates exceed: the r-th largest sample, r = 2 K s/n
+//   FILTER  every tile; candidates at or above the row's bound are appended,
+//           in ascending j, to the row's survivor list in this SM's slot of
+//           the workspace (L2-resident).  A list about to overflow is
+//           compacted in place to its exact top K and the bound is raised to
+//           its K-th entry.  At the end each row's exact top-min(K, n) is
+//           taken from the list (radix select on the fp32 bits, ties to the
+//           lower j, output ascending) -- or, if fewer than min(K, n)
+//           candidates passed (tau overestimated), the row is marked,
+//   RETRY   re-runs only the tiles with a marked row, with bound 0.
+// Ordering of equal scores: the survivor lists are ascending in j, and every
+// selection step keeps the first (lowest-j) entries among equal keys.
+#include <cudaTypedefs.h>
+
+#include "hs2_kernels.h"
+#include "tc05.cuh"
+
+namespace hs2 {
+
+bool make_map(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z);  // k1_full_tc.cu
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();                                      // k1_full_tc.cu
+
+namespace {
+
+constexpr int SL_QT = 32;          // queries per CTA
+constexpr int SL_BN = 128;         // keys per tile (MMA M)
+constexpr int SL_NS = 3;           // K pipeline stages
+constexpr int SL_EPI_WARPS = 16;   // four warpgroups, each a quarter of the query columns
+constexpr int SL_NWG = SL_EPI_WARPS / 4;
+constexpr int SL_TMA_WARP = SL_EPI_WARPS;
+constexpr int SL_MMA_WARP = SL_EPI_WARPS + 1;
+constexpr int SL_THREADS = 32 * (SL_EPI_WARPS + 2);
+constexpr int SL_SAMPLE_TILES = 8; // sample tiles per CTA
+constexpr int SL_SPR = SL_SAMPLE_TILES * SL_BN;  // sample slots per row
+constexpr int SL_CMAX = 4096;      // survivor list capacity per row
+constexpr int SL_SLOTS = 256;      // per-SM survivor slots (indexed by %smid)
+constexpr int SL_MIN_SMEM = 120 * 1024;  // keeps one CTA per SM (slots are per SM)
+
+enum { MODE_SAMPLE = 0, MODE_FILTER = 1, MODE_RETRY = 2 };
+
+template <int D, int G>
+struct SlCfg {
+    static constexpr int N = SL_QT * G;            // MMA N: (query, head) columns
+    static constexpr int KB = D / 64;
+    static constexpr int QBLK = N * 128;           // one 64-wide column block of Q (N rows x 128 B)
+    static constexpr int KBLK = SL_BN * 128;       // one 64-wide column block of a K tile
+    static constexpr int Q_OFF = 0;
+    static constexpr int K_OFF = Q_OFF + KB * QBLK;
+    static constexpr int MISC_OFF = K_OFF + SL_NS * KB * KBLK;
+    // misc: barriers, l2[N], row state, per-warp histograms and counts
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int L2_OFF = MISC_OFF + BAR_BYTES;
+    static constexpr int ROW_OFF = L2_OFF + N * 4;
+    static constexpr int ROW_BYTES = SL_QT * 4 * 4;       // cnt, bound_s, bound_j, t
+    static constexpr int WCNT_OFF = ROW_OFF + ROW_BYTES;  // [4 warps][32 rows]
+    static constexpr int HIST_OFF = WCNT_OFF + 4 * SL_QT * 4;
+    static constexpr int END = HIST_OFF + SL_EPI_WARPS * 256 * 4;
+    static constexpr int SMEM_NEED = END + 1024;
+    static constexpr int SMEM = SMEM_NEED > SL_MIN_SMEM ? SMEM_NEED : SL_MIN_SMEM;
+    static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
+};
+
+enum : int { SB_Q = 0, SB_KFULL = 1, SB_KEMPTY = SB_KFULL + SL_NS, SB_SFULL = SB_KEMPTY + SL_NS,
+             SB_SEMPTY = SB_SFULL + 2, SB_DRAIN = SB_SEMPTY + 2, SB_COUNT = SB_DRAIN + 1 };
+
+struct SelArgs {
+    const float* lse;       // [B, H_q, n_q]
+    int32_t* idx;           // [B, H_kv, n_q, K]
+    float* samples;         // [rows][SL_SPR]
+    int32_t* s_valid;       // [rows] valid samples per row
+    float* tau;             // [rows] threshold estimate
+    int32_t* status;        // [rows] 1 = needs the retry pass
+    uint2* slots;           // [n_slots][32][cmax] (score bits, j)
+    int i_begin, i_count;   // query chunk of this call
+    int cmax;               // survivor list capacity per row
+    int slot_by_block;      // 1: slot = block id (small grids); 0: slot = %smid (one CTA per SM)
+};
+
+__device__ __forceinline__ uint32_t smid() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%smid;\n" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n)); }
+
+// ---------------------------------------------------------------------------
+// warp-level exact selection on (score bits, j) lists
+
+// The K-th largest key among the first n entries of `buf` (key = fp32 bits of a
+// non-negative score) and how many entries equal to it belong to the top K.
+__device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uint32_t* hist, uint32_t& kth,
+                         uint32_t& need_eq) {
+    const int lane = threadIdx.x & 31;
+    uint32_t prefix = 0, pmask = 0, k_rem = K;
+#pragma unroll 1
+    for (int pass = 0; pass < 4; ++pass) {
+        const int shift = 24 - 8 * pass;
+        for (int u = lane; u < 256; u += 32) hist[u] = 0;
+        __syncwarp();
+        for (int i = lane; i < n; i += 32) {
+            const uint32_t x = key[(int64_t)i * stride];
+            if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+        }
+        __syncwarp();
+        uint32_t bins[8], s = 0;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            bins[u] = hist[8 * (31 - lane) + u];
+            s += bins[u];
+        }
+        uint32_t incl = s;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        const uint32_t excl = incl - s;
+        uint32_t digit = 0, krem_new = 0;
+        const bool mine = excl < k_rem && k_rem <= incl;
+        if (mine) {
+            uint32_t above = excl;
+#pragma unroll
+            for (int u = 7; u >= 0; --u) {
+                if (above + bins[u] >= k_rem) {
+                    digit = 8 * (31 - lane) + u;
+                    krem_new = k_rem - above;
+                    break;
+                }
+                above += bins[u];
+            }
+        }
+        const uint32_t who = __ballot_sync(0xffffffffu, mine);
+        const int src = who ? __ffs(who) - 1 : 0;
+        digit = __shfl_sync(0xffffffffu, digit, src);
+        krem_new = __shfl_sync(0xffffffffu, krem_new, src);
+        prefix |= digit << shift;
+        pmask |= 255u << shift;
+        k_rem = krem_new;
+        __syncwarp();
+    }
+    kth = prefix;
+    need_eq = k_rem;
+}
+
+// Keep, in list order, the entries with key > kth plus the first need_eq with
+// key == kth.  compact: write kept entries to the front of `list`; otherwise
+// write their j to `out`.  Returns the number kept.
+__device__ int warp_keep(uint2* list, int n, uint32_t kth, uint32_t need_eq, int32_t* out, bool compact) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t eq_seen = 0, written = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        uint2 e = make_uint2(0u, 0u);
+        if (i < n) e = list[i];
+        const bool gt = i < n && e.x > kth;
+        const bool eq = i < n && e.x == kth;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < need_eq);
+        const uint32_t tb = __ballot_sync(0xffffffffu, take);
+        const uint32_t pos = written + __popc(tb & lt);
+        __syncwarp();
+        if (take) {
+            if (compact) list[pos] = e;
+            else out[pos] = (int32_t)e.y;
+        }
+        eq_seen += __popc(eqb);
+        written += __popc(tb);
+    }
+    __syncwarp();
+    return (int)written;
+}
+
+// ---------------------------------------------------------------------------
+
+template <int D, int G, int MODE>
+__global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                                    const __grid_constant__ CUtensorMap tm_k,
+                                                                    Problem p, SelArgs a) {
+    using C = SlCfg<D, G>;
+    constexpr int N = C::N;
+    constexpr int NH = N / SL_NWG;           // columns of one epilogue warpgroup
+    constexpr int CW = NH < 32 ? NH : 32;    // columns per TMEM load
+    constexpr int QH = SL_QT / SL_NWG;       // queries of one epilogue warpgroup
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
+    const uint32_t sQ = sbase + C::Q_OFF, sK = sbase + C::K_OFF;
+    const uint32_t bars = sbase + C::MISC_OFF;
+    auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::MISC_OFF + 8 * SB_COUNT);
+    tc::Abort* ab = reinterpret_cast<tc::Abort*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 8);
+    volatile int* okv = reinterpret_cast<volatile int*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 16);  // [wg][2]
+    float* l2s = reinterpret_cast<float*>(sgen + C::L2_OFF);
+    int32_t* r_cnt = reinterpret_cast<int32_t*>(sgen + C::ROW_OFF);
+    float* r_lo = reinterpret_cast<float*>(r_cnt + SL_QT);      // keep scores >= r_lo
+    int32_t* r_tlim = reinterpret_cast<int32_t*>(r_lo + SL_QT);  // last candidate key of the row
+    int32_t* r_act = r_tlim + SL_QT;                             // row takes part in this pass
+    int32_t* wcnt = reinterpret_cast<int32_t*>(sgen + C::WCNT_OFF);  // [4 key quarters][32 rows]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sgen + C::HIST_OFF);  // [8 warps][256]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = blockIdx.y, b = blockIdx.z;
+    const int q0 = blockIdx.x * SL_QT;  // first query of the CTA within the chunk
+    const int nq_here = min(SL_QT, a.i_count - q0);
+    const int64_t pos0 = seq_pos0(p, b, KID_SCORE) + a.i_begin;
+    const int64_t t_max = pos0 + q0 + nq_here - 1;
+    const int64_t cand_end = t_max - p.window + 1;  // candidate keys are j < cand_end
+    const int64_t row0 = (int64_t)(b * p.hkv + g) * a.i_count + q0;  // chunk row of query q0
+    if (cand_end <= 0 && MODE != MODE_FILTER) return;
+    const int n_ct = cand_end > 0 ? (int)((cand_end + SL_BN - 1) / SL_BN) : 0;
+
+    if (MODE == MODE_RETRY) {
+        // only tiles with a row marked by the filter pass run again
+        int need = 0;
+        for (int q = 0; q < nq_here; ++q) need |= a.status[row0 + q];
+        if (!need) return;
+    }
+    const uint32_t slot = a.slot_by_block ? (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x : smid();
+    if (MODE != MODE_SAMPLE && slot >= SL_SLOTS) {
+        if (tid == 0) report_error(p.err, HS2_ERR_DEVICE_CHECK, KID_SCORE, slot, 0);
+        return;
+    }
+    const int cmax = a.cmax;
+    uint2* lists = a.slots + (int64_t)slot * SL_QT * cmax;
+    const int n_tiles = MODE == MODE_SAMPLE ? min(SL_SAMPLE_TILES, n_ct) : n_ct;
+    auto tile_of = [&](int it) -> int {
+        if (MODE != MODE_SAMPLE) return it;
+        return (int)(((2 * (int64_t)it + 1) * n_ct) / (2 * n_tiles));
+    };
+
+    // row state
+    if (tid < SL_QT) {
+        const int q = tid;
+        const bool live = q < nq_here;
+        const int64_t t = pos0 + q0 + q;
+        const int64_t n = t - p.window + 1;
+        float bs = 0.f;
+        int32_t act = live && n > 0;
+        if (MODE == MODE_FILTER && act) bs = a.tau[row0 + q];
+        if (MODE == MODE_RETRY) act = live && a.status[row0 + q] != 0;
+        r_cnt[q] = 0;
+        r_lo[q] = act ? bs : INFINITY;
+        r_tlim[q] = (int32_t)(t - p.window);
+        r_act[q] = act;
+    }
+    for (int c = tid; c < N; c += SL_THREADS) {
+        const int q = c / G, hh = c % G;
+        const int i = a.i_begin + q0 + q;
+        l2s[c] = (q < nq_here) ? a.lse[(int64_t)(b * p.hq + g * G + hh) * p.nq + i] * kLog2e : INFINITY;
+    }
+    if (tid == 0) {
+        for (int i = 0; i < SB_COUNT; ++i)
+            tc::mbar_init(bar(i), (i >= SB_SEMPTY && i < SB_SEMPTY + 2) ? 32 * SL_EPI_WARPS : 1);
+        ab->flag = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == SL_MMA_WARP) tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == SL_TMA_WARP) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0 && n_tiles > 0) {
+            tc::mbar_expect_tx(bar(SB_Q), C::KB * C::QBLK);
+            for (int kb = 0; kb < C::KB; ++kb)
+                tc::tma_load_4d(sQ + kb * C::QBLK, &tm_q, bar(SB_Q), kb * 64, g * G, a.i_begin + q0, b);
+            int issued = 0;
+            for (int it = 0; it < n_tiles; ++it) {
+                const int s = it % SL_NS;
+                if (it >= SL_NS && !tc::mbar_wait(bar(SB_KEMPTY + s), ((it - SL_NS) / SL_NS) & 1, ab, p.err, KID_SCORE, 1))
+                    break;
+                tc::mbar_expect_tx(bar(SB_KFULL + s), C::KB * C::KBLK);
+                const int kt = tile_of(it);
+                for (int kb = 0; kb < C::KB; ++kb)
+                    tc::tma_load_3d(sK + (s * C::KB + kb) * C::KBLK, &tm_k, bar(SB_KFULL + s), kb * 64, kt * SL_BN,
+                                    b * p.hkv + g);
+                issued = it + 1;
+            }
+            if (ab->flag) {
+                tc::Abort none{0};
+                tc::mbar_wait(bar(SB_Q), 0, &none, nullptr, 0, 0);
+                for (int it = (issued > SL_NS ? issued - SL_NS : 0); it < issued; ++it)
+                    tc::mbar_wait(bar(SB_KFULL + it % SL_NS), (it / SL_NS) & 1, &none, nullptr, 0, 0);
+            }
+        }
+    } else if (warp == SL_MMA_WARP) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0 && n_tiles > 0) {
+            constexpr uint32_t ID = tc::idesc_bf16(SL_BN, N, 0, 0);
+            bool ok = tc::mbar_wait(bar(SB_Q), 0, ab, p.err, KID_SCORE, 2);
+            for (int it = 0; ok && it < n_tiles; ++it) {
+                const int s = it % SL_NS, sb = it & 1;
+                ok = tc::mbar_wait(bar(SB_KFULL + s), (it / SL_NS) & 1, ab, p.err, KID_SCORE, 3);
+                if (ok && it >= 2) ok = tc::mbar_wait(bar(SB_SEMPTY + sb), ((it - 2) >> 1) & 1, ab, p.err, KID_SCORE, 4);
+                if (!ok) break;
+                tc::fence_after_sync();
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t da = tc::sdesc_sw128(sK + (s * C::KB + (kk >> 2)) * C::KBLK + (kk & 3) * 32, 16, 1024);
+                    const uint64_t db = tc::sdesc_sw128(sQ + (kk >> 2) * C::QBLK + (kk & 3) * 32, 16, 1024);
+                    tc::mma_ss(tmem + sb * N, da, db, ID, kk > 0);
+                }
+                tc::mma_commit(bar(SB_SFULL + sb));
+                tc::mma_commit(bar(SB_KEMPTY + s));
+            }
+            tc::mma_commit(bar(SB_DRAIN));
+            tc::Abort none{0};
+            tc::mbar_wait(bar(SB_DRAIN), 0, &none, nullptr, 0, 0);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue warps
+        // warp w reads TMEM lanes 32*(w%4).. (keys of quarter kq) and the columns of
+        // warpgroup wg = w/4 (queries QH*wg .. QH*wg+QH-1)
+        const int wg = warp >> 2, kq = warp & 3;
+        const int et = tid & 127;  // key lane within the tile
+        const uint32_t lane_off = (uint32_t)(kq * 32) << 16;
+        const uint32_t lt = (1u << lane) - 1u;
+        const int barid = 1 + wg;
+        bool ok = true;
+        float lo[QH];
+        int32_t tlim[QH];
+#pragma unroll
+        for (int qq = 0; qq < QH; ++qq) {
+            lo[qq] = r_lo[wg * QH + qq];
+            tlim[qq] = r_tlim[wg * QH + qq];
+        }
+        for (int it = 0; it < n_tiles; ++it) {
+            const int sb = it & 1;
+            const int64_t jb = (int64_t)tile_of(it) * SL_BN;
+            const int64_t j = jb + et;
+            // one thread per warpgroup waits (bounded) and the named barrier hands
+            // the result to its four warps, so they leave the loop together
+            if (et == 0) okv[wg * 2 + (it & 1)] = tc::mbar_wait(bar(SB_SFULL + sb), (it >> 1) & 1, ab, p.err, KID_SCORE, 5);
+            named_sync(barid, 128);
+            if (!okv[wg * 2 + (it & 1)]) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            float sc[QH];
+#pragma unroll
+            for (int c = 0; c < NH / CW; ++c) {
+                float v[CW];
+                const uint32_t col = sb * N + wg * NH + c * CW;
+                if constexpr (CW == 32) tc::tmem_ld32(tmem + lane_off + col, v);
+                else if constexpr (CW == 16) tc::tmem_ld16(tmem + lane_off + col, v);
+                else tc::tmem_ld8(tmem + lane_off + col, v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int qq = 0; qq < CW / G; ++qq) {
+                    // p_h = 2^(s2 - lse2) for the G heads, summed as a tree
+                    float e[G];
+#pragma unroll
+                    for (int hh = 0; hh < G; ++hh)
+                        e[hh] = ex2(fmaf(v[qq * G + hh], p.scale_log2, -l2s[wg * NH + c * CW + qq * G + hh]));
+#pragma unroll
+                    for (int w2 = 1; w2 < G; w2 *= 2)
+#pragma unroll
+                        for (int hh = 0; hh + w2 < G; hh += 2 * w2) e[hh] += e[hh + w2];
+                    sc[c * (CW / G) + qq] = e[0];
+                }
+            }
+            tc::fence_before_sync();
+            tc::mbar_arrive(bar(SB_SEMPTY + sb));
+
+            if constexpr (MODE == MODE_SAMPLE) {
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    const int q = wg * QH + qq;
+                    if (q < nq_here) {
+                        const int64_t t = pos0 + q0 + q;
+                        a.samples[(row0 + q) * SL_SPR + it * SL_BN + et] = (j <= t - p.window) ? sc[qq] : 0.f;
+                    }
+                }
+            } else {
+                // FILTER / RETRY: ordered append (ascending j) of the candidates at or
+                // above each row's bound; key quarter kq's entries follow quarters < kq.
+                // Tiles entirely below every row's candidate limit skip the per-row test.
+                const bool all_valid = (int64_t)jb + SL_BN - 1 <= pos0 + q0 - p.window;
+                uint32_t bal[QH];
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    bool keep = sc[qq] >= lo[qq];
+                    if (!all_valid) keep = keep && (int32_t)j <= tlim[qq];
+                    bal[qq] = __ballot_sync(0xffffffffu, keep);
+                }
+                if (lane < QH) {
+                    uint32_t mine = 0;
+#pragma unroll
+                    for (int qq = 0; qq < QH; ++qq) mine = (lane == qq) ? bal[qq] : mine;
+                    wcnt[kq * SL_QT + wg * QH + lane] = __popc(mine);
+                }
+                named_sync(barid, 128);
+                // lane qq: base position of row (wg, qq) for this warp's key quarter
+                int mybase = 0;
+                if (lane < QH) {
+                    const int q = wg * QH + lane;
+                    mybase = r_cnt[q];
+                    for (int w = 0; w < kq; ++w) mybase += wcnt[w * SL_QT + q];
+                }
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    const int pos = __shfl_sync(0xffffffffu, mybase, qq) + __popc(bal[qq] & lt);
+                    if (((bal[qq] >> lane) & 1u) && pos < cmax)
+                        lists[(wg * QH + qq) * cmax + pos] = make_uint2(__float_as_uint(sc[qq]), (uint32_t)j);
+                }
+                named_sync(barid, 128);
+                if (et < QH) {
+                    const int q = wg * QH + et;
+                    r_cnt[q] += wcnt[q] + wcnt[SL_QT + q] + wcnt[2 * SL_QT + q] + wcnt[3 * SL_QT + q];
+                }
+                named_sync(barid, 128);
+                // rare: a list that could overflow on the next tile is cut to its exact top K;
+                // later keys (larger j) then need a score strictly above the K-th kept one
+                bool changed = false;
+                for (int qq = 0; qq < QH; ++qq) {
+                    const int q = wg * QH + qq;
+                    const int cnt = r_cnt[q];
+                    if (cnt > cmax - SL_BN && cnt > p.topk) {
+                        changed = true;
+                        if ((qq & 3) == kq) {
+                            uint2* lst = lists + (int64_t)q * cmax;
+                            uint32_t kth, need_eq;
+                            warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, min(cnt, cmax), (uint32_t)p.topk,
+                                     hist + warp * 256, kth, need_eq);
+                            const int kept = warp_keep(lst, min(cnt, cmax), kth, need_eq, nullptr, true);
+                            if (lane == 0) {
+                                r_cnt[q] = kept;
+                                r_lo[q] = nextafterf(__uint_as_float(kth), INFINITY);
+                            }
+                        }
+                    }
+                }
+                if (changed) {
+                    named_sync(barid, 128);
+#pragma unroll
+                    for (int qq = 0; qq < QH; ++qq) lo[qq] = r_lo[wg * QH + qq];
+                }
+            }
+        }
+        if constexpr (MODE == MODE_SAMPLE) {
+            // unused sample slots hold 0 (they rank below every valid sample)
+            for (int it2 = n_tiles; it2 < SL_SAMPLE_TILES; ++it2)
+                for (int qq = 0; qq < QH; ++qq) {
+                    const int q = wg * QH + qq;
+                    if (q < nq_here) a.samples[(row0 + q) * SL_SPR + it2 * SL_BN + et] = 0.f;
+                }
+            if (et < QH && wg * QH + et < nq_here) {
+                // valid samples of the row: sampled keys j <= t - window
+                const int q = wg * QH + et;
+                const int64_t t = pos0 + q0 + q;
+                int cnt = 0;
+                for (int it2 = 0; it2 < n_tiles; ++it2) {
+                    const int64_t jb2 = (int64_t)tile_of(it2) * SL_BN;
+                    const int64_t hi = t - p.window - jb2 + 1;
+                    cnt += (int)(hi < 0 ? 0 : (hi > SL_BN ? SL_BN : hi));
+                }
+                a.s_valid[row0 + q] = cnt;
+            }
+        } else if (ok) {
+            // exact top-min(K, n) of every active row, ascending j, -1 padded
+            for (int qq = kq; qq < QH; qq += 4) {
+                const int q = wg * QH + qq;
+                if (q >= nq_here) continue;
+                int32_t* orow = a.idx + ((int64_t)(b * p.hkv + g) * p.nq + a.i_begin + q0 + q) * p.topk;
+                if (!r_act[q]) {
+                    if (MODE == MODE_FILTER) {  // no candidates at all (t < window)
+                        for (int u = lane; u < p.topk; u += 32) orow[u] = -1;
+                        if (lane == 0) a.status[row0 + q] = 0;
+                    }
+                    continue;
+                }
+                const int64_t t = pos0 + q0 + q;
+                const int64_t n = t - p.window + 1;
+                const int n_sel = (int)(n < p.topk ? n : p.topk);
+                const int cnt = min(r_cnt[q], cmax);
+                uint2* lst = lists + (int64_t)q * cmax;
+                if (cnt < n_sel) {
+                    if (lane == 0) a.status[row0 + q] = 1;  // the estimate was too high: retry
+                    continue;
+                }
+                int written;
+                if (cnt == n_sel) {
+                    for (int u = lane; u < cnt; u += 32) orow[u] = (int32_t)lst[u].y;
+                    written = cnt;
+                } else {
+                    uint32_t kth, need_eq;
+                    warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)n_sel, hist + warp * 256, kth,
+                             need_eq);
+                    written = warp_keep(lst, cnt, kth, need_eq, orow, false);
+                }
+                for (int u = written + lane; u < p.topk; u += 32) orow[u] = -1;
+                if (lane == 0) a.status[row0 + q] = 0;
+            }
+        }
+    }
+
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == SL_MMA_WARP) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+// Per row: tau = the r-th largest sample, r = ceil(2 K s / n) (s valid
+// samples, n candidates); 0 when every candidate fits the survivor list.
+__global__ void __launch_bounds__(128) k2_thresh_kernel(Problem p, SelArgs a) {
+    __shared__ uint32_t hist[4][256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)p.B * p.hkv * a.i_count;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+    if (row >= rows) return;
+    const int qi = (int)(row % a.i_count);
+    const int b = (int)(row / ((int64_t)p.hkv * a.i_count));
+    const int64_t t = seq_pos0(p, b, KID_TOPK) + a.i_begin + qi;
+    const int64_t n = t - p.window + 1;
+    const int s = a.s_valid[row];
+    float tau = 0.f;
+    if (n > a.cmax / 2 && s > 0) {
+        int64_t r = (2 * (int64_t)p.topk * s + n - 1) / n;
+        if (r < 1) r = 1;
+        if (r <= s) {
+            uint32_t kth, need_eq;
+            warp_kth(reinterpret_cast<const uint32_t*>(a.samples + row * SL_SPR), 1, SL_SPR, (uint32_t)r, hist[warp],
+                     kth, need_eq);
+            tau = __uint_as_float(kth);
+        }
+    }
+    if (lane == 0) a.tau[row] = tau;
+}
+
+// [B][H_q][n_q][D] bf16 seen as (D, H_q, n_q, B) with box (64, G, 32, 1): the
+// shared-memory tile rows come out ordered (query, head), 128 bytes each.
+bool make_q_map(CUtensorMap* m, const void* base, int D, int hq, int nq, int B, int G) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)hq, (cuuint64_t)nq, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)nq * D * 2, (cuuint64_t)D * 2, (cuuint64_t)hq * nq * D * 2};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)SL_QT, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int G, int MODE>
+cudaError_t launch_mode(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mk, const SelArgs& a,
+                        cudaStream_t st) {
+    using C = SlCfg<D, G>;
+    auto kern = k2_select_tc_kernel<D, G, MODE>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.i_count + SL_QT - 1) / SL_QT, p.hkv, p.B);
+    prof_begin(MODE == MODE_SAMPLE ? KID_SCORE : MODE == MODE_FILTER ? KID_FILTER : KID_RETRY, st);
+    kern<<<grid, SL_THREADS, C::SMEM, st>>>(mq, mk, p, a);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+    CUtensorMap mq, mk;
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv))
+        return cudaErrorInvalidValue;
+    cudaError_t e = launch_mode<D, G, MODE_SAMPLE>(p, mq, mk, a, st);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)p.B * p.hkv * a.i_count;
+    prof_begin(KID_THRESH, st);
+    k2_thresh_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(p, a);
+    prof_end(st);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_mode<D, G, MODE_FILTER>(p, mq, mk, a, st)) != cudaSuccess) return e;
+    return launch_mode<D, G, MODE_RETRY>(p, mq, mk, a, st);
+}
+
+template <int D>
+cudaError_t launch_select_d(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+    switch (p.hq / p.hkv) {
+        case 1: return launch_select_dg<D, 1>(p, q, k, a, st);
+        case 2: return launch_select_dg<D, 2>(p, q, k, a, st);
+        case 4: return launch_select_dg<D, 4>(p, q, k, a, st);
+        default: return launch_select_dg<D, 8>(p, q, k, a, st);
+    }
+}
+
+}  // namespace
+
+// Survivor list capacity and slot count of a call over queries with up to
+// n_cand_max candidates, in CTAs of 32 queries.
+static void select_tc_geometry(const Problem& p, int i_count, int64_t n_cand_max, int& cmax, int& n_slots,
+                               int& by_block) {
+    cmax = n_cand_max <= SL_CMAX ? (int)((n_cand_max + 31) / 32 * 32) : SL_CMAX;
+    if (cmax < 32) cmax = 32;
+    const int64_t grid = (int64_t)((i_count + SL_QT - 1) / SL_QT) * p.hkv * p.B;
+    by_block = grid <= SL_SLOTS;
+    n_slots = by_block ? (int)grid : SL_SLOTS;
+}
+
+size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max) {
+    int cmax, n_slots, by_block;
+    select_tc_geometry(p, i_count, n_cand_max, cmax, n_slots, by_block);
+    const int64_t rows = (int64_t)p.B * p.hkv * i_count;
+    const size_t per_row = SL_SPR * 4 + 3 * 4;
+    return (size_t)n_slots * SL_QT * cmax * sizeof(uint2) + (size_t)rows * per_row;
+}
+
+cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
+                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st) {
+    const int64_t rows = (int64_t)p.B * p.hkv * i_count;
+    uint8_t* base = reinterpret_cast<uint8_t*>(scratch);
+    SelArgs a;
+    int n_slots;
+    select_tc_geometry(p, i_count, n_cand_max, a.cmax, n_slots, a.slot_by_block);
+    a.lse = lse;
+    a.idx = idx;
+    a.slots = reinterpret_cast<uint2*>(base);
+    base += (size_t)n_slots * SL_QT * a.cmax * sizeof(uint2);
+    a.samples = reinterpret_cast<float*>(base);
+    base += (size_t)rows * SL_SPR * 4;
+    a.s_valid = reinterpret_cast<int32_t*>(base);
+    base += (size_t)rows * 4;
+    a.tau = reinterpret_cast<float*>(base);
+    base += (size_t)rows * 4;
+    a.status = reinterpret_cast<int32_t*>(base);
+    a.i_begin = i_begin;
+    a.i_count = i_count;
+    if (p.D == 64) return launch_select_d<64>(p, q, k, a, st);
+    return launch_select_d<128>(p, q, k, a, st);
+}
+
+}  // namespace hs2

@@ -29,7 +29,8 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
-                6: "decode_combine", 7: "fused_attn_select"}
+                6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
+                10: "select_retry"}
 
 
 class HS2Error(RuntimeError):
@@ -212,7 +213,7 @@ def hs2_profile_start(checked=False) -> None:
 
 def hs2_profile_stop(checked=False) -> dict:
     """{kernel name: (total ms, launches)} recorded since hs2_profile_start."""
-    n = 8
+    n = 16
     ms = (ctypes.c_float * n)()
     cnt = (ctypes.c_uint64 * n)()
     _check(load(checked).hs2_profile_stop(n, ms, cnt), "hs2_profile_stop")

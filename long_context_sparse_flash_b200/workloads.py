@@ -66,6 +66,8 @@ WORKLOADS: Dict[str, Workload] = {
         # 1M context: batch-8 decode over independent 1M contexts, seed 4
         Workload("decode_1m", 8, 1, 1048575, 1048576, 32, 4, 128, 128, 1024, 4, "segments", 64, 4,
                  decode=True),
+        # profiling case: the last 4096 queries of the 32K prefill (same per-row work, 1/8 of the rows)
+        Workload("prefill_32k_tail", 1, 4096, 28672, 32768, 32, 4, 128, 128, 1024, 4, "gaussian", 16, 1),
     ]
 }
 

@@ -51,7 +51,12 @@ def test_workspace_size_rules():
     s = shape(n_q=4096, kv_len=4096)
     n = nv.hs2_workspace_size(s, nv.HS2_ENTRY_FULL_SELECT)
     cand = 4096 - 128
-    assert n == 256 + 4096 * 4 * ((cand + 3) // 4 * 4) * 4
+    # prefill: per-SM survivor lists (256 slots x 32 rows x capacity) + 4108 B of state per row
+    cap = (cand + 31) // 32 * 32
+    assert n == 256 + 256 * 32 * cap * 8 + 4 * 4096 * (1024 * 4 + 12)
+    # decode: every candidate's score is stored
+    d = shape(n_q=1, batch=8, q_pos0=4095, kv_len=4096)
+    assert nv.hs2_workspace_size(d, nv.HS2_ENTRY_DECODE) == 256 + 8 * 4 * ((cand + 3) // 4 * 4) * 4
     # invalid shapes size to 0
     assert nv.hs2_workspace_size(shape(h_q=30), nv.HS2_ENTRY_FULL_SELECT) == 0
     assert nv.hs2_workspace_size(shape(q_pos0=1), nv.HS2_ENTRY_FULL_SELECT) == 0
