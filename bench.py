@@ -441,7 +441,7 @@ def main():
     ap.add_argument("--workload", default="prefill_32k", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=64, help="query rows in the oracle baseline sample")
+    ap.add_argument("--cpu-rows", type=int, default=1536, help="query rows in the oracle baseline sample (about 10 s of host work)")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference-arm step")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":

@@ -6,14 +6,14 @@
 //
 // One CTA = one (sequence, query, KV group); its G heads share every gathered
 // K/V row.  The attended rows S = idx U window are listed in shared memory,
-// split over 4 warps in 16-row tiles, and gathered with 16-byte cp.async into
+// split over 2 warps in 16-row tiles, and gathered with 16-byte cp.async into
 // per-warp double-buffered, swizzled staging.  Per tile:
 //   S^T (16 keys x 8 heads) = K_tile Q^T      mma.sync m16n8k16, A = K rows
 //   P^T = 2^(S^T - m) per head column, online softmax over the warp's tiles
 //   O^T (D x 8 heads) += V_tile^T P^T         A = V^T via ldmatrix.trans,
 //                                             B = P^T via movmatrix.trans
 // The group's heads sit in the MMA's N = 8 columns (padded when G < 8), so no
-// tensor-core work is spent on padding rows of M.  The 4 warps' partial
+// tensor-core work is spent on padding rows of M.  The warps' partial
 // (max, sum, O) are merged exactly at the end.
 #include "hs2_kernels.h"
 
@@ -21,7 +21,7 @@ namespace hs2 {
 
 namespace {
 
-constexpr int SP_WARPS = 4;
+constexpr int SP_WARPS = 2;  // more, smaller CTAs per SM hide the gather latency best
 
 template <int D>
 struct K3Cfg {
@@ -125,14 +125,17 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
         __syncwarp();
         const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES, sv = sk + C::TILE_BYTES;
 
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        // two independent accumulation chains (even / odd k-steps) halve the MMA latency
+        float c[4] = {0.f, 0.f, 0.f, 0.f}, c2[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
             uint32_t a[4];
             const int mi = lane >> 3;
             ldsm_x4(a, sk + swz<C::CH>((mi & 1) * 8 + (lane & 7), 2 * ks + (mi >> 1)));
-            mma16816(c, a, qb[ks]);
+            mma16816((ks & 1) ? c2 : c, a, qb[ks]);
         }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) c[e] += c2[e];
         // rows lane/4 and lane/4 + 8 of the tile; columns 2*(lane%4) + {0, 1}
         bool row_ok[2];
 #pragma unroll
