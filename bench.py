@@ -67,8 +67,12 @@ def kernel_work(w: wl.Workload):
         "sparse_attn": dict(bound="hbm", bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
     }
     if w.decode:
-        # decode: every candidate's score is computed (QK^T) and stored, then a radix top-k reads it
-        work["select_score"] = dict(bound="tensor", flops=f["select_qk_flops"])
+        # decode: the attention pass stores each candidate's G scaled logits (fp32); the score
+        # kernel streams them (32 B per candidate for G = 8) and writes one fp32 score each;
+        # the radix top-k reads every score (at least once) and writes idx
+        work["decode_attn"] = dict(bound="hbm", bytes=f["kv_bytes"] + 2 * f["q_bytes"] + 4 * n_rows * Hq
+                                   + 4.0 * 8 * cand)
+        work["select_score"] = dict(bound="hbm", bytes=(4.0 * 8 + 4.0) * cand)
         work["select_topk"] = dict(bound="hbm", bytes=4.0 * cand + f["idx_bytes"])
     else:
         # prefill: the filtered sweep recomputes QK^T over every candidate of every query
@@ -81,7 +85,8 @@ def source_sha(path: str) -> str:
 
 
 KERNEL_SOURCE = {
-    "full_attn": "k1_full_tc.cu", "select_score": "k2_select.cu", "select_topk": "k2_select.cu",
+    "full_attn": "k1_full_tc.cu", "select_score": "k1_decode.cu", "select_topk": "k2_select.cu",
+    "decode_attn": "k1_decode.cu",
     "select_filter": "k2_select_tc.cu", "sparse_attn": "k3_sparse_attn.cu",
 }
 

@@ -155,10 +155,22 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
         !aligned(idx, 4) || !aligned(ws, 256) || (seq_len && !aligned(seq_len, 8)))
         return HS2_ERR_INVALID_ARG;
     const ScorePlan sp = score_plan(p, decode);
-    if (ws_bytes < kHeader + sp.bytes) return HS2_ERR_WORKSPACE;
+    const size_t extra = decode ? decode_scratch_bytes(p) : 0;
+    if (ws_bytes < kHeader + (decode ? (sp.bytes + 255) / 256 * 256 : sp.bytes) + extra) return HS2_ERR_WORKSPACE;
     p.seq_len = seq_len;
     p.err = reinterpret_cast<WsHeader*>(ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (decode) {
+        // split-KV attention (+ stored logits) -> combine -> scores -> exact top-k
+        float* scores = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kHeader);
+        void* scratch = reinterpret_cast<uint8_t*>(ws) + kHeader + (sp.bytes + 255) / 256 * 256;
+        const bool sel = p.topk > 0 && sp.sstride > 0;
+        cudaError_t e = launch_decode(p, q, k, v, out, lse, scratch, sel ? scores : nullptr, sp.sstride, st);
+        if (e != cudaSuccess) return HS2_ERR_CUDA;
+        if (p.topk == 0) return HS2_OK;
+        e = launch_topk(p, scores, sp.sstride, idx, 0, 1, st);
+        return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+    }
     cudaError_t e = launch_full(p, q, k, v, out, lse, st);
     if (e != cudaSuccess) return HS2_ERR_CUDA;
     if (p.topk == 0) return HS2_OK;
@@ -195,7 +207,10 @@ size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
         case HS2_ENTRY_SPARSE: return kHeader;
         case HS2_ENTRY_FULL_SELECT:
         case HS2_ENTRY_PREFILL: return kHeader + score_plan(p, false).bytes;
-        case HS2_ENTRY_DECODE: return kHeader + score_plan(p, true).bytes;
+        case HS2_ENTRY_DECODE: {
+            if (p.nq != 1) return 0;
+            return kHeader + (score_plan(p, true).bytes + 255) / 256 * 256 + decode_scratch_bytes(p);
+        }
         default: return 0;
     }
 }

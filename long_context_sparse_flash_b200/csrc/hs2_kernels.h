@@ -49,6 +49,13 @@ size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
                              void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st);
 
+// Decode (one query per sequence): split-KV partial attention that also stores
+// the candidates' logits, exact combine -> out/lse, and (scores != nullptr)
+// the selection scores [B][H_kv][sstride] for the radix top-k.
+size_t decode_scratch_bytes(const Problem& p);
+cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const void* v, void* out, float* lse,
+                          void* scratch, float* scores, int64_t sstride, cudaStream_t st);
+
 // K3: one sparse KV-reuse layer.
 cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* out, cudaStream_t st);

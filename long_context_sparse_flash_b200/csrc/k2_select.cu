@@ -10,9 +10,10 @@
 // 8-column tile holds one query's 8 heads (G = 8) in one row of the fragment and
 // the group sum is two in-thread adds plus two quad shuffles.  Part 2
 // (k2_topk_kernel) selects the top-k of each (query, group) row exactly: a
-// 4-pass, 8-bit radix select on the fp32 bit patterns (non-negative floats order
-// like their bits) finds the k-th key, then one ordered pass keeps every key
-// above it plus the lowest-index keys equal to it, writing indices ascending.
+// 3-pass (11, 11, 10 bits) radix select on the fp32 bit patterns (non-negative
+// floats order like their bits; histogram updates aggregated per warp with
+// match_any) finds the k-th key, then one ordered pass keeps every key above
+// it plus the lowest-index keys equal to it, writing indices ascending.
 #include "hs2_kernels.h"
 
 namespace hs2 {
@@ -159,38 +160,51 @@ __global__ void __launch_bounds__(SC_WARPS * 32) k2_score_kernel(Problem p, cons
 
 // ---------------------------------------------------------------------------
 
-constexpr int TK_THREADS = 256;
+constexpr int TK_THREADS = 1024;
+constexpr int TK_WARPS = TK_THREADS / 32;
+constexpr int TK_BINS = 2048;
 
 struct TopkSmem {
-    uint32_t hist[256];
-    uint32_t warp_tot[TK_THREADS / 32];
-    uint32_t warp_tot2[TK_THREADS / 32];
+    uint32_t hist[TK_BINS];
+    uint32_t warp_tot[TK_WARPS];
+    uint32_t warp_tot2[TK_WARPS];
     uint32_t digit, k_rem;
 };
 
-// exclusive prefix of `flag` over the block; returns the prefix, writes the block total
-__device__ __forceinline__ uint32_t block_excl_scan(bool flag, uint32_t* warp_tot, uint32_t& total) {
+// exclusive prefix of per-thread counts over the block; returns the prefix,
+// writes the block total
+__device__ __forceinline__ uint32_t block_excl_sum(uint32_t x, uint32_t* warp_tot, uint32_t& total) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const uint32_t bal = __ballot_sync(0xffffffffu, flag);
-    const uint32_t in_warp = __popc(bal & ((1u << lane) - 1u));
-    if (lane == 0) warp_tot[warp] = __popc(bal);
+    uint32_t incl = x;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
     __syncthreads();
     uint32_t before = 0, tot = 0;
 #pragma unroll
-    for (int w = 0; w < TK_THREADS / 32; ++w) {
-        const uint32_t x = warp_tot[w];
-        before += (w < warp) ? x : 0u;
-        tot += x;
+    for (int w = 0; w < TK_WARPS; ++w) {
+        const uint32_t v = warp_tot[w];
+        before += (w < warp) ? v : 0u;
+        tot += v;
     }
     total = tot;
-    return before + in_warp;
+    return before + incl - x;
+}
+
+// Radix digit boundaries: bits [31,21], [20,10], [9,0] of the fp32 score.
+__device__ __forceinline__ void digit_of(int pass, int& shift, uint32_t& mask) {
+    shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+    mask = pass == 2 ? 1023u : 2047u;
 }
 
 __global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const float* __restrict__ scores,
                                                              int64_t sstride, int32_t* __restrict__ idx,
                                                              int i_begin, int i_count) {
     __shared__ TopkSmem sm;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int qi = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int i = i_begin + qi;
     const int64_t pos0 = seq_pos0(p, b, KID_TOPK);
@@ -203,71 +217,108 @@ __global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const fl
         return;
     }
     const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + ((int64_t)(b * p.hkv + g) * i_count + qi) * sstride);
+    const int n4 = n / 4;  // rows start 16-byte aligned (sstride is a multiple of 4)
 
-    // radix select: find the key value of the topk-th largest
+    // radix select: the key value of the topk-th largest (non-negative floats
+    // order like their bit patterns), three passes of 11, 11 and 10 bits
     uint32_t prefix = 0, pmask = 0;
     uint32_t k_rem = (uint32_t)p.topk;
 #pragma unroll 1
-    for (int pass = 0; pass < 4; ++pass) {
-        const int shift = 24 - 8 * pass;
-        sm.hist[tid] = 0;
+    for (int pass = 0; pass < 3; ++pass) {
+        int shift;
+        uint32_t dmask;
+        digit_of(pass, shift, dmask);
+        for (int u = tid; u < TK_BINS; u += TK_THREADS) sm.hist[u] = 0;
         __syncthreads();
-        for (int j = tid; j < n; j += TK_THREADS) {
-            const uint32_t x = key[j];
-            if ((x & pmask) == prefix) atomicAdd(&sm.hist[(x >> shift) & 255u], 1u);
+        auto add = [&](uint32_t x, bool valid) {
+            const bool part = valid && (x & pmask) == prefix;
+            const uint32_t act = __ballot_sync(0xffffffffu, part);
+            if (part) {
+                const uint32_t bin = (x >> shift) & dmask;
+                const uint32_t peers = __match_any_sync(act, bin);
+                if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
+            }
+        };
+        for (int base = 0; base < n4; base += TK_THREADS) {
+            const int j4 = base + tid;
+            uint4 x = make_uint4(0u, 0u, 0u, 0u);
+            if (j4 < n4) x = reinterpret_cast<const uint4*>(key)[j4];
+            const bool ok = j4 < n4;
+            add(x.x, ok);
+            add(x.y, ok);
+            add(x.z, ok);
+            add(x.w, ok);
+        }
+        {  // tail of up to 3 keys; every lane takes part in the warp-wide vote
+            const int j = n4 * 4 + tid;
+            const bool ok = tid < 32 && j < n;
+            if (tid < 32) add(ok ? key[j] : 0u, ok);
         }
         __syncthreads();
         if (tid < 32) {
-            // lane l owns bins 8*(31-l) .. 8*(31-l)+7, so lane order is descending digit
-            uint32_t bins[8], s = 0;
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                bins[u] = sm.hist[8 * (31 - tid) + u];
-                s += bins[u];
-            }
-            uint32_t incl = s;  // inclusive prefix over lanes 0..tid (descending digits)
+            // lane l owns bins [64*(31-l), 64*(31-l)+63], so lane order is descending digit
+            uint32_t s = 0;
+            const int nb = (int)dmask + 1;
+            const int per = nb / 32;
+            for (int u = 0; u < per; ++u) s += sm.hist[per * (31 - lane) + u];
+            uint32_t incl = s;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-                if (tid >= o) incl += y;
+                if (lane >= o) incl += y;
             }
             const uint32_t excl = incl - s;
             if (excl < k_rem && k_rem <= incl) {
                 uint32_t above = excl;
-#pragma unroll
-                for (int u = 7; u >= 0; --u) {
-                    if (above + bins[u] >= k_rem) {
-                        sm.digit = 8 * (31 - tid) + u;
+                for (int u = per - 1; u >= 0; --u) {
+                    const uint32_t c = sm.hist[per * (31 - lane) + u];
+                    if (above + c >= k_rem) {
+                        sm.digit = (uint32_t)(per * (31 - lane) + u);
                         sm.k_rem = k_rem - above;
                         break;
                     }
-                    above += bins[u];
+                    above += c;
                 }
             }
         }
         __syncthreads();
         prefix |= sm.digit << shift;
-        pmask |= 255u << shift;
+        pmask |= dmask << shift;
         k_rem = sm.k_rem;
         __syncthreads();
     }
     const uint32_t kth = prefix;
     const uint32_t need_eq = k_rem;  // how many keys equal to kth are taken (lowest j first)
 
-    // ordered pass: keep keys > kth and the first need_eq keys == kth, ascending j
+    // ordered pass: keep keys > kth and the first need_eq keys == kth, ascending j;
+    // each thread takes 4 consecutive keys per step
     uint32_t eq_seen = 0, written = 0;
-    for (int base = 0; base < n; base += TK_THREADS) {
-        const int j = base + tid;
-        const uint32_t x = j < n ? key[j] : 0u;
-        const bool gt = j < n && x > kth;
-        const bool eq = j < n && x == kth;
+    for (int base = 0; base < n; base += 4 * TK_THREADS) {
+        const int j0 = base + 4 * tid;
+        uint32_t x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = (j0 + u < n) ? key[j0 + u] : 0u;
+        uint32_t neq = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) neq += (j0 + u < n && x[u] == kth) ? 1u : 0u;
         uint32_t eq_tot;
-        const uint32_t eq_rank = block_excl_scan(eq, sm.warp_tot, eq_tot);
-        const bool take = gt || (eq && eq_seen + eq_rank < need_eq);
+        uint32_t eq_rank = eq_seen + block_excl_sum(neq, sm.warp_tot, eq_tot);
+        bool take[4];
+        uint32_t ntake = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool valid = j0 + u < n;
+            const bool eq = valid && x[u] == kth;
+            take[u] = (valid && x[u] > kth) || (eq && eq_rank < need_eq);
+            eq_rank += eq ? 1u : 0u;
+            ntake += take[u] ? 1u : 0u;
+        }
         __syncthreads();
         uint32_t take_tot;
-        const uint32_t pos = block_excl_scan(take, sm.warp_tot2, take_tot);
-        if (take) orow[written + pos] = j;
+        uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (take[u]) orow[pos++] = j0 + u;
         eq_seen += eq_tot;
         written += take_tot;
         __syncthreads();

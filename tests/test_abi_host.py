@@ -54,9 +54,16 @@ def test_workspace_size_rules():
     # prefill: per-SM survivor lists (256 slots x 32 rows x capacity) + 4108 B of state per row
     cap = (cand + 31) // 32 * 32
     assert n == 256 + 256 * 32 * cap * 8 + 4 * 4096 * (1024 * 4 + 12)
-    # decode: every candidate's score is stored
+    # decode: every candidate's score, the chunk states and the stored logits
     d = shape(n_q=1, batch=8, q_pos0=4095, kv_len=4096)
-    assert nv.hs2_workspace_size(d, nv.HS2_ENTRY_DECODE) == 256 + 8 * 4 * ((cand + 3) // 4 * 4) * 4
+    scores = 8 * 4 * ((cand + 3) // 4 * 4) * 4
+    want = -(-(4 * 148 + 31) // 32)                 # chunks wanted per (sequence, group)
+    chunk = max(256, -(-(-(-4096 // want)) // 64) * 64)
+    n_chunks = -(-4096 // chunk)
+    part = 8 * 4 * n_chunks * (8 * 128 + 16) * 4
+    logits = 8 * 4 * 4096 * 8 * 4
+    rnd = lambda x: -(-x // 256) * 256
+    assert nv.hs2_workspace_size(d, nv.HS2_ENTRY_DECODE) == 256 + rnd(scores) + rnd(part) + rnd(logits)
     # invalid shapes size to 0
     assert nv.hs2_workspace_size(shape(h_q=30), nv.HS2_ENTRY_FULL_SELECT) == 0
     assert nv.hs2_workspace_size(shape(q_pos0=1), nv.HS2_ENTRY_FULL_SELECT) == 0
