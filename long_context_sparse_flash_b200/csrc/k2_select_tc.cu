@@ -67,7 +67,7 @@ struct SlCfg {
     static constexpr int BAR_BYTES = 256;
     static constexpr int L2_OFF = MISC_OFF + BAR_BYTES;
     static constexpr int ROW_OFF = L2_OFF + N * 4;
-    static constexpr int ROW_BYTES = SL_QT * 4 * 4;       // cnt, bound_s, bound_j, t
+    static constexpr int ROW_BYTES = SL_QT * 5 * 4;       // cnt[2], lo, tlim, act
     static constexpr int WCNT_OFF = ROW_OFF + ROW_BYTES;  // [4 warps][32 rows]
     static constexpr int HIST_OFF = WCNT_OFF + 4 * SL_QT * 4;
     static constexpr int END = HIST_OFF + SL_EPI_WARPS * 256 * 4;
@@ -209,8 +209,8 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     tc::Abort* ab = reinterpret_cast<tc::Abort*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 8);
     volatile int* okv = reinterpret_cast<volatile int*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 16);  // [wg][2]
     float* l2s = reinterpret_cast<float*>(sgen + C::L2_OFF);
-    int32_t* r_cnt = reinterpret_cast<int32_t*>(sgen + C::ROW_OFF);
-    float* r_lo = reinterpret_cast<float*>(r_cnt + SL_QT);      // keep scores >= r_lo
+    int32_t* r_cnt = reinterpret_cast<int32_t*>(sgen + C::ROW_OFF);  // [tile parity][32]
+    float* r_lo = reinterpret_cast<float*>(r_cnt + 2 * SL_QT);  // keep scores >= r_lo
     int32_t* r_tlim = reinterpret_cast<int32_t*>(r_lo + SL_QT);  // last candidate key of the row
     int32_t* r_act = r_tlim + SL_QT;                             // row takes part in this pass
     int32_t* wcnt = reinterpret_cast<int32_t*>(sgen + C::WCNT_OFF);  // [4 key quarters][32 rows]
@@ -257,6 +257,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         if (MODE == MODE_FILTER && act) bs = a.tau[row0 + q];
         if (MODE == MODE_RETRY) act = live && a.status[row0 + q] != 0;
         r_cnt[q] = 0;
+        r_cnt[SL_QT + q] = 0;
         r_lo[q] = act ? bs : INFINITY;
         r_tlim[q] = (int32_t)(t - p.window);
         r_act[q] = act;
@@ -357,6 +358,39 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 break;
             }
             tc::fence_after_sync();
+            if constexpr (MODE != MODE_SAMPLE) {
+                // rare: a list that could overflow on this tile is first cut to its exact
+                // top K; later keys (larger j) then need a score strictly above its K-th entry
+                // every warp reads the counts before any of them changes (uniform decision)
+                uint32_t need = 0;
+                int cnts[QH];
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    cnts[qq] = r_cnt[(it & 1) * SL_QT + wg * QH + qq];
+                    if (cnts[qq] > cmax - SL_BN && cnts[qq] > p.topk) need |= 1u << qq;
+                }
+                if (need) {
+                    named_sync(barid, 128);
+#pragma unroll 1
+                    for (int qq = kq; qq < QH; qq += 4) {
+                        if (!((need >> qq) & 1u)) continue;
+                        const int q = wg * QH + qq;
+                        uint2* lst = lists + (int64_t)q * cmax;
+                        const int cnt = min(cnts[qq], cmax);
+                        uint32_t kth, need_eq;
+                        warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)p.topk, hist + warp * 256,
+                                 kth, need_eq);
+                        const int kept = warp_keep(lst, cnt, kth, need_eq, nullptr, true);
+                        if (lane == 0) {
+                            r_cnt[(it & 1) * SL_QT + q] = kept;
+                            r_lo[q] = nextafterf(__uint_as_float(kth), INFINITY);
+                        }
+                    }
+                    named_sync(barid, 128);
+#pragma unroll
+                    for (int qq = 0; qq < QH; ++qq) lo[qq] = r_lo[wg * QH + qq];
+                }
+            }
             float sc[QH];
 #pragma unroll
             for (int c = 0; c < NH / CW; ++c) {
@@ -369,10 +403,20 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
 #pragma unroll
                 for (int qq = 0; qq < CW / G; ++qq) {
                     // p_h = 2^(s2 - lse2) for the G heads, summed as a tree
-                    float e[G];
+                    float e[G], lv[G];
+                    const float* lrow = l2s + wg * NH + c * CW + qq * G;
+                    if constexpr (G % 4 == 0) {
 #pragma unroll
-                    for (int hh = 0; hh < G; ++hh)
-                        e[hh] = ex2(fmaf(v[qq * G + hh], p.scale_log2, -l2s[wg * NH + c * CW + qq * G + hh]));
+                        for (int h4 = 0; h4 < G / 4; ++h4) {
+                            const float4 x = reinterpret_cast<const float4*>(lrow)[h4];
+                            lv[4 * h4] = x.x; lv[4 * h4 + 1] = x.y; lv[4 * h4 + 2] = x.z; lv[4 * h4 + 3] = x.w;
+                        }
+                    } else {
+#pragma unroll
+                        for (int hh = 0; hh < G; ++hh) lv[hh] = lrow[hh];
+                    }
+#pragma unroll
+                    for (int hh = 0; hh < G; ++hh) e[hh] = ex2(fmaf(v[qq * G + hh], p.scale_log2, -lv[hh]));
 #pragma unroll
                     for (int w2 = 1; w2 < G; w2 *= 2)
 #pragma unroll
@@ -411,12 +455,14 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     wcnt[kq * SL_QT + wg * QH + lane] = __popc(mine);
                 }
                 named_sync(barid, 128);
-                // lane qq: base position of row (wg, qq) for this warp's key quarter
+                // lane qq: base position of row (wg, qq) for this warp's key quarter; the
+                // last quarter's warp publishes the row's new count for the next tile
                 int mybase = 0;
                 if (lane < QH) {
                     const int q = wg * QH + lane;
-                    mybase = r_cnt[q];
+                    mybase = r_cnt[(it & 1) * SL_QT + q];
                     for (int w = 0; w < kq; ++w) mybase += wcnt[w * SL_QT + q];
+                    if (kq == 3) r_cnt[((it + 1) & 1) * SL_QT + q] = mybase + wcnt[3 * SL_QT + q];
                 }
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
@@ -424,40 +470,9 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     if (((bal[qq] >> lane) & 1u) && pos < cmax)
                         lists[(wg * QH + qq) * cmax + pos] = make_uint2(__float_as_uint(sc[qq]), (uint32_t)j);
                 }
-                named_sync(barid, 128);
-                if (et < QH) {
-                    const int q = wg * QH + et;
-                    r_cnt[q] += wcnt[q] + wcnt[SL_QT + q] + wcnt[2 * SL_QT + q] + wcnt[3 * SL_QT + q];
-                }
-                named_sync(barid, 128);
-                // rare: a list that could overflow on the next tile is cut to its exact top K;
-                // later keys (larger j) then need a score strictly above the K-th kept one
-                bool changed = false;
-                for (int qq = 0; qq < QH; ++qq) {
-                    const int q = wg * QH + qq;
-                    const int cnt = r_cnt[q];
-                    if (cnt > cmax - SL_BN && cnt > p.topk) {
-                        changed = true;
-                        if ((qq & 3) == kq) {
-                            uint2* lst = lists + (int64_t)q * cmax;
-                            uint32_t kth, need_eq;
-                            warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, min(cnt, cmax), (uint32_t)p.topk,
-                                     hist + warp * 256, kth, need_eq);
-                            const int kept = warp_keep(lst, min(cnt, cmax), kth, need_eq, nullptr, true);
-                            if (lane == 0) {
-                                r_cnt[q] = kept;
-                                r_lo[q] = nextafterf(__uint_as_float(kth), INFINITY);
-                            }
-                        }
-                    }
-                }
-                if (changed) {
-                    named_sync(barid, 128);
-#pragma unroll
-                    for (int qq = 0; qq < QH; ++qq) lo[qq] = r_lo[wg * QH + qq];
-                }
             }
         }
+        if constexpr (MODE != MODE_SAMPLE) named_sync(barid, 128);  // every append is in place
         if constexpr (MODE == MODE_SAMPLE) {
             // unused sample slots hold 0 (they rank below every valid sample)
             for (int it2 = n_tiles; it2 < SL_SAMPLE_TILES; ++it2)
@@ -493,7 +508,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 const int64_t t = pos0 + q0 + q;
                 const int64_t n = t - p.window + 1;
                 const int n_sel = (int)(n < p.topk ? n : p.topk);
-                const int cnt = min(r_cnt[q], cmax);
+                const int cnt = min(r_cnt[(n_tiles & 1) * SL_QT + q], cmax);
                 uint2* lst = lists + (int64_t)q * cmax;
                 if (cnt < n_sel) {
                     if (lane == 0) a.status[row0 + q] = 1;  // the estimate was too high: retry

@@ -191,3 +191,18 @@ def test_empty_call_launches_nothing():
     before = nv.hs2_launch_count()
     out, lse, idx = nv.full_attn_select(q, k, k, window=4, topk=4, q_pos0=0)
     assert nv.hs2_launch_count() == before
+
+
+def test_exact_ties_force_list_compaction():
+    """q = 0 makes every candidate's score exactly G/(t+1): the tie rule fixes the
+    selection to indices 0..K-1, and with more than 4096 candidates per row every
+    survivor list overflows and is compacted (the rare path of the selection)."""
+    w = wl.custom("all_ties", n_q=96, q_pos0=9000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=1, seed=4)
+    inp = wl.make_inputs(w, "cuda")
+    inp["q"].zero_()
+    gpu = P.run_gpu(w, inp)
+    want = torch.arange(w.topk, dtype=torch.int32, device="cuda")
+    assert torch.equal(gpu["idx"], want.expand_as(gpu["idx"]))
+    rows = np.array([0, 1, 47, 95])
+    P.compare_rows(w, inp, gpu, 0, rows)
