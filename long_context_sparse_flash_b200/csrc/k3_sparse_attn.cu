@@ -95,18 +95,25 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     const __nv_bfloat16* kg = k + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
     const __nv_bfloat16* vg = v + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
     const uint32_t s_w = smem_u32(smem) + warp * C::WARP_BYTES;
+    // Tile loads: lanes 0-15 copy one row and lanes 16-31 the next (16-byte
+    // chunk = lane % 16 for D = 128), eight row pairs per 16-row tile.  A lane
+    // reads the tile's row indices once and takes each row's index by shuffle;
+    // the swizzled chunk is (lane chunk ^ row parity) ^ (2 * it mod 8).
     auto load_tile = [&](int mt, int stage) {
-        const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES, sv = sk + C::TILE_BYTES;
+        const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES;
+        const int li = mt * 16 + (lane & 15);
+        const int32_t jl = li < n ? list[li] : -1;
+        const int32_t myj = (jl >= 0 && (int64_t)jl <= t) ? jl : -1;
+        constexpr int RPI = 32 / C::CH;  // rows per iteration (2 for D = 128, 4 for D = 64)
+        const int hi = lane / C::CH, ch = lane % C::CH;
 #pragma unroll
-        for (int it = 0; it < 16 * C::CH / 32; ++it) {
-            const int c = it * 32 + lane;
-            const int r = c / C::CH, ch = c % C::CH;
-            const int li = mt * 16 + r;
-            const int32_t j = li < n ? list[li] : -1;
-            const bool ok = j >= 0 && (int64_t)j <= t;
-            const int64_t off = (int64_t)(ok ? j : 0) * D + ch * 8;
-            cp_async16(sk + swz<C::CH>(r, ch), kg + off, ok ? 16 : 0);
-            cp_async16(sv + swz<C::CH>(r, ch), vg + off, ok ? 16 : 0);
+        for (int it = 0; it < 16 / RPI; ++it) {
+            const int r = it * RPI + hi;
+            const int32_t j = __shfl_sync(0xffffffffu, myj, r);
+            const size_t goff = (size_t)(j < 0 ? 0 : j) * (size_t)(D * 2) + (size_t)ch * 16u;
+            const uint32_t so = sk + swz<C::CH>(r, ch);
+            cp_async16(so, (const char*)kg + goff, j < 0 ? 0 : 16);
+            cp_async16(so + C::TILE_BYTES, (const char*)vg + goff, j < 0 ? 0 : 16);
         }
     };
 
@@ -138,11 +145,12 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
         for (int e = 0; e < 4; ++e) c[e] += c2[e];
         // rows lane/4 and lane/4 + 8 of the tile; columns 2*(lane%4) + {0, 1}
         bool row_ok[2];
-#pragma unroll
-        for (int r = 0; r < 2; ++r) {
-            const int li = mt * 16 + (lane >> 2) + 8 * r;
-            const int32_t j = li < n ? list[li] : -1;
-            row_ok[r] = j >= 0 && (int64_t)j <= t;
+        {
+            const int li = mt * 16 + (lane & 15);
+            const int32_t jl = li < n ? list[li] : -1;
+            const bool okl = jl >= 0 && (int64_t)jl <= t;
+            row_ok[0] = __shfl_sync(0xffffffffu, okl, lane >> 2);
+            row_ok[1] = __shfl_sync(0xffffffffu, okl, (lane >> 2) + 8);
         }
         float s[4];
 #pragma unroll
