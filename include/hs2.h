@@ -204,6 +204,12 @@ uint64_t hs2_launch_count(void);
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 
+/* Diagnostics: evaluate the library's exp2 implementations at n device points
+ * x: y[0..n) = hardware ex2, y[n..2n) = degree-3 polynomial, y[2n..3n) =
+ * degree-5 polynomial (the FMA-pipe 2^x used beside the hardware unit in the
+ * softmax and selection kernels).  Asynchronous on `stream`. */
+hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t stream);
+
 /* 1 when the library was built with device-side input checks (HS2_CHECKED). */
 int hs2_is_checked_build(void);
 

@@ -6,22 +6,23 @@
 //
 // One CTA = one (sequence, query, KV group); its G heads share every gathered
 // K/V row.  The attended rows S = idx U window are listed in shared memory,
-// split over 2 warps in 16-row tiles, and gathered with 16-byte cp.async into
-// per-warp double-buffered, swizzled staging.  Per tile:
+// cut into 16-row tiles and gathered with 16-byte cp.async into double-buffered,
+// swizzled staging.  One warp per CTA: the gather is latency-bound, and many
+// small CTAs per SM (about eleven) keep the most tiles in flight.  Per tile:
 //   S^T (16 keys x 8 heads) = K_tile Q^T      mma.sync m16n8k16, A = K rows
 //   P^T = 2^(S^T - m) per head column, online softmax over the warp's tiles
 //   O^T (D x 8 heads) += V_tile^T P^T         A = V^T via ldmatrix.trans,
 //                                             B = P^T via movmatrix.trans
 // The group's heads sit in the MMA's N = 8 columns (padded when G < 8), so no
-// tensor-core work is spent on padding rows of M.  The warps' partial
-// (max, sum, O) are merged exactly at the end.
+// tensor-core work is spent on padding rows of M.  With SP_WARPS > 1 the
+// warps' partial (max, sum, O) would be merged exactly at the end.
 #include "hs2_kernels.h"
 
 namespace hs2 {
 
 namespace {
 
-constexpr int SP_WARPS = 2;  // more, smaller CTAs per SM hide the gather latency best
+constexpr int SP_WARPS = 1;  // more, smaller CTAs per SM hide the gather latency best
 
 template <int D>
 struct K3Cfg {

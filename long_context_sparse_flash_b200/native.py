@@ -26,7 +26,7 @@ HS2_ENTRY_FULL_SELECT, HS2_ENTRY_SPARSE, HS2_ENTRY_PREFILL, HS2_ENTRY_DECODE = 0
 EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_sparse_attn",
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
-           "hs2_full_attn_select_static", "hs2_static_scratch_bytes")
+           "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
@@ -83,9 +83,10 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_full_attn_select_static.argtypes = [sh, P, P, P, P, P, P, P]
     lib.hs2_static_scratch_bytes.argtypes = []
     lib.hs2_static_scratch_bytes.restype = S
+    lib.hs2_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
-                 "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static"):
+                 "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -190,6 +191,14 @@ def hs2_full_attn_select_static(shape, q, k, v, out, lse, idx, stream=None, chec
     _check(load(checked).hs2_full_attn_select_static(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                                      _ptr(lse), _ptr(idx), _stream(stream)),
            "hs2_full_attn_select_static")
+
+
+def hs2_selftest_exp2(x: torch.Tensor, stream=None):
+    """(hardware ex2, degree-3, degree-5) evaluations of 2^x on the device."""
+    n = x.numel()
+    y = torch.empty(3 * n, dtype=torch.float32, device=x.device)
+    _check(load().hs2_selftest_exp2(_ptr(x), _ptr(y), int(n), _stream(stream)), "hs2_selftest_exp2")
+    return y[:n], y[n:2 * n], y[2 * n:]
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):

@@ -19,7 +19,7 @@ FAKE = ctypes.c_void_p(1 << 40)
 def declared_symbols():
     text = open(HEADER).read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(hs2_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(hs2_[a-z0-9_]+)\s*\(", text)))
 
 
 @pytest.fixture(scope="module", params=[False, True], ids=["release", "checked"])

@@ -1,0 +1,27 @@
+"""The FMA-pipe 2^x polynomials against float64 2^x and the hardware ex2, on
+the device: relative error within the fitted bounds over the range the
+kernels use, exact powers of two, and 0 below -127 (masked entries)."""
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_flash_b200 import native as nv
+
+pytestmark = pytest.mark.gpu
+
+
+def test_exp2_polynomials_error_bounds():
+    xs = torch.cat([torch.linspace(-126.0, 20.0, 400001), torch.arange(-126, 21, dtype=torch.float32),
+                    torch.tensor([-127.5, -200.0, float("-inf")])]).cuda()
+    hw, p3, p5 = (y.cpu().numpy().astype(np.float64) for y in nv.hs2_selftest_exp2(xs))
+    x = xs.cpu().numpy().astype(np.float64)
+    ref = np.exp2(x)
+    ok = x >= -125.0  # normal results
+    rel = lambda y: np.abs(y[ok] / ref[ok] - 1)
+    assert rel(hw).max() < 1e-6
+    assert rel(p3).max() < 1.3e-4
+    assert rel(p5).max() < 3e-7
+    ints = np.isin(x, np.arange(-125, 21))
+    assert np.all(p3[ints] == ref[ints]) and np.all(p5[ints] == ref[ints])  # exact powers of two
+    low = x < -127.0
+    assert np.all(p3[low] == 0) and np.all(p5[low] == 0)
