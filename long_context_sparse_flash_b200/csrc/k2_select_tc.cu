@@ -33,7 +33,7 @@
 
 namespace hs2 {
 
-bool make_map(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z);  // k1_full_tc.cu
+bool make_map(CUtensorMap* m, const void* base, uint64_t x, uint64_t y, uint64_t z, uint32_t box_rows);  // k1_full_tc.cu
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn();                                      // k1_full_tc.cu
 
 namespace {
@@ -598,7 +598,7 @@ cudaError_t launch_mode(const Problem& p, const CUtensorMap& mq, const CUtensorM
 template <int D, int G>
 cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
     CUtensorMap mq, mk;
-    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv))
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
         return cudaErrorInvalidValue;
     cudaError_t e = launch_mode<D, G, MODE_SAMPLE>(p, mq, mk, a, st);
     if (e != cudaSuccess) return e;
