@@ -6,17 +6,20 @@
 // One CTA = two 128-row query tiles (A, B) of one head, 10 warps:
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
 //              warpgroup owns query row r of its tile = TMEM lane r
-//   warp 8     TMA producer: both Q tiles once, then K/V tiles of 64 keys
-//              (3-stage ring)
-//   warp 9     TMEM allocator and single-thread tcgen05.mma issuer
+//   warp 8     TMA producer: both Q tiles once, then K and V tiles of 128 keys
+//              (separate rings, since K of a tile is consumed a step before V)
+//   warp 9     TMEM allocator and MMA issuer (one elected lane)
+//   warps 10-11 idle; with warps 8-9 they form the warpgroup that hands its
+//              registers to the softmax warpgroups (setmaxnreg)
 // Per key tile j, for each query tile X in {A, B}:
-//   S_X,j (TMEM, double buffered) = Q_X K_j^T      tcgen05.mma, A = Q_X, B = K (K-major)
-//   softmax X: tcgen05.ld S_X,j, scale + causal mask, running max with lazy
-//   rescale (O_X is only rescaled when the max grows by more than 2^8),
-//   P_X,j = 2^(S - m) as bf16 into a 128B-swizzled shared tile
-//   O_X (TMEM) += P_X,j V_j                         tcgen05.mma, A = P_X, B = V (MN-major)
-// The two warpgroups' softmaxes overlap with each other's MMAs, so the tensor
-// core is not left idle while one tile's exponentials are computed.
+//   S_X,j (TMEM, 128 columns) = Q_X K_j^T           tcgen05.mma, A = Q_X, B = K (smem, K-major)
+//   softmax X: tcgen05.ld S_X,j, causal mask, running max with lazy rescale
+//   (O_X is only rescaled when the max grows by more than 2^8),
+//   P_X,j = 2^(S - m) as bf16 pairs, tcgen05.st over the first half of S_X
+//   O_X (TMEM) += P_X,j V_j                          tcgen05.mma, A = P_X (TMEM), B = V (smem, MN-major)
+// Keeping P in tensor memory leaves the shared-memory operand reads of the
+// P V product to V alone; the two tiles' softmaxes alternate with each other's
+// MMAs, so the tensor core is not left idle while one tile's exponentials run.
 // Operand tiles are 128-byte swizzled (TMA SWIZZLE_128B), rows of 64 bf16.
 // Every wait is bounded (tc::mbar_wait): a stalled CTA reports HS2_ERR_TIMEOUT
 // through the error word, drains its own copies, frees its TMEM and exits.
@@ -60,46 +63,48 @@ namespace {
 
 constexpr int PP_QT = 2;      // query tiles per CTA
 constexpr int PP_BM = 128;    // rows per query tile
-constexpr int PP_BN = 64;     // keys per K/V tile
-constexpr int PP_NS = 3;      // K/V ring stages
+constexpr int PP_BN = 128;    // keys per K/V tile
 constexpr int PP_TMA_WARP = 8;
 constexpr int PP_MMA_WARP = 9;
-constexpr int PP_THREADS = 320;
+constexpr int PP_THREADS = 384;   // warps 10-11 only complete the third warpgroup
+// register budgets after the split: softmax warpgroups up, the rest down
+constexpr uint32_t PP_REG_SOFTMAX = 208, PP_REG_OTHER = 80;
 constexpr uint32_t PP_TMEM_COLS = 512;
 
 template <int D>
 struct PpCfg {
     static constexpr int KB = D / 64;                  // 64-element (128-byte) column blocks
-    static constexpr int QBLK = PP_BM * 128;           // 128 rows x 128 B
-    static constexpr int KBLK = PP_BN * 128;           // 64 rows x 128 B
-    static constexpr int Q_OFF = 0;                    // [tile][kb] QBLK
-    static constexpr int K_OFF = Q_OFF + PP_QT * KB * QBLK;
-    static constexpr int V_OFF = K_OFF + PP_NS * KB * KBLK;
-    static constexpr int P_OFF = V_OFF + PP_NS * KB * KBLK;   // [tile] 128 rows x 64 keys (one block)
-    static constexpr int BAR_OFF = P_OFF + PP_QT * QBLK;
+    static constexpr int BLK = 128 * 128;              // one block: 128 rows x 128 B
+    static constexpr int NS = D == 64 ? 4 : 2;         // K/V ring stages
+    static constexpr int Q_OFF = 0;                    // [tile][kb] BLK
+    static constexpr int K_OFF = Q_OFF + PP_QT * KB * BLK;
+    static constexpr int V_OFF = K_OFF + NS * KB * BLK;
+    static constexpr int BAR_OFF = V_OFF + NS * KB * BLK;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
-    // TMEM columns: S[tile][buf] 64 each at 0..255, O[tile] D each from 256
-    static constexpr int O_COL = 4 * PP_BN;
+    // TMEM columns: S[tile] 128 each at 0 and 128 (P[tile], 128 bf16 keys =
+    // 64 columns, overwrites the first half of S[tile] once it has been read),
+    // O[tile] D each from 256
+    static constexpr int O_COL = PP_QT * PP_BN;
 };
 
 enum : int {
     PB_Q = 0,
     PB_KFULL = 1,
-    PB_VFULL = PB_KFULL + PP_NS,
-    PB_KVEMPTY = PB_VFULL + PP_NS,
-    PB_SFULL = PB_KVEMPTY + PP_NS,   // [tile][buf]
-    PB_SEMPTY = PB_SFULL + 4,        // [tile][buf]
-    PB_PFULL = PB_SEMPTY + 4,        // [tile]
-    PB_ODONE = PB_PFULL + 2,         // [tile]
+    PB_VFULL = PB_KFULL + 4,
+    PB_KEMPTY = PB_VFULL + 4,
+    PB_VEMPTY = PB_KEMPTY + 4,
+    PB_SFULL = PB_VEMPTY + 4,   // [tile]
+    PB_PFULL = PB_SFULL + 2,    // [tile], 128 arrivals
+    PB_ODONE = PB_PFULL + 2,    // [tile]
     PB_DRAIN = PB_ODONE + 2,
     PB_COUNT = PB_DRAIN + 1,
 };
 
-// Row of 64 scores of one S tile from TMEM (this thread's lane); keys past
-// the causal limit t are set to -inf.
+// This thread's row of one 128-key S tile from TMEM; keys past the causal
+// limit t are set to -inf.
 __device__ __forceinline__ void load_scores(uint32_t addr, float* s, bool diag, int64_t j0, int64_t t) {
-    tc::tmem_ld32(addr, s);
-    tc::tmem_ld32(addr + 32, s + 32);
+#pragma unroll
+    for (int c = 0; c < PP_BN / 32; ++c) tc::tmem_ld32(addr + 32 * c, s + 32 * c);
     tc::tmem_wait_ld();
     if (diag) {
 #pragma unroll
@@ -108,23 +113,25 @@ __device__ __forceinline__ void load_scores(uint32_t addr, float* s, bool diag, 
     }
 }
 
-// Max of the 64 raw scores: four independent three-input max chains.
+// Max of the raw scores: four independent three-input max chains.
 __device__ __forceinline__ float tile_max(const float* s) {
+    constexpr int L = PP_BN / 4;
     float mc[4];
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
-        const float* sq = s + q4 * (PP_BN / 4);
+        const float* sq = s + q4 * L;
         float a = sq[0];
 #pragma unroll
-        for (int c = 1; c + 1 < PP_BN / 4; c += 2) a = fmax3f(a, sq[c], sq[c + 1]);
-        mc[q4] = fmaxf(a, sq[PP_BN / 4 - 1]);
+        for (int c = 1; c + 1 < L; c += 2) a = fmax3f(a, sq[c], sq[c + 1]);
+        mc[q4] = fmaxf(a, sq[L - 1]);
     }
     return fmax3f(mc[0], mc[1], fmaxf(mc[2], mc[3]));
 }
 
-// In place s <- 2^(s * scale - m) for 64 scores, two lanes per instruction;
-// returns the row sum (four packed accumulators).
-__device__ __forceinline__ float exp_tile(float* s, float scale, float m) {
+// p = 2^(s * scale - m) for the row's 128 scores, two lanes per instruction,
+// packed to bf16 pairs in place (s[0..63] hold the pairs afterwards); returns the
+// row sum of the fp32 values (four packed accumulators).
+__device__ __forceinline__ float exp_pack_tile(float* s, float scale, float m) {
     const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
@@ -132,10 +139,9 @@ __device__ __forceinline__ float exp_tile(float* s, float scale, float m) {
         float2 e = ffma2(make_float2(s[c], s[c + 1]), sc2, nm2);
         e.x = ex2(e.x);
         e.y = ex2(e.y);
-        s[c] = e.x;
-        s[c + 1] = e.y;
         const int a4 = (c >> 1) & 3;
         acc[a4] = (c < 8) ? e : fadd2(acc[a4], e);
+        s[c >> 1] = __uint_as_float(pack_bf16(e.x, e.y));
     }
     const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
     return (a01.x + a01.y) + (a23.x + a23.y);
@@ -148,10 +154,11 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                                                                   Problem p, __nv_bfloat16* __restrict__ out,
                                                                   float* __restrict__ lse) {
     using C = PpCfg<D>;
+    constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
-    const uint32_t sQ = sbase + C::Q_OFF, sK = sbase + C::K_OFF, sV = sbase + C::V_OFF, sP = sbase + C::P_OFF;
+    const uint32_t sQ = sbase + C::Q_OFF, sK = sbase + C::K_OFF, sV = sbase + C::V_OFF;
     const uint32_t bars = sbase + C::BAR_OFF;
     auto bar = [&](int i) { return bars + 8u * (uint32_t)i; };
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sgen + C::BAR_OFF + 8 * PB_COUNT);
@@ -168,11 +175,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
     const int n_tiles = (int)((pos0 + i_last + PP_BN) / PP_BN);
 
     if (tid == 0) {
-        for (int i = 0; i < PB_COUNT; ++i) {
-            uint32_t cnt = 1;
-            if ((i >= PB_SEMPTY && i < PB_SEMPTY + 4) || (i >= PB_PFULL && i < PB_PFULL + 2)) cnt = 128;
-            tc::mbar_init(bar(i), cnt);
-        }
+        for (int i = 0; i < PB_COUNT; ++i) tc::mbar_init(bar(i), (i == PB_PFULL || i == PB_PFULL + 1) ? 128u : 1u);
         ab->flag = 0;
         tc::fence_mbar_init();
     }
@@ -182,172 +185,169 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == PP_TMA_WARP) {
+    if (warp >= 8) {
+      tc::setmaxnreg_dec<PP_REG_OTHER>();
+      if (warp == PP_TMA_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             const int zq = b * p.hq + h, zk = b * p.hkv + g;
-            tc::mbar_expect_tx(bar(PB_Q), PP_QT * C::KB * C::QBLK);
+            tc::mbar_expect_tx(bar(PB_Q), PP_QT * C::KB * C::BLK);
             for (int x = 0; x < PP_QT; ++x)
                 for (int kb = 0; kb < C::KB; ++kb)
-                    tc::tma_load_3d(sQ + (x * C::KB + kb) * C::QBLK, &tm_q, bar(PB_Q), kb * 64, i0 + x * PP_BM, zq);
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int s = j % PP_NS;
-                if (j >= PP_NS &&
-                    !tc::mbar_wait(bar(PB_KVEMPTY + s), ((j - PP_NS) / PP_NS) & 1, ab, p.err, KID_FULL, 1))
-                    break;
-                tc::mbar_expect_tx(bar(PB_KFULL + s), C::KB * C::KBLK);
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tc::tma_load_3d(sK + (s * C::KB + kb) * C::KBLK, &tm_k, bar(PB_KFULL + s), kb * 64, j * PP_BN, zk);
-                tc::mbar_expect_tx(bar(PB_VFULL + s), C::KB * C::KBLK);
-                for (int kb = 0; kb < C::KB; ++kb)
-                    tc::tma_load_3d(sV + (s * C::KB + kb) * C::KBLK, &tm_v, bar(PB_VFULL + s), kb * 64, j * PP_BN, zk);
-                issued = j + 1;
-            }
-            if (ab->flag) {  // drain: every issued load lands before the CTA exits
-                tc::Abort none{0};
-                tc::mbar_wait(bar(PB_Q), 0, &none, nullptr, 0, 0);
-                for (int j = (issued > PP_NS ? issued - PP_NS : 0); j < issued; ++j) {
-                    const int s = j % PP_NS;
-                    tc::mbar_wait(bar(PB_KFULL + s), (j / PP_NS) & 1, &none, nullptr, 0, 0);
-                    tc::mbar_wait(bar(PB_VFULL + s), (j / PP_NS) & 1, &none, nullptr, 0, 0);
+                    tc::tma_load_3d(sQ + (x * C::KB + kb) * C::BLK, &tm_q, bar(PB_Q), kb * 64, i0 + x * PP_BM, zq);
+            // K of tile j is needed one step before V of tile j: issue K(j), then V(j - 1)
+            int k_issued = 0, v_issued = 0;
+            bool ok = true;
+            for (int j = 0; ok && j <= n_tiles; ++j) {
+                if (j < n_tiles) {
+                    const int s = j % NS;
+                    if (j >= NS) ok = tc::mbar_wait(bar(PB_KEMPTY + s), ((j - NS) / NS) & 1, ab, p.err, KID_FULL, 1);
+                    if (!ok) break;
+                    tc::mbar_expect_tx(bar(PB_KFULL + s), C::KB * C::BLK);
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_3d(sK + (s * C::KB + kb) * C::BLK, &tm_k, bar(PB_KFULL + s), kb * 64, j * PP_BN, zk);
+                    k_issued = j + 1;
+                }
+                if (j >= 1) {
+                    const int jv = j - 1, s = jv % NS;
+                    if (jv >= NS) ok = tc::mbar_wait(bar(PB_VEMPTY + s), ((jv - NS) / NS) & 1, ab, p.err, KID_FULL, 2);
+                    if (!ok) break;
+                    tc::mbar_expect_tx(bar(PB_VFULL + s), C::KB * C::BLK);
+                    for (int kb = 0; kb < C::KB; ++kb)
+                        tc::tma_load_3d(sV + (s * C::KB + kb) * C::BLK, &tm_v, bar(PB_VFULL + s), kb * 64, jv * PP_BN, zk);
+                    v_issued = jv + 1;
                 }
             }
+            if (!ok || ab->flag) {  // drain: every issued load lands before the CTA exits
+                tc::Abort none{0};
+                tc::mbar_wait(bar(PB_Q), 0, &none, nullptr, 0, 0);
+                for (int j = (k_issued > NS ? k_issued - NS : 0); j < k_issued; ++j)
+                    tc::mbar_wait(bar(PB_KFULL + j % NS), (j / NS) & 1, &none, nullptr, 0, 0);
+                for (int j = (v_issued > NS ? v_issued - NS : 0); j < v_issued; ++j)
+                    tc::mbar_wait(bar(PB_VFULL + j % NS), (j / NS) & 1, &none, nullptr, 0, 0);
+            }
         }
-    } else if (warp == PP_MMA_WARP) {
+      } else if (warp == PP_MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         // The whole warp runs the loop and its waits (votes keep it converged);
-        // one elected lane issues the MMAs and their commits.
+        // one elected lane issues the MMAs and their commits.  Per key tile j:
+        //   O_A += P_A,j V_j ; S_A,j+1 = Q_A K_j+1 ; O_B += P_B,j V_j ; S_B,j+1 = Q_B K_j+1
+        // so the tensor core runs one tile's products while the other tile's
+        // softmax runs.  S_X,j+1 overwrites the columns P_X,j is read from; the
+        // MMAs of this thread execute in issue order, so P V reads P first.
         constexpr uint32_t ID_S = tc::idesc_bf16(PP_BM, PP_BN, 0, 0);  // A = Q, B = K: both K-major
-        constexpr uint32_t ID_O = tc::idesc_bf16(PP_BM, D, 0, 1);      // A = P K-major, B = V MN-major
+        constexpr uint32_t ID_O = tc::idesc_bf16(PP_BM, D, 0, 1);      // A = P (TMEM), B = V MN-major
         // descriptors of the first block of each operand; a byte offset o moves
         // the start address field by o / 16
         const uint64_t dq0 = tc::sdesc_sw128(sQ, 16, 1024), dk0 = tc::sdesc_sw128(sK, 16, 1024);
-        const uint64_t dp0 = tc::sdesc_sw128(sP, 16, 1024), dv0 = tc::sdesc_sw128(sV, C::KBLK, 1024);
-        bool ok = __all_sync(~0u, tc::mbar_wait(bar(PB_Q), 0, ab, p.err, KID_FULL, 2));
-        for (int j = 0; ok && j <= n_tiles; ++j) {
-            if (j < n_tiles) {
-                const int s = j % PP_NS, sb = j & 1;
-                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL + s), (j / PP_NS) & 1, ab, p.err, KID_FULL, 3));
-                for (int x = 0; ok && x < PP_QT; ++x) {
-                    if (j >= 2)
-                        ok = __all_sync(~0u, tc::mbar_wait(bar(PB_SEMPTY + 2 * x + sb), ((j - 2) >> 1) & 1, ab, p.err,
-                                                           KID_FULL, 4));
-                    if (!ok) break;
-                    tc::fence_after_sync();
-                    if (tc::elect_one()) {
+        const uint64_t dv0 = tc::sdesc_sw128(sV, C::BLK, 1024);
+        auto issue_s = [&](int x, int j) {
+            const int s = j % NS;
+            if (tc::elect_one()) {
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint64_t da = dq0 + (uint64_t)(((x * C::KB + (kk >> 2)) * C::QBLK + (kk & 3) * 32) >> 4);
-                            const uint64_t db = dk0 + (uint64_t)(((s * C::KB + (kk >> 2)) * C::KBLK + (kk & 3) * 32) >> 4);
-                            tc::mma_ss(tmem + (2 * x + sb) * PP_BN, da, db, ID_S, kk > 0);
-                        }
-                        tc::mma_commit(bar(PB_SFULL + 2 * x + sb));
-                    }
-                    __syncwarp();
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint64_t da = dq0 + (uint64_t)(((x * C::KB + (kk >> 2)) * C::BLK + (kk & 3) * 32) >> 4);
+                    const uint64_t db = dk0 + (uint64_t)(((s * C::KB + (kk >> 2)) * C::BLK + (kk & 3) * 32) >> 4);
+                    tc::mma_ss(tmem + x * PP_BN, da, db, ID_S, kk > 0);
                 }
-                if (!ok) break;
+                tc::mma_commit(bar(PB_SFULL + x));
             }
-            if (j >= 1) {
-                const int jp = j - 1, sp = jp % PP_NS;
-                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_VFULL + sp), (jp / PP_NS) & 1, ab, p.err, KID_FULL, 5));
-                for (int x = 0; ok && x < PP_QT; ++x) {
-                    ok = __all_sync(~0u, tc::mbar_wait(bar(PB_PFULL + x), jp & 1, ab, p.err, KID_FULL, 6));
-                    if (!ok) break;
-                    tc::fence_after_sync();
-                    if (tc::elect_one()) {
+            __syncwarp();
+        };
+        auto issue_pv = [&](int x, int j) {
+            const int s = j % NS;
+            if (tc::elect_one()) {
 #pragma unroll
-                        for (int kk = 0; kk < PP_BN / 16; ++kk) {
-                            const uint64_t da = dp0 + (uint64_t)((x * C::QBLK + kk * 32) >> 4);
-                            const uint64_t db = dv0 + (uint64_t)((sp * C::KB * C::KBLK + kk * 2048) >> 4);
-                            tc::mma_ss(tmem + C::O_COL + x * D, da, db, ID_O, (jp > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        tc::mma_commit(bar(PB_ODONE + x));
-                    }
-                    __syncwarp();
+                for (int kk = 0; kk < PP_BN / 16; ++kk) {
+                    const uint64_t db = dv0 + (uint64_t)((s * C::KB * C::BLK + kk * 2048) >> 4);
+                    tc::mma_ts(tmem + C::O_COL + x * D, tmem + x * PP_BN + kk * 8, db, ID_O, (j > 0 || kk > 0) ? 1u : 0u);
                 }
-                if (!ok) break;
-                if (tc::elect_one()) tc::mma_commit(bar(PB_KVEMPTY + sp));
-                __syncwarp();
             }
+            __syncwarp();
+        };
+        auto commit = [&](int i) {
+            if (tc::elect_one()) tc::mma_commit(bar(i));
+            __syncwarp();
+        };
+        bool ok = __all_sync(~0u, tc::mbar_wait(bar(PB_Q), 0, ab, p.err, KID_FULL, 3));
+        if (ok) ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL), 0, ab, p.err, KID_FULL, 4));
+        if (ok) {
+            tc::fence_after_sync();
+            issue_s(0, 0);
+            issue_s(1, 0);
+            commit(PB_KEMPTY);
+        }
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            const int s = j % NS, s1 = (j + 1) % NS;
+            const bool more = j + 1 < n_tiles;
+            ok = __all_sync(~0u, tc::mbar_wait(bar(PB_VFULL + s), (j / NS) & 1, ab, p.err, KID_FULL, 5));
+            if (ok && more)
+                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL + s1), ((j + 1) / NS) & 1, ab, p.err, KID_FULL, 6));
+            for (int x = 0; ok && x < PP_QT; ++x) {
+                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_PFULL + x), j & 1, ab, p.err, KID_FULL, 7));
+                if (!ok) break;
+                tc::fence_after_sync();
+                issue_pv(x, j);
+                if (more)
+                    issue_s(x, j + 1);
+                else
+                    commit(PB_ODONE + x);
+            }
+            if (!ok) break;
+            commit(PB_VEMPTY + s);
+            if (more) commit(PB_KEMPTY + s1);
         }
         // every issued MMA completes before TMEM is released
-        if (tc::elect_one()) tc::mma_commit(bar(PB_DRAIN));
-        __syncwarp();
+        commit(PB_DRAIN);
         tc::Abort none{0};
         tc::mbar_wait(bar(PB_DRAIN), 0, &none, nullptr, 0, 0);
+      }
     } else {
+        tc::setmaxnreg_inc<PP_REG_SOFTMAX>();
         // ------------------------------------------------------------ softmax (warps 0-7)
         const int x = warp >> 2;                // query tile of this warpgroup
         const int r = tid & 127;                // row within the tile == TMEM lane
         const int64_t t = pos0 + min(i0 + x * PP_BM + r, p.nq - 1);
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t s_col = 2 * x * PP_BN, o_col = C::O_COL + x * D;
-        const uint32_t sPx = sP + x * C::QBLK;
+        const uint32_t s_addr = tmem + lane_off + x * PP_BN, o_addr = tmem + lane_off + C::O_COL + x * D;
         float m = -INFINITY, l = 0.f;
         bool ok = true;
         float s[PP_BN];
         for (int j = 0; j < n_tiles && ok; ++j) {
-            const int sb = j & 1;
-            ok = tc::mbar_wait(bar(PB_SFULL + 2 * x + sb), (j >> 1) & 1, ab, p.err, KID_FULL, 7);
+            ok = tc::mbar_wait(bar(PB_SFULL + x), j & 1, ab, p.err, KID_FULL, 8);
             if (!ok) break;
             tc::fence_after_sync();
-            const uint32_t s_addr = tmem + lane_off + s_col + sb * PP_BN;
             const int64_t j0 = (int64_t)j * PP_BN;
-            const bool diag = j0 + PP_BN - 1 > t;
-            load_scores(s_addr, s, diag, j0, t);
-            tc::fence_before_sync();
-            tc::mbar_arrive(bar(PB_SEMPTY + 2 * x + sb));
+            load_scores(s_addr, s, j0 + PP_BN - 1 > t, j0, t);
             const float mt = tile_max(s) * p.scale_log2;
-            bool waited_o = false;
             if (mt > m + 8.f) {
-                // the running max grew by more than 2^8: rescale l and O
+                // the running max grew by more than 2^8: rescale l and O.  The
+                // commit behind S_X,j covers O_X += P_X,j-1 V_j-1, so O is final.
                 const float alpha = ex2(m - mt);
                 if (j > 0) {
-                    ok = tc::mbar_wait(bar(PB_ODONE + x), (j - 1) & 1, ab, p.err, KID_FULL, 8);
-                    if (!ok) break;
-                    waited_o = true;
-                    tc::fence_after_sync();
                     float o[32];
 #pragma unroll
                     for (int c = 0; c < D / 32; ++c) {
-                        tc::tmem_ld32(tmem + lane_off + o_col + c * 32, o);
+                        tc::tmem_ld32(o_addr + c * 32, o);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] *= alpha;
-                        tc::tmem_st32(tmem + lane_off + o_col + c * 32, o);
+                        tc::tmem_st32(o_addr + c * 32, o);
                     }
-                    tc::tmem_wait_st();
                 }
                 l *= alpha;
                 m = mt;
             }
-            l += exp_tile(s, p.scale_log2, m);
-            // the P tile is free once the previous P V product has completed
-            if (j > 0 && !waited_o) {
-                ok = tc::mbar_wait(bar(PB_ODONE + x), (j - 1) & 1, ab, p.err, KID_FULL, 9);
-                if (!ok) break;
-            }
-            // P row r: 64 keys = one 128-byte row of the swizzled block
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-                const float* v8 = s + ch * 8;
-                uint4 v;
-                v.x = pack_bf16(v8[0], v8[1]);
-                v.y = pack_bf16(v8[2], v8[3]);
-                v.z = pack_bf16(v8[4], v8[5]);
-                v.w = pack_bf16(v8[6], v8[7]);
-                const uint32_t addr = sPx + r * 128 + ((ch ^ (r & 7)) << 4);
-                asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};\n" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z),
-                             "r"(v.w)
-                             : "memory");
-            }
-            tc::fence_proxy_async();
+            l += exp_pack_tile(s, p.scale_log2, m);
+            // P_X,j (bf16 pairs) over the first 64 columns of S_X
+            tc::tmem_st32(s_addr, s);
+            tc::tmem_st32(s_addr + 32, s + 32);
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             tc::mbar_arrive(bar(PB_PFULL + x));
         }
         // epilogue: O / l -> out (bf16), lse
-        if (ok) ok = tc::mbar_wait(bar(PB_ODONE + x), (n_tiles - 1) & 1, ab, p.err, KID_FULL, 10);
+        if (ok) ok = tc::mbar_wait(bar(PB_ODONE + x), 0, ab, p.err, KID_FULL, 9);
         if (ok) {
             tc::fence_after_sync();
             const int i = i0 + x * PP_BM + r;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
-                tc::tmem_ld32(tmem + lane_off + o_col + c * 32, o);
+                tc::tmem_ld32(o_addr + c * 32, o);
                 tc::tmem_wait_ld();
                 if (i < p.nq) {
 #pragma unroll
@@ -394,6 +394,12 @@ cudaError_t launch_full_tc_d(const Problem& p, const void* q, const void* k, con
     auto kern = k1_full_tc_kernel<D>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
+    // the register split must fit in what the CTA is launched with, or the
+    // increase would wait for registers that never come
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if ((long)fa.numRegs * PP_THREADS < 256L * PP_REG_SOFTMAX + 128L * PP_REG_OTHER) return cudaErrorInvalidConfiguration;
     dim3 grid((p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM), p.hq, p.B);
     prof_begin(KID_FULL, st);
     kern<<<grid, PP_THREADS, C::SMEM, st>>>(mq, mk, mv, p, (__nv_bfloat16*)out, lse);
