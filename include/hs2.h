@@ -206,8 +206,10 @@ hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launche
 
 /* Diagnostics: evaluate the library's exp2 implementations at n device points
  * x: y[0..n) = hardware ex2, y[n..2n) = degree-3 polynomial, y[2n..3n) =
- * degree-5 polynomial (the FMA-pipe 2^x used beside the hardware unit in the
- * softmax and selection kernels).  Asynchronous on `stream`. */
+ * degree-5 polynomial, y[3n..4n) and y[4n..5n) = the two-lane packed degree-5
+ * form at (x, x/2) (the FMA-pipe 2^x used beside the hardware unit in the
+ * softmax and selection kernels).  y holds 5n floats.  Asynchronous on
+ * `stream`. */
 hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t stream);
 
 /* 1 when the library was built with device-side input checks (HS2_CHECKED). */

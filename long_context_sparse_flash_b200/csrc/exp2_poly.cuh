@@ -11,6 +11,8 @@
 // give 0 (also -inf); inputs must stay below 127.
 #pragma once
 
+#include "hs2_common.cuh"
+
 namespace hs2 {
 
 // degree 3: max relative error 1.136e-04 (float64 eval), 1.136e-04 (float32 Horner)
@@ -34,6 +36,25 @@ __device__ __forceinline__ float exp2_poly(float x) {
                             2.402223796e-01f), f, 6.931468844e-01f), f, 1.0f);
     }
     return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two lanes at once: the same steps with packed fp32x2 adds and FMAs (the
+// clamp and the exponent insertion stay per lane).
+__device__ __forceinline__ float2 exp2_poly5_x2(float2 x) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    x.x = fmaxf(x.x, -127.0f);
+    x.y = fmaxf(x.y, -127.0f);
+    const float2 rnd = make_float2(kRound, kRound), nrnd = make_float2(-kRound, -kRound);
+    const float2 t = fadd2(x, rnd);
+    const float2 n = fadd2(t, nrnd);
+    const float2 f = fsub2(x, n);
+    float2 p = ffma2(make_float2(1.321867225e-03f, 1.321867225e-03f), f, make_float2(9.671698324e-03f, 9.671698324e-03f));
+    p = ffma2(p, f, make_float2(5.550893024e-02f, 5.550893024e-02f));
+    p = ffma2(p, f, make_float2(2.402223796e-01f, 2.402223796e-01f));
+    p = ffma2(p, f, make_float2(6.931468844e-01f, 6.931468844e-01f));
+    p = ffma2(p, f, make_float2(1.0f, 1.0f));
+    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
 }
 
 }  // namespace hs2

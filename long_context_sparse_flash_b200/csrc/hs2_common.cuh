@@ -118,6 +118,15 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
     asm("mov.b64 {%0, %1}, %2;\n" : "=f"(r.x), "=f"(r.y) : "l"(d));
     return r;
 }
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+    uint64_t d;
+    asm("{\n .reg .b64 ra, rb;\n mov.b64 ra, {%1, %2};\n mov.b64 rb, {%3, %4};\n sub.rn.f32x2 %0, ra, rb;\n}\n"
+        : "=l"(d)
+        : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;\n" : "=f"(r.x), "=f"(r.y) : "l"(d));
+    return r;
+}
 // max(a, b, c) in one instruction (sm_100a three-input form).
 __device__ __forceinline__ float fmax3f(float a, float b, float c) {
     float d;

@@ -12,6 +12,10 @@ __global__ void exp2_selftest_kernel(const float* __restrict__ x, float* __restr
     y[i] = ex2(v);
     y[n + i] = exp2_poly<3>(v);
     y[2 * n + i] = exp2_poly<5>(v);
+    // the packed form, fed (x, x/2) so both lanes see varied inputs
+    const float2 r = exp2_poly5_x2(make_float2(v, 0.5f * v));
+    y[3 * n + i] = r.x;
+    y[4 * n + i] = r.y;
 }
 }  // namespace
 }  // namespace hs2

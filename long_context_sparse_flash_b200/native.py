@@ -194,11 +194,12 @@ def hs2_full_attn_select_static(shape, q, k, v, out, lse, idx, stream=None, chec
 
 
 def hs2_selftest_exp2(x: torch.Tensor, stream=None):
-    """(hardware ex2, degree-3, degree-5) evaluations of 2^x on the device."""
+    """(hardware ex2, degree-3, degree-5, packed degree-5 at x, packed degree-5
+    at x/2) evaluations of 2^x on the device."""
     n = x.numel()
-    y = torch.empty(3 * n, dtype=torch.float32, device=x.device)
+    y = torch.empty(5 * n, dtype=torch.float32, device=x.device)
     _check(load().hs2_selftest_exp2(_ptr(x), _ptr(y), int(n), _stream(stream)), "hs2_selftest_exp2")
-    return y[:n], y[n:2 * n], y[2 * n:]
+    return tuple(y[u * n:(u + 1) * n] for u in range(5))
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):

@@ -13,8 +13,14 @@ pytestmark = pytest.mark.gpu
 def test_exp2_polynomials_error_bounds():
     xs = torch.cat([torch.linspace(-126.0, 20.0, 400001), torch.arange(-126, 21, dtype=torch.float32),
                     torch.tensor([-127.5, -200.0, float("-inf")])]).cuda()
-    hw, p3, p5 = (y.cpu().numpy().astype(np.float64) for y in nv.hs2_selftest_exp2(xs))
+    hw, p3, p5, q5, q5h = (y.cpu().numpy().astype(np.float64) for y in nv.hs2_selftest_exp2(xs))
     x = xs.cpu().numpy().astype(np.float64)
+    # the packed two-lane form computes the same function, bit for bit
+    assert np.array_equal(q5, p5)
+    xh = (xs * 0.5).cpu().numpy().astype(np.float64)
+    okh = xh >= -125.0
+    assert np.abs(q5h[okh] / np.exp2(xh[okh]) - 1).max() < 3e-7
+    assert np.all(q5h[xh < -127.0] == 0)
     ref = np.exp2(x)
     ok = x >= -125.0  # normal results
     rel = lambda y: np.abs(y[ok] / ref[ok] - 1)
