@@ -37,6 +37,10 @@ from long_context_sparse_flash_b200 import workloads as wl  # noqa: E402
 METRIC = "query tokens/s (full-attn+select + sparse-reuse layers) and % of TC/HBM roofline"
 UNIT = "query tokens/s"
 FLUSH_BYTES = 256 << 20  # > 126 MB L2
+# a call whose K/V (both tensors) is at most this large keeps it in the 126 MB
+# L2 between the sparse layer's gathers: that kernel is then bound by L2 gather
+# bandwidth, not by HBM
+L2_RESIDENT_BYTES = 96 << 20
 
 
 def peaks():
@@ -64,7 +68,8 @@ def kernel_work(w: wl.Workload):
         "full_attn": dict(bound="tensor", flops=f["full_flops"]),
         "decode_attn": dict(bound="hbm", bytes=f["kv_bytes"] + 2 * f["q_bytes"] + 4 * n_rows * Hq),
         # gathered K/V rows + q + out + idx, per layer
-        "sparse_attn": dict(bound="hbm", bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
+        "sparse_attn": dict(bound="l2" if f["kv_bytes"] <= L2_RESIDENT_BYTES else "hbm",
+                            bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
     }
     if w.decode:
         # decode: the attention pass stores each candidate's G scaled logits (fp32); the score
@@ -78,6 +83,28 @@ def kernel_work(w: wl.Workload):
         # prefill: the filtered sweep recomputes QK^T over every candidate of every query
         work["select_filter"] = dict(bound="tensor", flops=f["select_qk_flops"])
     return work
+
+
+def measure_l2_gather(dev, reps: int = 5) -> float:
+    """GB/s of a random 256-byte-row gather from a 64 MiB L2-resident buffer
+    (the sparse layer's access pattern), measured here with the library's probe."""
+    g = torch.Generator().manual_seed(7)
+    rows = torch.randint(0, 255, (64 << 20,), dtype=torch.uint8, generator=g).to(dev)
+    order = torch.randint(0, (64 << 20) // 256, (1 << 22,), dtype=torch.int32, generator=g).to(dev)
+    sink = torch.zeros(4, dtype=torch.int32, device=dev)
+    passes = 4
+    for _ in range(3):
+        nv.hs2_gather_probe(rows, order, passes, sink)
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(st)
+    for _ in range(reps):
+        nv.hs2_gather_probe(rows, order, passes, sink)
+    e1.record(st)
+    e1.synchronize()
+    ms = e0.elapsed_time(e1) / reps
+    return order.numel() * 256.0 * passes / (ms / 1e3) / 1e9
 
 
 def source_sha(path: str) -> str:
@@ -312,6 +339,9 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
         if wk["bound"] == "tensor":
             achieved = wk["flops"] * calls / (ms / 1e3) / 1e12
             peak, unit = pk["tc_sustained"], "TFLOP/s"
+        elif wk["bound"] == "l2":
+            achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
+            peak, unit = round(pk["l2_gather"], 1), "GB/s"
         else:
             achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
             peak, unit = pk["hbm"], "GB/s"
@@ -323,9 +353,11 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
     p = per[top]
     launches_total = prof[top][1]
     traffic = dram_traffic(top, w.name)
-    rf = {"kernel": top, "bound": "hbm" if p["bound"] == "hbm" else "tensor", "achieved": p["achieved"],
+    src = {"tensor": pk["src"] + " (sustained bf16)", "hbm": pk["src"] + " (copy GB/s)",
+           "l2": "measured here (random 256-byte-row gather from a 64 MiB L2-resident buffer, hs2_gather_probe)"}
+    rf = {"kernel": top, "bound": p["bound"], "achieved": p["achieved"],
           "peak": p["peak"], "unit": p["unit"], "frac": p["frac"],
-          "peak_source": pk["src"] + (" (sustained bf16)" if p["bound"] == "tensor" else " (copy GB/s)"),
+          "peak_source": src[p["bound"]],
           "launches_per_step": launches_total / K, "traffic": traffic,
           "share_of_step": None}
     return rf, per
@@ -368,6 +400,8 @@ def run_ours(args):
                "d2h_bytes_per_step": bo, "ms_per_step": round(e_total / args.steps, 3)}
 
     pk = peaks()
+    if any(wk["bound"] == "l2" for wk in kernel_work(w).values()):
+        pk["l2_gather"] = measure_l2_gather(dev)
     rf, per_kernel = roofline(w, prof, args.steps, pk)
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)

@@ -212,6 +212,19 @@ hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launche
  * `stream`. */
 hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t stream);
 
+/* Diagnostics: the gather-bandwidth probe behind the sparse layer's roofline
+ * (the sparse layer reads whole 256-byte K/V rows in data-dependent order).
+ * Reads, `passes` times, the 256-byte rows rows[order[u]] (u < n_order) of
+ * `rows` (device, n_rows x 256 bytes, 16-byte aligned) with 16-byte loads,
+ * sixteen in flight per thread, on (SM count x 8) CTAs of 256 threads; indices
+ * outside [0, n_rows) are skipped.  `sink` (device, 16 bytes, 16-byte aligned)
+ * is written only in a case that keeps the loads alive and is practically never
+ * taken.  The caller times the call on `stream`; bytes read = passes *
+ * n_order * 256.  Requires n_order > 0, n_order % 32 == 0, passes >= 1, else
+ * HS2_ERR_INVALID_ARG.  Not part of the method (no counterpart in the paper). */
+hs2_status hs2_gather_probe(const void* rows, int64_t n_rows, const int32_t* order, int64_t n_order,
+                            int32_t passes, void* sink, hs2_stream_t stream);
+
 /* 1 when the library was built with device-side input checks (HS2_CHECKED). */
 int hs2_is_checked_build(void);
 

@@ -27,3 +27,53 @@ extern "C" hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_str
     hs2::count_launch();
     return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
+
+namespace hs2 {
+namespace {
+// Each warp reads 32 rows of 256 bytes per step (two rows per 16-byte load
+// instruction, sixteen loads in flight per thread); rows whose index is out of
+// range are skipped.
+__global__ void __launch_bounds__(256) gather_probe_kernel(const uint4* __restrict__ rows, int64_t n_rows,
+                                                           const int32_t* __restrict__ order, int64_t n_chunks,
+                                                           int64_t n_steps, uint4* __restrict__ sink) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    uint4 acc = make_uint4(0u, 0u, 0u, 0u);
+    for (int64_t s = warp0; s < n_steps; s += n_warps) {
+        const int64_t c = s % n_chunks;
+        uint4 v[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const int32_t r = order[32 * c + 2 * u + (lane >> 4)];
+            v[u] = (r >= 0 && r < n_rows) ? __ldcg(rows + (int64_t)r * 16 + (lane & 15)) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            acc.x ^= v[u].x;
+            acc.y ^= v[u].y;
+            acc.z ^= v[u].z;
+            acc.w ^= v[u].w;
+        }
+    }
+    if (acc.x == 0x9e3779b9u && acc.y == 0x7f4a7c15u) *sink = acc;  // keeps the loads; practically never taken
+}
+}  // namespace
+}  // namespace hs2
+
+extern "C" hs2_status hs2_gather_probe(const void* rows, int64_t n_rows, const int32_t* order, int64_t n_order,
+                                       int32_t passes, void* sink, hs2_stream_t stream) {
+    if (rows == nullptr || order == nullptr || sink == nullptr || n_rows <= 0 || n_order <= 0 || n_order % 32 != 0 ||
+        passes < 1)
+        return HS2_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(rows) & 15u) != 0 || (reinterpret_cast<uintptr_t>(sink) & 15u) != 0)
+        return HS2_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return HS2_ERR_CUDA;
+    const int64_t n_chunks = n_order / 32;
+    hs2::gather_probe_kernel<<<sms * 8, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<const uint4*>(rows), n_rows, order, n_chunks, n_chunks * passes, reinterpret_cast<uint4*>(sink));
+    hs2::count_launch();
+    return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}

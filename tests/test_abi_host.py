@@ -138,3 +138,15 @@ def test_binding_refuses_host_tensors():
     q = torch.zeros(1, 8, 4, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         nv.sparse_attn(q, q[:, :2], q[:, :2], torch.zeros(1, 2, 4, 1, dtype=torch.int32), window=2)
+
+
+def test_gather_probe_argument_checks():
+    """The diagnostic gather probe rejects bad sizes and pointers on the host."""
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    assert L.hs2_gather_probe(None, 16, FAKE, 32, 1, FAKE, None) == 1
+    assert L.hs2_gather_probe(FAKE, 16, FAKE, 16, 1, FAKE, None) == 1   # n_order not a multiple of 32
+    assert L.hs2_gather_probe(FAKE, 16, FAKE, 32, 0, FAKE, None) == 1   # passes < 1
+    assert L.hs2_gather_probe(FAKE, 0, FAKE, 32, 1, FAKE, None) == 1    # no rows
+    assert L.hs2_gather_probe(ctypes.c_void_p((1 << 40) + 4), 16, FAKE, 32, 1, FAKE, None) == 1  # misaligned
+    assert nv.hs2_launch_count() == before

@@ -31,3 +31,18 @@ def test_exp2_polynomials_error_bounds():
     assert np.all(p3[ints] == ref[ints]) and np.all(p5[ints] == ref[ints])  # exact powers of two
     low = x < -127.0
     assert np.all(p3[low] == 0) and np.all(p5[low] == 0)
+
+
+def test_gather_probe_reads_and_skips_bad_indices():
+    """The gather probe behind the sparse layer's roofline runs, counts as a launch,
+    and tolerates out-of-range indices (skipped on the device)."""
+    rows = torch.ones(1 << 20, dtype=torch.uint8, device="cuda")  # 4096 rows of 256 bytes
+    order = torch.randint(0, 4096, (4096,), dtype=torch.int32, device="cuda")
+    order[::97] = -5
+    order[::89] = 1 << 30
+    sink = torch.zeros(4, dtype=torch.int32, device="cuda")
+    before = nv.hs2_launch_count()
+    nv.hs2_gather_probe(rows, order, 2, sink)
+    torch.cuda.synchronize()
+    assert nv.hs2_launch_count() == before + 1
+    assert torch.all(sink == 0)  # the keep-alive store is not taken
