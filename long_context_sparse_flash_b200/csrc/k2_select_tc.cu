@@ -12,9 +12,13 @@
 // and the epilogue thread that owns TMEM lane r (= key j) forms the group sum
 // for each of the 32 queries inside one thread.  Three passes keep the work
 // on chip and exact:
-//   SAMPLE  8 evenly spaced tiles per CTA -> 1024 sample scores per row
-//   (k2_thresh_kernel) per row, an estimate tau of a score that about 2 K
-//           candidates exceed: the r-th largest sample, r = 2 K s/n
+//   SAMPLE  1024 keys at a fixed stride S = kv_len / 1024 over the whole cache
+//           (a strided tensor-map view, 8 tiles of 128): sample scores spread
+//           over every segment of the context, not a few contiguous runs
+//   (k2_thresh_kernel) per row, a bound tau that at least K candidates
+//           exceed with high probability: the r-th largest sample, r = L +
+//           4.5 sqrt(L) + 2, where L = K s/n is the expected number of samples
+//           above the K-th best candidate
 //   FILTER  every tile; candidates at or above the row's bound are appended,
 //           in ascending j, to the row's survivor list in this SM's slot of
 //           the workspace (L2-resident).  A list about to overflow is
@@ -90,6 +94,7 @@ struct SelArgs {
     int i_begin, i_count;   // query chunk of this call
     int cmax;               // survivor list capacity per row
     int slot_by_block;      // 1: slot = block id (small grids); 0: slot = %smid (one CTA per SM)
+    int64_t sample_stride;  // S: the sampling pass reads keys 0, S, 2S, ...
 };
 
 __device__ __forceinline__ uint32_t smid() {
@@ -240,11 +245,11 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     }
     const int cmax = a.cmax;
     uint2* lists = a.slots + (int64_t)slot * SL_QT * cmax;
-    const int n_tiles = MODE == MODE_SAMPLE ? min(SL_SAMPLE_TILES, n_ct) : n_ct;
-    auto tile_of = [&](int it) -> int {
-        if (MODE != MODE_SAMPLE) return it;
-        return (int)(((2 * (int64_t)it + 1) * n_ct) / (2 * n_tiles));
-    };
+    // sampling pass: tile it holds keys S (128 it + u), u < 128, of the strided view
+    const int64_t S = a.sample_stride;
+    const int64_t n_sb = cand_end > 0 ? (cand_end + S - 1) / S : 0;  // sampled keys below the candidate limit
+    const int n_tiles = MODE == MODE_SAMPLE ? (int)min((int64_t)SL_SAMPLE_TILES, (n_sb + SL_BN - 1) / SL_BN) : n_ct;
+    auto tile_of = [&](int it) -> int { return it; };
 
     // row state
     if (tid < SL_QT) {
@@ -348,7 +353,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         for (int it = 0; it < n_tiles; ++it) {
             const int sb = it & 1;
             const int64_t jb = (int64_t)tile_of(it) * SL_BN;
-            const int64_t j = jb + et;
+            const int64_t j = MODE == MODE_SAMPLE ? S * (jb + et) : jb + et;
             // one thread per warpgroup waits (bounded) and the named barrier hands
             // the result to its four warps, so they leave the loop together
             if (et == 0) okv[wg * 2 + (it & 1)] = tc::mbar_wait(bar(SB_SFULL + sb), (it >> 1) & 1, ab, p.err, KID_SCORE, 5);
@@ -484,13 +489,9 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 // valid samples of the row: sampled keys j <= t - window
                 const int q = wg * QH + et;
                 const int64_t t = pos0 + q0 + q;
-                int cnt = 0;
-                for (int it2 = 0; it2 < n_tiles; ++it2) {
-                    const int64_t jb2 = (int64_t)tile_of(it2) * SL_BN;
-                    const int64_t hi = t - p.window - jb2 + 1;
-                    cnt += (int)(hi < 0 ? 0 : (hi > SL_BN ? SL_BN : hi));
-                }
-                a.s_valid[row0 + q] = cnt;
+                // sampled keys S b <= t - window among the n_tiles * 128 read
+                const int64_t nv = t >= p.window ? (t - p.window) / S + 1 : 0;
+                a.s_valid[row0 + q] = (int)min(nv, (int64_t)n_tiles * SL_BN);
             }
         } else if (ok) {
             // exact top-min(K, n) of every active row, ascending j, -1 padded
@@ -538,8 +539,9 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     }
 }
 
-// Per row: tau = the r-th largest sample, r = ceil(2 K s / n) (s valid
-// samples, n candidates); 0 when every candidate fits the survivor list.
+// Per row: tau = the r-th largest sample, r = ceil(L + 4.5 sqrt(L) + 2) with
+// L = K s / n (s valid samples, n candidates); 0 when every candidate fits the
+// survivor list, or when r exceeds s.
 __global__ void __launch_bounds__(128) k2_thresh_kernel(Problem p, SelArgs a) {
     __shared__ uint32_t hist[4][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -553,8 +555,12 @@ __global__ void __launch_bounds__(128) k2_thresh_kernel(Problem p, SelArgs a) {
     const int s = a.s_valid[row];
     float tau = 0.f;
     if (n > a.cmax / 2 && s > 0) {
-        int64_t r = (2 * (int64_t)p.topk * s + n - 1) / n;
-        if (r < 1) r = 1;
+        // L = samples expected above the K-th best candidate; the number that are
+        // is about Poisson(L), so r = L + 4.5 sqrt(L) + 2 is reached with
+        // probability about 1e-5 (the retry pass covers those rows), while about
+        // r n / s candidates pass and the list compaction absorbs any overflow
+        const float lam = (float)p.topk * (float)s / (float)n;
+        int64_t r = (int64_t)ceilf(lam + 4.5f * sqrtf(lam) + 2.f);
         if (r <= s) {
             uint32_t kth, need_eq;
             warp_kth(reinterpret_cast<const uint32_t*>(a.samples + row * SL_SPR), 1, SL_SPR, (uint32_t)r, hist[warp],
@@ -595,12 +601,27 @@ cudaError_t launch_mode(const Problem& p, const CUtensorMap& mq, const CUtensorM
     return cudaGetLastError();
 }
 
+// K seen with rows S apart: (D, kv_len / S, B * H_kv), box (64, 128, 1).
+bool make_strided_map(CUtensorMap* m, const void* base, int D, int64_t kv_len, int64_t S, int64_t z) {
+    auto fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)(kv_len / S), (cuuint64_t)z};
+    cuuint64_t strides[2] = {(cuuint64_t)(S * D * 2), (cuuint64_t)(kv_len * D * 2)};
+    cuuint32_t box[3] = {64, (cuuint32_t)SL_BN, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 template <int D, int G>
 cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
-    CUtensorMap mq, mk;
-    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
+    CUtensorMap mq, mk, mks;
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128) ||
+        !make_strided_map(&mks, k, D, p.kv_len, a.sample_stride, (int64_t)p.B * p.hkv))
         return cudaErrorInvalidValue;
-    cudaError_t e = launch_mode<D, G, MODE_SAMPLE>(p, mq, mk, a, st);
+    cudaError_t e = launch_mode<D, G, MODE_SAMPLE>(p, mq, mks, a, st);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)p.B * p.hkv * a.i_count;
     prof_begin(KID_THRESH, st);
@@ -650,6 +671,7 @@ cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, con
     SelArgs a;
     int n_slots;
     select_tc_geometry(p, i_count, n_cand_max, a.cmax, n_slots, a.slot_by_block);
+    a.sample_stride = p.kv_len / (SL_SAMPLE_TILES * SL_BN) > 1 ? p.kv_len / (SL_SAMPLE_TILES * SL_BN) : 1;
     a.lse = lse;
     a.idx = idx;
     a.slots = reinterpret_cast<uint2*>(base);
