@@ -1,0 +1,68 @@
+"""The multi-rank plumbing of bench.py on CPU: world size 2 over gloo (no GPU).
+Ranks run independent replicas (different seeds, no data exchange); the only
+collectives are the barrier and the max over ranks of the timed region; the
+reference arm runs on rank 0 alone."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, ws: int, port: int, q):
+    import datetime
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=60))
+    try:
+        import bench
+        from long_context_sparse_flash_b200 import workloads as wl
+        w = wl.WORKLOADS["tiny"]
+        # independent replicas: each rank draws its own inputs
+        inp = wl.make_inputs(w, "cpu", seed=bench.replica_seed(w, rank), with_sparse=False)
+        digest = float(inp["q"].float().sum())
+        bench.barrier(ws)
+        slowest = bench.max_over_ranks(10.0 + rank, ws)  # rank r "took" 10 + r ms
+        value = bench.job_value(w.query_tokens, ws, 3, 3 * slowest)
+        q.put((rank, digest, slowest, value))
+    finally:
+        torch.distributed.destroy_process_group()
+
+
+def test_two_ranks_over_gloo():
+    ws, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=180)
+    assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
+    res = sorted(q.get(timeout=5) for _ in range(ws))
+    digests = [r[1] for r in res]
+    assert digests[0] != digests[1]                     # different sequences per rank
+    assert all(r[2] == 11.0 for r in res)               # every rank sees the slowest rank's time
+    from long_context_sparse_flash_b200 import workloads as wl
+    tokens = wl.WORKLOADS["tiny"].query_tokens
+    assert all(abs(r[3] - tokens * ws / 11e-3) < 1e-6 * r[3] for r in res)  # all ranks' tokens / slowest time
+
+
+def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
+    import argparse
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    args = argparse.Namespace(workload="tiny", ref_rows=1, warmup=3, steps=2, gpus=2)
+    assert bench.run_reference(args) is None
+    assert capsys.readouterr().out == ""
