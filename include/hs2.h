@@ -216,8 +216,8 @@ hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t strea
  * (the sparse layer reads whole 256-byte K/V rows in data-dependent order).
  * Reads, `passes` times, the 256-byte rows rows[order[u]] (u < n_order) of
  * `rows` (device, n_rows x 256 bytes, 16-byte aligned) with 16-byte loads,
- * sixteen in flight per thread, on (SM count x 8) CTAs of 256 threads; indices
- * outside [0, n_rows) are skipped.  `sink` (device, 16 bytes, 16-byte aligned)
+ * sixteen in flight per thread, on (SM count x 8) CTAs of 256 threads; an
+ * index outside [0, n_rows) reads row 0 instead.  `sink` (device, 16 bytes, 16-byte aligned)
  * is written only in a case that keeps the loads alive and is practically never
  * taken.  The caller times the call on `stream`; bytes read = passes *
  * n_order * 256.  Requires n_order > 0, n_order % 32 == 0, passes >= 1, else

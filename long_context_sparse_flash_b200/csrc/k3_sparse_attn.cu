@@ -5,10 +5,13 @@
 // most-recent window, all from the one shared cache).
 //
 // One CTA = one (sequence, query, KV group); its G heads share every gathered
-// K/V row.  The attended rows S = idx U window are listed in shared memory,
-// cut into 16-row tiles and gathered with 16-byte cp.async into double-buffered,
-// swizzled staging.  One warp per CTA: the gather is latency-bound, and many
-// small CTAs per SM (about eleven) keep the most tiles in flight.  Per tile:
+// K/V row.  The attended rows S = idx U window (the selection's valid prefix,
+// then the window) are cut into 16-row tiles and gathered with 16-byte
+// cp.async into a ring of SP_STAGES swizzled stages; each tile's row indices
+// are fetched into registers a tile before its copies are issued, so shared
+// memory holds only the staging.  One warp per CTA: the gather is
+// latency-bound, and many small CTAs per SM keep the most tiles in flight.
+// Per tile:
 //   S^T (16 keys x 8 heads) = K_tile Q^T      mma.sync m16n8k16, A = K rows
 //   P^T = 2^(S^T - m) per head column, online softmax over the warp's tiles
 //   O^T (D x 8 heads) += V_tile^T P^T         A = V^T via ldmatrix.trans,
@@ -23,12 +26,13 @@ namespace hs2 {
 namespace {
 
 constexpr int SP_WARPS = 1;  // more, smaller CTAs per SM hide the gather latency best
+constexpr int SP_STAGES = 2;  // tiles in the staging ring
 
 template <int D>
 struct K3Cfg {
     static constexpr int CH = D / 8;
     static constexpr int TILE_BYTES = 16 * D * 2;                 // one 16-row K (or V) tile
-    static constexpr int WARP_BYTES = 2 * 2 * TILE_BYTES;         // 2 stages x (K, V)
+    static constexpr int WARP_BYTES = SP_STAGES * 2 * TILE_BYTES;  // stages x (K, V)
     static constexpr int STAGE_BYTES = SP_WARPS * WARP_BYTES;
     static constexpr int COMB_BYTES = SP_WARPS * (D * 8 + 16) * 4;  // per warp: O^T, m, l
     static constexpr int FIXED = STAGE_BYTES > COMB_BYTES ? STAGE_BYTES : COMB_BYTES;
@@ -42,8 +46,6 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
                                                                    __nv_bfloat16* __restrict__ out) {
     using C = K3Cfg<D>;
     extern __shared__ __align__(128) uint8_t smem[];
-    int32_t* list = reinterpret_cast<int32_t*>(smem + C::FIXED);
-    __shared__ int s_nsel;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int64_t pos0 = seq_pos0(p, b, KID_SPARSE);
@@ -51,14 +53,12 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     const int64_t w0 = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
     const int nwin = (int)(t - w0 + 1);
 
-    // attended list: the selection's valid prefix, then the window
-    if (tid == 0) s_nsel = 0;
-    __syncthreads();
+    // attended rows: the selection's valid prefix (its length counted here),
+    // then the window
     const int32_t* irow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
     int cnt = 0;
     for (int r = tid; r < p.topk; r += SP_WARPS * 32) {
         const int32_t j = irow[r];
-        list[r] = j;
         cnt += j >= 0;
 #ifdef HS2_CHECKED
         const bool bad_range = j < -1 || (int64_t)j > t - p.window;
@@ -71,13 +71,19 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
-    if (lane == 0) atomicAdd(&s_nsel, cnt);
-    __syncthreads();
-    const int nsel = s_nsel;
-    for (int r = tid; r < nwin; r += SP_WARPS * 32) list[nsel + r] = (int32_t)(w0 + r);
-    __syncthreads();
+    static_assert(SP_WARPS == 1, "the row count is a warp reduction");
+    const int nsel = cnt;
     const int n = nsel + nwin;
     const int n_mt = (n + 15) / 16;
+    // row index of attended position li, -1 past the end or when invalid
+    auto row_of = [&](int li) -> int32_t {
+        int32_t j = -1;
+        if (li < nsel)
+            j = irow[li];
+        else if (li < n)
+            j = (int32_t)(w0 + (li - nsel));
+        return (j >= 0 && (int64_t)j <= t) ? j : -1;
+    };
 
     // Q^T B fragments: column = head (lane / 4) of the group, zero beyond G
     uint32_t qb[D / 16][2];
@@ -97,14 +103,11 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     const __nv_bfloat16* vg = v + ((int64_t)(b * p.hkv + g) * p.kv_len) * D;
     const uint32_t s_w = smem_u32(smem) + warp * C::WARP_BYTES;
     // Tile loads: lanes 0-15 copy one row and lanes 16-31 the next (16-byte
-    // chunk = lane % 16 for D = 128), eight row pairs per 16-row tile.  A lane
-    // reads the tile's row indices once and takes each row's index by shuffle;
+    // chunk = lane % 16 for D = 128), eight row pairs per 16-row tile.  Lane l
+    // holds the index of the tile's row l % 16 and the others take it by shuffle;
     // the swizzled chunk is (lane chunk ^ row parity) ^ (2 * it mod 8).
-    auto load_tile = [&](int mt, int stage) {
+    auto load_tile = [&](int stage, int32_t myj) {
         const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES;
-        const int li = mt * 16 + (lane & 15);
-        const int32_t jl = li < n ? list[li] : -1;
-        const int32_t myj = (jl >= 0 && (int64_t)jl <= t) ? jl : -1;
         constexpr int RPI = 32 / C::CH;  // rows per iteration (2 for D = 128, 4 for D = 64)
         const int hi = lane / C::CH, ch = lane % C::CH;
 #pragma unroll
@@ -123,13 +126,25 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     for (int dt = 0; dt < D / 16; ++dt) acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
     float m_c[2] = {-INFINITY, -INFINITY}, l_c[2] = {0.f, 0.f};
 
-    int mt = warp, stage = 0;
-    if (mt < n_mt) load_tile(mt, 0);
-    cp_async_commit();
-    for (; mt < n_mt; mt += SP_WARPS, stage ^= 1) {
-        if (mt + SP_WARPS < n_mt) load_tile(mt + SP_WARPS, stage ^ 1);
+    // ring: tile mt lives in stage mt % SP_STAGES; tiles mt + 1 .. mt + SP_STAGES - 1
+    // are in flight while tile mt is computed.  jr[u] = row index of tile mt + u
+    // (lane l: row l % 16), u < SP_STAGES; the next one is fetched a tile ahead.
+    const int r16 = lane & 15;
+    int32_t jr[SP_STAGES];
+#pragma unroll
+    for (int u = 0; u < SP_STAGES; ++u) jr[u] = row_of(u * 16 + r16);
+#pragma unroll
+    for (int u = 0; u < SP_STAGES - 1; ++u) {
+        if (u < n_mt) load_tile(u, jr[u]);
         cp_async_commit();
-        cp_async_wait<1>();
+    }
+    int stage = 0;
+    for (int mt = 0; mt < n_mt; ++mt) {
+        const int32_t j_next = row_of((mt + SP_STAGES) * 16 + r16);
+        const int lstage = (stage + SP_STAGES - 1) % SP_STAGES;
+        if (mt + SP_STAGES - 1 < n_mt) load_tile(lstage, jr[SP_STAGES - 1]);
+        cp_async_commit();
+        cp_async_wait<SP_STAGES - 1>();
         __syncwarp();
         const uint32_t sk = s_w + stage * 2 * C::TILE_BYTES, sv = sk + C::TILE_BYTES;
 
@@ -146,13 +161,8 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
         for (int e = 0; e < 4; ++e) c[e] += c2[e];
         // rows lane/4 and lane/4 + 8 of the tile; columns 2*(lane%4) + {0, 1}
         bool row_ok[2];
-        {
-            const int li = mt * 16 + (lane & 15);
-            const int32_t jl = li < n ? list[li] : -1;
-            const bool okl = jl >= 0 && (int64_t)jl <= t;
-            row_ok[0] = __shfl_sync(0xffffffffu, okl, lane >> 2);
-            row_ok[1] = __shfl_sync(0xffffffffu, okl, (lane >> 2) + 8);
-        }
+        row_ok[0] = __shfl_sync(0xffffffffu, jr[0], lane >> 2) >= 0;
+        row_ok[1] = __shfl_sync(0xffffffffu, jr[0], (lane >> 2) + 8) >= 0;
         float s[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) s[e] = row_ok[e >> 1] ? c[e] * p.scale_log2 : -INFINITY;
@@ -193,6 +203,10 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
             mma16816(acc[dt], a, pb);
         }
         __syncwarp();
+#pragma unroll
+        for (int u = 0; u + 1 < SP_STAGES; ++u) jr[u] = jr[u + 1];
+        jr[SP_STAGES - 1] = j_next;
+        stage = stage + 1 == SP_STAGES ? 0 : stage + 1;
     }
     cp_async_wait<0>();
 
@@ -244,7 +258,7 @@ template <int D, int G>
 cudaError_t launch_sparse_dg(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
                              void* out, cudaStream_t st) {
     using C = K3Cfg<D>;
-    const int smem = C::FIXED + (p.topk + p.window) * 4;
+    const int smem = C::FIXED;
     auto kern = k3_sparse_kernel<D, G>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;

@@ -35,7 +35,7 @@ def test_exp2_polynomials_error_bounds():
 
 def test_gather_probe_reads_and_skips_bad_indices():
     """The gather probe behind the sparse layer's roofline runs, counts as a launch,
-    and tolerates out-of-range indices (skipped on the device)."""
+    and tolerates out-of-range indices (read as row 0 on the device)."""
     rows = torch.ones(1 << 20, dtype=torch.uint8, device="cuda")  # 4096 rows of 256 bytes
     order = torch.randint(0, 4096, (4096,), dtype=torch.int32, device="cuda")
     order[::97] = -5
