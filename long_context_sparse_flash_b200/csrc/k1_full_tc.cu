@@ -25,6 +25,7 @@
 // through the error word, drains its own copies, frees its TMEM and exits.
 #include <cudaTypedefs.h>
 
+#include "exp2_poly.cuh"
 #include "hs2_kernels.h"
 #include "tc05.cuh"
 
@@ -130,15 +131,23 @@ __device__ __forceinline__ float tile_max(const float* s) {
 
 // p = 2^(s * scale - m) for the row's 128 scores, two lanes per instruction,
 // packed to bf16 pairs in place (s[0..63] hold the pairs afterwards); returns the
-// row sum of the fp32 values (four packed accumulators).
+// row sum of the fp32 values (four packed accumulators).  One pair in PP_POLY_EVERY
+// is computed on the FMA pipe (degree-5 polynomial, the accuracy of the hardware
+// ex2): the special-function unit's ex2 rate otherwise equals the tensor core's
+// rate for this kernel, so the unit would cap it.
+constexpr int PP_POLY_EVERY = 8;
 __device__ __forceinline__ float exp_pack_tile(float* s, float scale, float m) {
     const float2 sc2 = make_float2(scale, scale), nm2 = make_float2(-m, -m);
     float2 acc[4];
 #pragma unroll
     for (int c = 0; c < PP_BN; c += 2) {
         float2 e = ffma2(make_float2(s[c], s[c + 1]), sc2, nm2);
-        e.x = ex2(e.x);
-        e.y = ex2(e.y);
+        if ((c >> 1) % PP_POLY_EVERY == PP_POLY_EVERY - 1) {
+            e = exp2_poly5_x2(e);
+        } else {
+            e.x = ex2(e.x);
+            e.y = ex2(e.y);
+        }
         const int a4 = (c >> 1) & 3;
         acc[a4] = (c < 8) ? e : fadd2(acc[a4], e);
         s[c >> 1] = __uint_as_float(pack_bf16(e.x, e.y));
