@@ -163,6 +163,9 @@ __global__ void __launch_bounds__(SC_WARPS * 32) k2_score_kernel(Problem p, cons
 constexpr int TK_THREADS = 1024;
 constexpr int TK_WARPS = TK_THREADS / 32;
 constexpr int TK_BINS = 2048;
+constexpr int TK_SAMPLES = 8192;  // keys sampled per row for the threshold
+constexpr int TK_CAP = 8192;      // survivor buffer (keys and indices in shared memory)
+constexpr int TK_DYN_SMEM = 2 * TK_CAP * 4;
 
 struct TopkSmem {
     uint32_t hist[TK_BINS];
@@ -200,29 +203,16 @@ __device__ __forceinline__ void digit_of(int pass, int& shift, uint32_t& mask) {
     mask = pass == 2 ? 1023u : 2047u;
 }
 
-__global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const float* __restrict__ scores,
-                                                             int64_t sstride, int32_t* __restrict__ idx,
-                                                             int i_begin, int i_count) {
-    __shared__ TopkSmem sm;
+// Exact top-k of one row over all n keys in global memory (the fallback):
+// 3-pass radix select for the k-th key, then an ordered pass, indices ascending.
+__device__ void topk_exact_global(const uint32_t* __restrict__ key, int n, int topk, int32_t* __restrict__ orow,
+                                  TopkSmem& sm) {
     const int tid = threadIdx.x, lane = tid & 31;
-    const int qi = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-    const int i = i_begin + qi;
-    const int64_t pos0 = seq_pos0(p, b, KID_TOPK);
-    const int64_t t = pos0 + i;
-    const int64_t n64 = t - p.window + 1;
-    const int n = n64 > 0 ? (int)n64 : 0;
-    int32_t* orow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
-    if (n <= p.topk) {
-        for (int r = tid; r < p.topk; r += TK_THREADS) orow[r] = r < n ? r : -1;
-        return;
-    }
-    const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + ((int64_t)(b * p.hkv + g) * i_count + qi) * sstride);
     const int n4 = n / 4;  // rows start 16-byte aligned (sstride is a multiple of 4)
-
     // radix select: the key value of the topk-th largest (non-negative floats
     // order like their bit patterns), three passes of 11, 11 and 10 bits
     uint32_t prefix = 0, pmask = 0;
-    uint32_t k_rem = (uint32_t)p.topk;
+    uint32_t k_rem = (uint32_t)topk;
 #pragma unroll 1
     for (int pass = 0; pass < 3; ++pass) {
         int shift;
@@ -325,6 +315,188 @@ __global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const fl
     }
 }
 
+
+// Exact radix select over n keys (fp32 bit patterns) of a shared-memory array:
+// the K-th largest key value and how many keys equal to it belong to the top K.
+__device__ void block_kth_shared(const uint32_t* keys, int n, uint32_t K, TopkSmem& sm, uint32_t& kth,
+                                 uint32_t& need_eq) {
+    const int tid = threadIdx.x, lane = tid & 31;
+    uint32_t prefix = 0, pmask = 0, k_rem = K;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        int shift;
+        uint32_t dmask;
+        digit_of(pass, shift, dmask);
+        for (int u = tid; u < TK_BINS; u += TK_THREADS) sm.hist[u] = 0;
+        __syncthreads();
+        for (int base = 0; base < n; base += TK_THREADS) {
+            const int j = base + tid;
+            const bool valid = j < n;
+            const uint32_t x = valid ? keys[j] : 0u;
+            const bool part = valid && (x & pmask) == prefix;
+            const uint32_t act = __ballot_sync(0xffffffffu, part);
+            if (part) {
+                const uint32_t bin = (x >> shift) & dmask;
+                const uint32_t peers = __match_any_sync(act, bin);
+                if (lane == __ffs(peers) - 1) atomicAdd(&sm.hist[bin], (uint32_t)__popc(peers));
+            }
+        }
+        __syncthreads();
+        if (tid < 32) {
+            uint32_t s = 0;
+            const int per = ((int)dmask + 1) / 32;
+            for (int u = 0; u < per; ++u) s += sm.hist[per * (31 - lane) + u];
+            uint32_t incl = s;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const uint32_t excl = incl - s;
+            if (excl < k_rem && k_rem <= incl) {
+                uint32_t above = excl;
+                for (int u = per - 1; u >= 0; --u) {
+                    const uint32_t c = sm.hist[per * (31 - lane) + u];
+                    if (above + c >= k_rem) {
+                        sm.digit = (uint32_t)(per * (31 - lane) + u);
+                        sm.k_rem = k_rem - above;
+                        break;
+                    }
+                    above += c;
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sm.digit << shift;
+        pmask |= dmask << shift;
+        k_rem = sm.k_rem;
+        __syncthreads();
+    }
+    kth = prefix;
+    need_eq = k_rem;
+}
+
+// One row per CTA.  Fast path: a threshold tau from 8192 keys sampled at a
+// fixed stride (the r-th largest, r = L + 4.5 sqrt(L) + 2 with L = K s / n the
+// expected number of samples above the K-th best key; tau = 0 when n fits the
+// survivor buffer), one streaming pass that compacts the keys >= tau, in j
+// order, into shared memory, then the exact select over those survivors.  A
+// row with fewer than K survivors (tau too high) or more than the buffer holds
+// (e.g. many equal scores) takes the exact passes over the whole row instead.
+__global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const float* __restrict__ scores,
+                                                             int64_t sstride, int32_t* __restrict__ idx,
+                                                             int i_begin, int i_count) {
+    __shared__ TopkSmem sm;
+    extern __shared__ __align__(16) uint32_t tk_dyn[];
+    uint32_t* lk = tk_dyn;            // survivor keys (also the samples, before the compaction)
+    uint32_t* lj = tk_dyn + TK_CAP;   // survivor indices
+    const int tid = threadIdx.x;
+    const int qi = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int i = i_begin + qi;
+    const int64_t pos0 = seq_pos0(p, b, KID_TOPK);
+    const int64_t t = pos0 + i;
+    const int64_t n64 = t - p.window + 1;
+    const int n = n64 > 0 ? (int)n64 : 0;
+    int32_t* orow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
+    if (n <= p.topk) {
+        for (int r = tid; r < p.topk; r += TK_THREADS) orow[r] = r < n ? r : -1;
+        return;
+    }
+    const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + ((int64_t)(b * p.hkv + g) * i_count + qi) * sstride);
+
+    // threshold
+    uint32_t tau = 0u;
+    if (n > TK_CAP) {
+        const int stride = n / TK_SAMPLES;  // >= 1
+        for (int u = tid; u < TK_SAMPLES; u += TK_THREADS) lk[u] = key[(int64_t)u * stride];
+        __syncthreads();
+        const float lam = (float)p.topk * (float)TK_SAMPLES / (float)n;
+        const int r = (int)ceilf(lam + 4.5f * sqrtf(lam) + 2.f);
+        if (r < TK_SAMPLES) {
+            uint32_t need_eq;
+            block_kth_shared(lk, TK_SAMPLES, (uint32_t)r, sm, tau, need_eq);
+        }
+        __syncthreads();  // samples consumed before the compaction overwrites them
+    }
+
+    // ordered compaction of the keys >= tau: 16 consecutive keys per thread per
+    // step, their four 16-byte loads issued together
+    constexpr int KPT = 16;
+    uint32_t cnt = 0;
+    for (int base = 0; base < n; base += KPT * TK_THREADS) {
+        const int j0 = base + KPT * tid;
+        uint32_t x[KPT];
+        if (j0 + KPT - 1 < n) {
+#pragma unroll
+            for (int v = 0; v < KPT / 4; ++v) {
+                const uint4 v4 = *reinterpret_cast<const uint4*>(key + j0 + 4 * v);
+                x[4 * v] = v4.x, x[4 * v + 1] = v4.y, x[4 * v + 2] = v4.z, x[4 * v + 3] = v4.w;
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < KPT; ++u) x[u] = (j0 + u < n) ? key[j0 + u] : 0u;
+        }
+        uint32_t ntake = 0;
+#pragma unroll
+        for (int u = 0; u < KPT; ++u) ntake += (j0 + u < n && x[u] >= tau) ? 1u : 0u;
+        uint32_t tot;
+        uint32_t pos = cnt + block_excl_sum(ntake, sm.warp_tot, tot);
+        if (ntake) {
+#pragma unroll
+            for (int u = 0; u < KPT; ++u) {
+                if (j0 + u < n && x[u] >= tau) {
+                    if (pos < (uint32_t)TK_CAP) {
+                        lk[pos] = x[u];
+                        lj[pos] = (uint32_t)(j0 + u);
+                    }
+                    ++pos;
+                }
+            }
+        }
+        cnt += tot;
+        __syncthreads();  // warp_tot is reused by the next step
+    }
+    if (cnt < (uint32_t)p.topk || cnt > (uint32_t)TK_CAP) {
+        topk_exact_global(key, n, p.topk, orow, sm);
+        return;
+    }
+
+    // exact top K among the survivors, then an ordered keep (they are in j order)
+    uint32_t kth, need_eq;
+    block_kth_shared(lk, (int)cnt, (uint32_t)p.topk, sm, kth, need_eq);
+    uint32_t eq_seen = 0, written = 0;
+    for (int base = 0; base < (int)cnt; base += 4 * TK_THREADS) {
+        const int e0 = base + 4 * tid;
+        uint32_t x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = (e0 + u < (int)cnt) ? lk[e0 + u] : 0u;
+        uint32_t neq = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) neq += (e0 + u < (int)cnt && x[u] == kth) ? 1u : 0u;
+        uint32_t eq_tot;
+        uint32_t eq_rank = eq_seen + block_excl_sum(neq, sm.warp_tot, eq_tot);
+        bool take[4];
+        uint32_t ntake = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool valid = e0 + u < (int)cnt;
+            const bool eq = valid && x[u] == kth;
+            take[u] = (valid && x[u] > kth) || (eq && eq_rank < need_eq);
+            eq_rank += eq ? 1u : 0u;
+            ntake += take[u] ? 1u : 0u;
+        }
+        __syncthreads();
+        uint32_t take_tot;
+        uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (take[u]) orow[pos++] = (int32_t)lj[e0 + u];
+        eq_seen += eq_tot;
+        written += take_tot;
+        __syncthreads();
+    }
+}
+
 template <int D, int G>
 cudaError_t launch_score_dg(const Problem& p, const void* q, const void* k, const float* lse, float* scores,
                             int i_begin, int i_count, int64_t sstride, cudaStream_t st) {
@@ -377,9 +549,11 @@ cudaError_t launch_score(const Problem& p, const void* q, const void* k, const f
 
 cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, int32_t* idx, int i_begin,
                         int i_count, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(k2_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_DYN_SMEM);
+    if (e != cudaSuccess) return e;
     dim3 grid(i_count, p.hkv, p.B);
     prof_begin(KID_TOPK, st);
-    k2_topk_kernel<<<grid, TK_THREADS, 0, st>>>(p, scores, sstride, idx, i_begin, i_count);
+    k2_topk_kernel<<<grid, TK_THREADS, TK_DYN_SMEM, st>>>(p, scores, sstride, idx, i_begin, i_count);
     prof_end(st);
     count_launch();
     return cudaGetLastError();

@@ -206,3 +206,18 @@ def test_exact_ties_force_list_compaction():
     assert torch.equal(gpu["idx"], want.expand_as(gpu["idx"]))
     rows = np.array([0, 1, 47, 95])
     P.compare_rows(w, inp, gpu, 0, rows)
+
+
+def test_decode_exact_ties_take_the_full_radix_path():
+    """q = 0 gives every candidate the same score G/(t+1): the sampled threshold
+    then admits all 19873 candidates, more than the survivor buffer holds, so
+    the decode top-k falls back to the exact passes over the whole row; the tie
+    rule fixes the selection to indices 0..K-1."""
+    w = wl.custom("decode_ties", batch=2, n_q=1, q_pos0=19999, kv_len=20000, h_q=32, h_kv=4, head_dim=128,
+                  window=128, topk=1024, n_sparse=1, decode=True, seed=6)
+    inp = wl.make_inputs(w, "cuda")
+    inp["q"].zero_()
+    gpu = P.run_gpu(w, inp)
+    want = torch.arange(w.topk, dtype=torch.int32, device="cuda")
+    assert torch.equal(gpu["idx"], want.expand_as(gpu["idx"]))
+    P.compare_rows(w, inp, gpu, 1, np.array([0]), ts=np.array([w.kv_len - 1]))
