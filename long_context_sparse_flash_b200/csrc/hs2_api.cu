@@ -141,6 +141,13 @@ ScorePlan score_plan(const Problem& p, bool decode) {
 
 hs2_status cuda_status(cudaError_t e) { return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA; }
 
+// Workspace after the header for prefill-shaped calls: the selection scratch,
+// or the full layer's split parts if larger (the two are never live together).
+size_t prefill_body_bytes(const Problem& p, const ScorePlan& sp) {
+    const size_t split = full_tc_split_scratch_bytes(p);
+    return sp.bytes > split ? sp.bytes : split;
+}
+
 hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool decode, const void* q,
                            const void* k, const void* v, void* out, float* lse, int32_t* idx, void* ws,
                            size_t ws_bytes, hs2_stream_t stream) {
@@ -156,7 +163,8 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
         return HS2_ERR_INVALID_ARG;
     const ScorePlan sp = score_plan(p, decode);
     const size_t extra = decode ? decode_scratch_bytes(p) : 0;
-    if (ws_bytes < kHeader + (decode ? (sp.bytes + 255) / 256 * 256 : sp.bytes) + extra) return HS2_ERR_WORKSPACE;
+    const size_t body = decode ? (sp.bytes + 255) / 256 * 256 + extra : prefill_body_bytes(p, sp);
+    if (ws_bytes < kHeader + body) return HS2_ERR_WORKSPACE;
     p.seq_len = seq_len;
     p.err = reinterpret_cast<WsHeader*>(ws);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -171,7 +179,9 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
         e = launch_topk(p, scores, sp.sstride, idx, 0, 1, st);
         return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
     }
-    cudaError_t e = launch_full(p, q, k, v, out, lse, st);
+    // the full layer's split parts (if any) use the selection scratch, which is
+    // only written after the layer's merge has read them (same stream)
+    cudaError_t e = launch_full(p, q, k, v, out, lse, reinterpret_cast<uint8_t*>(ws) + kHeader, ws_bytes - kHeader, st);
     if (e != cudaSuccess) return HS2_ERR_CUDA;
     if (p.topk == 0) return HS2_OK;
     float* scores = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kHeader);
@@ -206,7 +216,7 @@ size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
     switch (entry) {
         case HS2_ENTRY_SPARSE: return kHeader;
         case HS2_ENTRY_FULL_SELECT:
-        case HS2_ENTRY_PREFILL: return kHeader + score_plan(p, false).bytes;
+        case HS2_ENTRY_PREFILL: return kHeader + prefill_body_bytes(p, score_plan(p, false));
         case HS2_ENTRY_DECODE: {
             if (p.nq != 1) return 0;
             return kHeader + (score_plan(p, true).bytes + 255) / 256 * 256 + decode_scratch_bytes(p);

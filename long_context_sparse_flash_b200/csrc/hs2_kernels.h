@@ -25,13 +25,19 @@ void count_launch(int n = 1);
 void prof_begin(uint32_t kid, cudaStream_t st);
 void prof_end(cudaStream_t st);
 
-// K1 on tcgen05/TMEM/TMA (prefill-shaped calls: 128-row query tiles).
+// K1 on tcgen05/TMEM/TMA (prefill-shaped calls: 128-row query tiles).  When
+// full_tc_splits(p) > 1 and `scratch` holds full_tc_split_scratch_bytes(p),
+// each CTA's key range is split and the parts merged exactly; otherwise no
+// scratch is used.
+int full_tc_splits(const Problem& p);
+size_t full_tc_split_scratch_bytes(const Problem& p);
 cudaError_t launch_full_tc(const Problem& p, const void* q, const void* k, const void* v, void* out,
-                           float* lse, cudaStream_t st);
+                           float* lse, void* scratch, size_t scratch_bytes, cudaStream_t st);
 
-// K1: causal full attention + LSE for every query of the call.
+// K1: causal full attention + LSE for every query of the call (scratch: see
+// launch_full_tc; may be null).
 cudaError_t launch_full(const Problem& p, const void* q, const void* k, const void* v, void* out,
-                        float* lse, cudaStream_t st);
+                        float* lse, void* scratch, size_t scratch_bytes, cudaStream_t st);
 
 // K2 part 1: selection scores of queries [i_begin, i_begin + i_count) into
 // scores[((b * hkv + g) * i_count + (i - i_begin)) * sstride + j], j <= t - window.

@@ -211,10 +211,10 @@ cudaError_t launch_full_d(const Problem& p, const void* q, const void* k, const 
 }  // namespace
 
 cudaError_t launch_full(const Problem& p, const void* q, const void* k, const void* v, void* out,
-                        float* lse, cudaStream_t st) {
+                        float* lse, void* scratch, size_t scratch_bytes, cudaStream_t st) {
     // prefill-shaped calls run on the tcgen05 kernel; decode-shaped ones (one
     // query per sequence) on the mma.sync kernel below
-    if (p.seq_len == nullptr && p.nq >= 64) return launch_full_tc(p, q, k, v, out, lse, st);
+    if (p.seq_len == nullptr && p.nq >= 64) return launch_full_tc(p, q, k, v, out, lse, scratch, scratch_bytes, st);
     if (p.D == 64) return launch_full_d<64>(p, q, k, v, out, lse, st);
     return launch_full_d<128>(p, q, k, v, out, lse, st);
 }

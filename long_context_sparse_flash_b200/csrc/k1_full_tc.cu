@@ -161,7 +161,9 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                                                                   const __grid_constant__ CUtensorMap tm_k,
                                                                   const __grid_constant__ CUtensorMap tm_v,
                                                                   Problem p, __nv_bfloat16* __restrict__ out,
-                                                                  float* __restrict__ lse) {
+                                                                  float* __restrict__ lse, int n_split,
+                                                                  float* __restrict__ part_o,
+                                                                  float* __restrict__ part_l) {
     using C = PpCfg<D>;
     constexpr int NS = C::NS;
     extern __shared__ uint8_t smem_raw[];
@@ -177,11 +179,17 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
     const int n_blk = (p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM);
     const int blk = n_blk - 1 - (int)blockIdx.x;  // longest causal rows first
     const int i0 = blk * PP_QT * PP_BM;
-    const int h = blockIdx.y, b = blockIdx.z;
+    const int h = blockIdx.y, b = (int)blockIdx.z / n_split, split = (int)blockIdx.z % n_split;
     const int G = p.hq / p.hkv, g = h / G;
     const int64_t pos0 = seq_pos0(p, b, KID_FULL);
     const int i_last = min(i0 + PP_QT * PP_BM, p.nq) - 1;
-    const int n_tiles = (int)((pos0 + i_last + PP_BN) / PP_BN);
+    // key tiles of the causal range; with a split, this CTA takes the split-th of
+    // n_split contiguous parts, tiles jt0 .. jt0 + n_tiles - 1 (loop indices below
+    // are local, tile jt0 + j is read)
+    const int n_all = (int)((pos0 + i_last + PP_BN) / PP_BN);
+    const int per = (n_all + n_split - 1) / n_split;
+    const int jt0 = min(split * per, n_all);
+    const int n_tiles = min(per, n_all - jt0);
 
     if (tid == 0) {
         for (int i = 0; i < PB_COUNT; ++i) tc::mbar_init(bar(i), (i == PB_PFULL || i == PB_PFULL + 1) ? 128u : 1u);
@@ -214,7 +222,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                     if (!ok) break;
                     tc::mbar_expect_tx(bar(PB_KFULL + s), C::KB * C::BLK);
                     for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_3d(sK + (s * C::KB + kb) * C::BLK, &tm_k, bar(PB_KFULL + s), kb * 64, j * PP_BN, zk);
+                        tc::tma_load_3d(sK + (s * C::KB + kb) * C::BLK, &tm_k, bar(PB_KFULL + s), kb * 64,
+                                        (jt0 + j) * PP_BN, zk);
                     k_issued = j + 1;
                 }
                 if (j >= 1) {
@@ -223,7 +232,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                     if (!ok) break;
                     tc::mbar_expect_tx(bar(PB_VFULL + s), C::KB * C::BLK);
                     for (int kb = 0; kb < C::KB; ++kb)
-                        tc::tma_load_3d(sV + (s * C::KB + kb) * C::BLK, &tm_v, bar(PB_VFULL + s), kb * 64, jv * PP_BN, zk);
+                        tc::tma_load_3d(sV + (s * C::KB + kb) * C::BLK, &tm_v, bar(PB_VFULL + s), kb * 64,
+                                        (jt0 + jv) * PP_BN, zk);
                     v_issued = jv + 1;
                 }
             }
@@ -279,8 +289,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             __syncwarp();
         };
         bool ok = __all_sync(~0u, tc::mbar_wait(bar(PB_Q), 0, ab, p.err, KID_FULL, 3));
-        if (ok) ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL), 0, ab, p.err, KID_FULL, 4));
-        if (ok) {
+        if (ok && n_tiles > 0) ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL), 0, ab, p.err, KID_FULL, 4));
+        if (ok && n_tiles > 0) {
             tc::fence_after_sync();
             issue_s(0, 0);
             issue_s(1, 0);
@@ -326,7 +336,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             ok = tc::mbar_wait(bar(PB_SFULL + x), j & 1, ab, p.err, KID_FULL, 8);
             if (!ok) break;
             tc::fence_after_sync();
-            const int64_t j0 = (int64_t)j * PP_BN;
+            const int64_t j0 = (int64_t)(jt0 + j) * PP_BN;
             load_scores(s_addr, s, j0 + PP_BN - 1 > t, j0, t);
             const float mt = tile_max(s) * p.scale_log2;
             if (mt > m + 8.f) {
@@ -347,7 +357,9 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                 l *= alpha;
                 m = mt;
             }
-            l += exp_pack_tile(s, p.scale_log2, m);
+            // (m stays -inf only while every key so far is masked, which a split
+            // can start with: those exponentials are 0)
+            l += exp_pack_tile(s, p.scale_log2, m == -INFINITY ? 0.f : m);
             // P_X,j (bf16 pairs) over the first 64 columns of S_X
             tc::tmem_st32(s_addr, s);
             tc::tmem_st32(s_addr + 32, s + 32);
@@ -355,9 +367,33 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             tc::fence_before_sync();
             tc::mbar_arrive(bar(PB_PFULL + x));
         }
-        // epilogue: O / l -> out (bf16), lse
-        if (ok) ok = tc::mbar_wait(bar(PB_ODONE + x), 0, ab, p.err, KID_FULL, 9);
-        if (ok) {
+        // epilogue: O / l -> out (bf16), lse; with a split, the part's O / l (fp32)
+        // and base-2 log-sum-exp for the merge
+        if (ok && n_tiles > 0) ok = tc::mbar_wait(bar(PB_ODONE + x), 0, ab, p.err, KID_FULL, 9);
+        if (ok && n_split > 1) {
+            tc::fence_after_sync();
+            const int i = i0 + x * PP_BM + r;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int64_t prow = (((int64_t)split * p.B + b) * p.hq + h) * p.nq + i;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                float o[32];
+                if (n_tiles > 0) {
+                    tc::tmem_ld32(o_addr + c * 32, o);
+                    tc::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
+                }
+                if (i < p.nq) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(part_o + prow * D + c * 32 + e) =
+                            make_float4(o[e] * inv, o[e + 1] * inv, o[e + 2] * inv, o[e + 3] * inv);
+                }
+            }
+            if (i < p.nq) part_l[prow] = l > 0.f ? m + log2f(l) : -INFINITY;
+        } else if (ok) {
             tc::fence_after_sync();
             const int i = i0 + x * PP_BM + r;
             const float inv = 1.f / l;
@@ -391,9 +427,55 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
     }
 }
 
+// Exact merge of the split parts of each row: with part lse2_s = m_s + log2(l_s)
+// and part output O_s = (sum p v) / l_s, out = sum_s 2^(lse2_s - M) O_s / L and
+// lse = ln 2 (M + log2 L), M = max_s lse2_s, L = sum_s 2^(lse2_s - M).
+// One warp per (sequence, head, query) row.
+template <int D>
+__global__ void __launch_bounds__(256) k1_split_combine_kernel(Problem p, int n_split, const float* __restrict__ part_o,
+                                                               const float* __restrict__ part_l,
+                                                               __nv_bfloat16* __restrict__ out,
+                                                               float* __restrict__ lse) {
+    const int64_t rows = (int64_t)p.B * p.hq * p.nq;
+    const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    float M = -INFINITY;
+    for (int s = 0; s < n_split; ++s) M = fmaxf(M, part_l[(int64_t)s * rows + row]);
+    constexpr int E = D / 32;  // elements per lane
+    float acc[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    float L = 0.f;
+    for (int s = 0; s < n_split; ++s) {
+        const float ls = part_l[(int64_t)s * rows + row];
+        const float w = ls == -INFINITY ? 0.f : ex2(ls - M);
+        L += w;
+        const float* o = part_o + ((int64_t)s * rows + row) * D + lane * E;
+        if constexpr (E == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(o);
+            acc[0] += w * v.x, acc[1] += w * v.y, acc[2] += w * v.z, acc[3] += w * v.w;
+        } else {
+            const float2 v = *reinterpret_cast<const float2*>(o);
+            acc[0] += w * v.x, acc[1] += w * v.y;
+        }
+    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    __nv_bfloat16* orow = out + row * D + lane * E;
+    if constexpr (E == 4) {
+        uint2 v;
+        v.x = pack_bf16(acc[0] * inv, acc[1] * inv);
+        v.y = pack_bf16(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2*>(orow) = v;
+    } else {
+        *reinterpret_cast<uint32_t*>(orow) = pack_bf16(acc[0] * inv, acc[1] * inv);
+    }
+    if (lane == 0) lse[row] = (M + log2f(L)) * kLn2;
+}
+
 template <int D>
 cudaError_t launch_full_tc_d(const Problem& p, const void* q, const void* k, const void* v, void* out, float* lse,
-                             cudaStream_t st) {
+                             int n_split, float* part_o, float* part_l, cudaStream_t st) {
     using C = PpCfg<D>;
     CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, D, (uint64_t)p.nq, (uint64_t)p.B * p.hq, PP_BM) ||
@@ -409,9 +491,15 @@ cudaError_t launch_full_tc_d(const Problem& p, const void* q, const void* k, con
     e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
     if ((long)fa.numRegs * PP_THREADS < 256L * PP_REG_SOFTMAX + 128L * PP_REG_OTHER) return cudaErrorInvalidConfiguration;
-    dim3 grid((p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM), p.hq, p.B);
+    dim3 grid((p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM), p.hq, p.B * n_split);
     prof_begin(KID_FULL, st);
-    kern<<<grid, PP_THREADS, C::SMEM, st>>>(mq, mk, mv, p, (__nv_bfloat16*)out, lse);
+    kern<<<grid, PP_THREADS, C::SMEM, st>>>(mq, mk, mv, p, (__nv_bfloat16*)out, lse, n_split, part_o, part_l);
+    if (n_split > 1) {
+        const int64_t rows = (int64_t)p.B * p.hq * p.nq;
+        k1_split_combine_kernel<D><<<(unsigned)((rows * 32 + 255) / 256), 256, 0, st>>>(
+            p, n_split, part_o, part_l, (__nv_bfloat16*)out, lse);
+        count_launch();
+    }
     prof_end(st);
     count_launch();
     return cudaGetLastError();
@@ -419,10 +507,53 @@ cudaError_t launch_full_tc_d(const Problem& p, const void* q, const void* k, con
 
 }  // namespace
 
+// Parts the key range of each full-attention CTA is split into.  Calls with
+// few, very long CTAs (a short chunk appended to a long cache) leave part of
+// the last wave of 148 SMs idle; splitting each CTA's keys into S parts (each
+// at least 256 tiles) and merging the parts exactly fills the waves.  S is the
+// smallest value whose idle fraction of the last wave is at least 2 points
+// better than S = 1 (deterministic: the workspace size depends on it).
+int full_tc_splits(const Problem& p) {
+    if (p.seq_len != nullptr || p.nq < 64) return 1;
+    const int64_t ctas = (int64_t)((p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM)) * p.hq * p.B;
+    const int64_t min_tiles = (p.q_pos0 + (p.nq < PP_QT * PP_BM ? p.nq : PP_QT * PP_BM) + PP_BN - 1) / PP_BN;
+    auto idle = [](int64_t n) {
+        const int64_t waves = (n + 147) / 148;
+        return (double)(waves * 148 - n) / (double)(waves * 148);
+    };
+    int best = 1;
+    double best_idle = idle(ctas);
+    for (int S = 2; S <= 4; ++S) {
+        if (min_tiles / S < 256) break;
+        const double f = idle(ctas * S);
+        if (f < best_idle - 0.02) {
+            best = S;
+            best_idle = f;
+        }
+    }
+    return best;
+}
+
+size_t full_tc_split_scratch_bytes(const Problem& p) {
+    const int S = full_tc_splits(p);
+    if (S <= 1) return 0;
+    const size_t rows = (size_t)p.B * p.hq * p.nq;
+    return (size_t)S * rows * ((size_t)p.D * 4 + 4) + 256;
+}
+
 cudaError_t launch_full_tc(const Problem& p, const void* q, const void* k, const void* v, void* out, float* lse,
-                           cudaStream_t st) {
-    if (p.D == 64) return launch_full_tc_d<64>(p, q, k, v, out, lse, st);
-    return launch_full_tc_d<128>(p, q, k, v, out, lse, st);
+                           void* scratch, size_t scratch_bytes, cudaStream_t st) {
+    int S = full_tc_splits(p);
+    float *part_o = nullptr, *part_l = nullptr;
+    if (S > 1 && scratch != nullptr && scratch_bytes >= full_tc_split_scratch_bytes(p)) {
+        const size_t rows = (size_t)p.B * p.hq * p.nq;
+        part_o = reinterpret_cast<float*>(scratch);
+        part_l = part_o + (size_t)S * rows * p.D;
+    } else {
+        S = 1;
+    }
+    if (p.D == 64) return launch_full_tc_d<64>(p, q, k, v, out, lse, S, part_o, part_l, st);
+    return launch_full_tc_d<128>(p, q, k, v, out, lse, S, part_o, part_l, st);
 }
 
 }  // namespace hs2

@@ -221,3 +221,16 @@ def test_decode_exact_ties_take_the_full_radix_path():
     want = torch.arange(w.topk, dtype=torch.int32, device="cuda")
     assert torch.equal(gpu["idx"], want.expand_as(gpu["idx"]))
     P.compare_rows(w, inp, gpu, 1, np.array([0]), ts=np.array([w.kv_len - 1]))
+
+
+@pytest.mark.parametrize("head_dim,h_q,h_kv", [(128, 8, 2), (64, 8, 1)])
+def test_split_key_range_full_attention(head_dim, h_q, h_kv):
+    """Few query tiles over a long cache: the full layer splits each CTA's key
+    range in parts and merges them exactly (out, lse and the selection built on
+    the merged lse)."""
+    w = wl.custom("split_kv", n_q=256, q_pos0=70000, kv_len=70256, h_q=h_q, h_kv=h_kv, head_dim=head_dim,
+                  window=128, topk=256, n_sparse=1, seed=8)
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    P.compare_rows(w, inp, gpu, 0, np.array([0, 1, 127, 128, 200, 255]))
+    _row_properties(gpu["idx"], w)
