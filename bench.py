@@ -81,7 +81,10 @@ def kernel_work(w: wl.Workload):
         work["select_topk"] = dict(bound="hbm", bytes=4.0 * cand + f["idx_bytes"])
     else:
         # prefill: the filtered sweep recomputes QK^T over every candidate of every query
-        work["select_filter"] = dict(bound="tensor", flops=f["select_qk_flops"])
+        # and takes one 2^x per (candidate, head): the special-function unit's ex2 rate is
+        # the binding limit ("alu"); the tensor-core fraction is reported beside it
+        G = w.h_q // w.h_kv
+        work["select_filter"] = dict(bound="alu", ex2=G * cand, flops=f["select_qk_flops"])
     return work
 
 
@@ -106,6 +109,25 @@ def measure_l2_gather(dev, reps: int = 10) -> float:
     torch.cuda.synchronize()
     ms = min(e0.elapsed_time(e1) for e0, e1 in ev)
     return order.numel() * 256.0 * passes / (ms / 1e3) / 1e9
+
+
+def measure_ex2(dev, reps: int = 10) -> float:
+    """ex2 per second of the special-function units (the library's probe: 8
+    independent 2^x chains per thread, 2048 threads per SM), fastest of `reps`."""
+    sink = torch.zeros(4, dtype=torch.float32, device=dev)
+    iters = 4096
+    for _ in range(3):
+        n = nv.hs2_ex2_probe(iters, sink)
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        e0.record(st)
+        n = nv.hs2_ex2_probe(iters, sink)
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = min(e0.elapsed_time(e1) for e0, e1 in ev)
+    return n / (ms / 1e3)
 
 
 def source_sha(path: str) -> str:
@@ -385,11 +407,16 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
         elif wk["bound"] == "l2":
             achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
             peak, unit = round(pk["l2_gather"], 1), "GB/s"
+        elif wk["bound"] == "alu":
+            achieved = wk["ex2"] * calls / (ms / 1e3) / 1e9
+            peak, unit = round(pk["ex2"] / 1e9, 1), "Gex2/s"
         else:
             achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
             peak, unit = pk["hbm"], "GB/s"
         per[name] = dict(ms=ms / K, launches=launches // K if K else launches, bound=wk["bound"],
                          achieved=round(achieved, 2), peak=peak, unit=unit, frac=round(achieved / peak, 4))
+        if wk["bound"] == "alu" and "flops" in wk:  # the contraction's share of the tensor peak, for reference
+            per[name]["tensor_frac"] = round(wk["flops"] * calls / (ms / 1e3) / 1e12 / pk["tc_sustained"], 4)
     if not per:
         return None, per
     top = max((n for n in per if "bound" in per[n]), key=lambda n: per[n]["ms"])
@@ -397,7 +424,8 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
     launches_total = prof[top][1]
     traffic = dram_traffic(top, w.name)
     src = {"tensor": pk["src"] + " (sustained bf16)", "hbm": pk["src"] + " (copy GB/s)",
-           "l2": "measured here (random 256-byte-row gather from a 64 MiB L2-resident buffer, hs2_gather_probe)"}
+           "l2": "measured here (random 256-byte-row gather from a 64 MiB L2-resident buffer, hs2_gather_probe)",
+           "alu": "measured here (special-function-unit ex2 rate, hs2_ex2_probe)"}
     rf = {"kernel": top, "bound": p["bound"], "achieved": p["achieved"],
           "peak": p["peak"], "unit": p["unit"], "frac": p["frac"],
           "peak_source": src[p["bound"]],
@@ -414,6 +442,7 @@ def run_ours(args):
     # the L2 gather peak is taken first, on an idle GPU (a burst figure, like
     # the other measured peaks), before the workload's tensors exist
     l2_gather = measure_l2_gather(dev) if any(wk["bound"] == "l2" for wk in kernel_work(w).values()) else None
+    ex2_rate = measure_ex2(dev) if any(wk["bound"] == "alu" for wk in kernel_work(w).values()) else None
     inp = wl.make_inputs(w, dev, seed=replica_seed(w, rank))  # independent replica per rank
     step = Step(w, inp, dev)
     flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
@@ -447,6 +476,7 @@ def run_ours(args):
 
     pk = peaks()
     pk["l2_gather"] = l2_gather
+    pk["ex2"] = ex2_rate
     rf, per_kernel = roofline(w, prof, args.steps, pk)
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)

@@ -225,6 +225,16 @@ hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t strea
 hs2_status hs2_gather_probe(const void* rows, int64_t n_rows, const int32_t* order, int64_t n_order,
                             int32_t passes, void* sink, hs2_stream_t stream);
 
+/* Diagnostics: the special-function-unit probe behind the selection sweep's
+ * roofline (its binding unit is the ex2 rate: one 2^x per candidate and head).
+ * Launches (SM count x 8) CTAs of 256 threads, each thread running 8
+ * independent chains of `iters` hardware ex2 steps, on `stream`; writes the
+ * number of ex2 executed to *ex2_count (host) at once.  `sink` (device, one
+ * float) is written only in a case that practically never occurs.  The caller
+ * times the call.  Requires iters >= 1 and non-null pointers, else
+ * HS2_ERR_INVALID_ARG.  Not part of the method (no counterpart in the paper). */
+hs2_status hs2_ex2_probe(int32_t iters, float* sink, hs2_stream_t stream, int64_t* ex2_count);
+
 /* 1 when the library was built with device-side input checks (HS2_CHECKED). */
 int hs2_is_checked_build(void);
 

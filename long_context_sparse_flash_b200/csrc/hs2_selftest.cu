@@ -77,3 +77,35 @@ extern "C" hs2_status hs2_gather_probe(const void* rows, int64_t n_rows, const i
     hs2::count_launch();
     return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }
+
+namespace hs2 {
+namespace {
+// Eight independent x <- 2^-x chains per thread (the values settle near 0.64,
+// so every step is an ordinary ex2 on the special-function unit).
+__global__ void __launch_bounds__(256, 8) ex2_probe_kernel(int iters, float* __restrict__ sink) {
+    float x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = 0.01f * (float)(threadIdx.x + u);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) asm volatile("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(x[u]) : "f"(-x[u]));
+    }
+    float s = 0.f;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) s += x[u];
+    if (s == 12345.f) *sink = s;  // keeps the chains; practically never taken
+}
+}  // namespace
+}  // namespace hs2
+
+extern "C" hs2_status hs2_ex2_probe(int32_t iters, float* sink, hs2_stream_t stream, int64_t* ex2_count) {
+    if (iters < 1 || sink == nullptr || ex2_count == nullptr) return HS2_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return HS2_ERR_CUDA;
+    const int blocks = sms * 8;
+    hs2::ex2_probe_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(iters, sink);
+    hs2::count_launch();
+    *ex2_count = (int64_t)blocks * 256 * 8 * iters;
+    return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}

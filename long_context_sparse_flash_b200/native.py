@@ -27,7 +27,7 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
-           "hs2_gather_probe")
+           "hs2_gather_probe", "hs2_ex2_probe")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
@@ -86,10 +86,11 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_static_scratch_bytes.restype = S
     lib.hs2_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     lib.hs2_gather_probe.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int32, P, P]
+    lib.hs2_ex2_probe.argtypes = [ctypes.c_int32, P, P, ctypes.POINTER(ctypes.c_int64)]
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
-                 "hs2_gather_probe"):
+                 "hs2_gather_probe", "hs2_ex2_probe"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -212,6 +213,13 @@ def hs2_gather_probe(rows: torch.Tensor, order: torch.Tensor, passes: int, sink:
     n_rows = rows.numel() * rows.element_size() // 256
     _check(load().hs2_gather_probe(_ptr(rows), int(n_rows), _ptr(order), int(order.numel()), int(passes),
                                    _ptr(sink), _stream(stream)), "hs2_gather_probe")
+
+
+def hs2_ex2_probe(iters: int, sink: torch.Tensor, stream=None) -> int:
+    """Special-function-unit probe; returns the number of ex2 it executes."""
+    n = ctypes.c_int64(0)
+    _check(load().hs2_ex2_probe(int(iters), _ptr(sink), _stream(stream), ctypes.byref(n)), "hs2_ex2_probe")
+    return int(n.value)
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):

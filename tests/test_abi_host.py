@@ -150,3 +150,13 @@ def test_gather_probe_argument_checks():
     assert L.hs2_gather_probe(FAKE, 0, FAKE, 32, 1, FAKE, None) == 1    # no rows
     assert L.hs2_gather_probe(ctypes.c_void_p((1 << 40) + 4), 16, FAKE, 32, 1, FAKE, None) == 1  # misaligned
     assert nv.hs2_launch_count() == before
+
+
+def test_ex2_probe_argument_checks():
+    L = nv.load()
+    n = ctypes.c_int64(0)
+    before = nv.hs2_launch_count()
+    assert L.hs2_ex2_probe(0, FAKE, None, ctypes.byref(n)) == 1
+    assert L.hs2_ex2_probe(4, None, None, ctypes.byref(n)) == 1
+    assert L.hs2_ex2_probe(4, FAKE, None, None) == 1
+    assert nv.hs2_launch_count() == before

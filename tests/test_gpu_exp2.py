@@ -46,3 +46,16 @@ def test_gather_probe_reads_and_skips_bad_indices():
     torch.cuda.synchronize()
     assert nv.hs2_launch_count() == before + 1
     assert torch.all(sink == 0)  # the keep-alive store is not taken
+
+
+def test_ex2_probe_counts_and_runs():
+    """The special-function-unit probe behind the selection sweep's roofline runs as
+    one launch and reports (SM count x 8 CTAs) x 256 threads x 8 chains x iters ex2."""
+    sink = torch.zeros(4, dtype=torch.float32, device="cuda")
+    before = nv.hs2_launch_count()
+    n = nv.hs2_ex2_probe(16, sink)
+    torch.cuda.synchronize()
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert n == sms * 8 * 256 * 8 * 16
+    assert nv.hs2_launch_count() == before + 1
+    assert torch.all(sink == 0)
