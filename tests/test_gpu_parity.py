@@ -234,3 +234,22 @@ def test_split_key_range_full_attention(head_dim, h_q, h_kv):
     gpu = P.run_gpu(w, inp)
     P.compare_rows(w, inp, gpu, 0, np.array([0, 1, 127, 128, 200, 255]))
     _row_properties(gpu["idx"], w)
+
+
+DECODE_SHAPES = [
+    # name, kwargs: other head dims, group sizes, budgets and windows than the decode workloads
+    ("d64_g4_k2048_w1024", dict(batch=2, q_pos0=49999, kv_len=50000, h_q=16, h_kv=4, head_dim=64, window=1024,
+                                topk=2048)),
+    ("d128_g2_k512_w16", dict(batch=3, q_pos0=2999, kv_len=3000, h_q=8, h_kv=4, head_dim=128, window=16, topk=512)),
+    ("d128_g1_k64", dict(batch=2, q_pos0=20479, kv_len=20480, h_q=4, h_kv=4, head_dim=128, window=128, topk=64)),
+]
+
+
+@pytest.mark.parametrize("name,kw", DECODE_SHAPES, ids=[d[0] for d in DECODE_SHAPES])
+def test_decode_shapes_every_sequence(name, kw):
+    w = wl.custom(name, n_q=1, n_sparse=2, decode=True, seed=11, **kw)
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    for b in range(w.batch):
+        P.compare_rows(w, inp, gpu, b, np.array([0]), ts=np.array([w.kv_len - 1]))
+    _row_properties(gpu["idx"], w)
