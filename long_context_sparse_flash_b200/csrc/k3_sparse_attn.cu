@@ -17,7 +17,7 @@
 //   O^T (D x 8 heads) += V_tile^T P^T         A = V^T via ldmatrix.trans,
 //                                             B = P^T via movmatrix.trans
 // The group's heads sit in the MMA's N = 8 columns (padded when G < 8), so no
-// tensor-core work is spent on padding rows of M.  With SP_WARPS > 1 the
+// tensor-core work is spent on padding rows of M.  With W > 1 warps per CTA the
 // warps' partial (max, sum, O) would be merged exactly at the end.
 #include "hs2_kernels.h"
 
@@ -25,26 +25,29 @@ namespace hs2 {
 
 namespace {
 
-constexpr int SP_WARPS = 1;  // more, smaller CTAs per SM hide the gather latency best
+// One warp per CTA when the grid fills the machine (more, smaller CTAs per SM
+// hide the gather latency best); four when it does not (decode-sized calls),
+// each warp then taking every fourth tile of the row.
+constexpr int SP_SMALL_GRID = 4 * 148;
 constexpr int SP_STAGES = 2;  // tiles in the staging ring
 
-template <int D>
+template <int D, int W>
 struct K3Cfg {
     static constexpr int CH = D / 8;
     static constexpr int TILE_BYTES = 16 * D * 2;                 // one 16-row K (or V) tile
     static constexpr int WARP_BYTES = SP_STAGES * 2 * TILE_BYTES;  // stages x (K, V)
-    static constexpr int STAGE_BYTES = SP_WARPS * WARP_BYTES;
-    static constexpr int COMB_BYTES = SP_WARPS * (D * 8 + 16) * 4;  // per warp: O^T, m, l
+    static constexpr int STAGE_BYTES = W * WARP_BYTES;
+    static constexpr int COMB_BYTES = W * (D * 8 + 16) * 4;  // per warp: O^T, m, l
     static constexpr int FIXED = STAGE_BYTES > COMB_BYTES ? STAGE_BYTES : COMB_BYTES;
 };
 
-template <int D, int G>
-__global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, const __nv_bfloat16* __restrict__ q,
+template <int D, int G, int W>
+__global__ void __launch_bounds__(W * 32) k3_sparse_kernel(Problem p, const __nv_bfloat16* __restrict__ q,
                                                                    const __nv_bfloat16* __restrict__ k,
                                                                    const __nv_bfloat16* __restrict__ v,
                                                                    const int32_t* __restrict__ idx,
                                                                    __nv_bfloat16* __restrict__ out) {
-    using C = K3Cfg<D>;
+    using C = K3Cfg<D, W>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int i = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -57,7 +60,7 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     // then the window
     const int32_t* irow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
     int cnt = 0;
-    for (int r = tid; r < p.topk; r += SP_WARPS * 32) {
+    for (int r = lane; r < p.topk; r += 32) {
         const int32_t j = irow[r];
         cnt += j >= 0;
 #ifdef HS2_CHECKED
@@ -71,7 +74,6 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 4);
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 2);
     cnt += __shfl_xor_sync(0xffffffffu, cnt, 1);
-    static_assert(SP_WARPS == 1, "the row count is a warp reduction");
     const int nsel = cnt;
     const int n = nsel + nwin;
     const int n_mt = (n + 15) / 16;
@@ -126,23 +128,26 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     for (int dt = 0; dt < D / 16; ++dt) acc[dt][0] = acc[dt][1] = acc[dt][2] = acc[dt][3] = 0.f;
     float m_c[2] = {-INFINITY, -INFINITY}, l_c[2] = {0.f, 0.f};
 
-    // ring: tile mt lives in stage mt % SP_STAGES; tiles mt + 1 .. mt + SP_STAGES - 1
-    // are in flight while tile mt is computed.  jr[u] = row index of tile mt + u
-    // (lane l: row l % 16), u < SP_STAGES; the next one is fetched a tile ahead.
+    // This warp's tiles are warp, warp + W, ...: its k-th tile lives in stage
+    // k % SP_STAGES; tiles k + 1 .. k + SP_STAGES - 1 are in flight while tile k is
+    // computed.  jr[u] = row index of its tile k + u (lane l: row l % 16), u <
+    // SP_STAGES; the next one is fetched a tile ahead.
     const int r16 = lane & 15;
+    const int n_loc = warp < n_mt ? (n_mt - warp + W - 1) / W : 0;
+    auto tile_row = [&](int kk) { return (warp + kk * W) * 16 + r16; };
     int32_t jr[SP_STAGES];
 #pragma unroll
-    for (int u = 0; u < SP_STAGES; ++u) jr[u] = row_of(u * 16 + r16);
+    for (int u = 0; u < SP_STAGES; ++u) jr[u] = row_of(tile_row(u));
 #pragma unroll
     for (int u = 0; u < SP_STAGES - 1; ++u) {
-        if (u < n_mt) load_tile(u, jr[u]);
+        if (u < n_loc) load_tile(u, jr[u]);
         cp_async_commit();
     }
     int stage = 0;
-    for (int mt = 0; mt < n_mt; ++mt) {
-        const int32_t j_next = row_of((mt + SP_STAGES) * 16 + r16);
+    for (int kt = 0; kt < n_loc; ++kt) {
+        const int32_t j_next = row_of(tile_row(kt + SP_STAGES));
         const int lstage = (stage + SP_STAGES - 1) % SP_STAGES;
-        if (mt + SP_STAGES - 1 < n_mt) load_tile(lstage, jr[SP_STAGES - 1]);
+        if (kt + SP_STAGES - 1 < n_loc) load_tile(lstage, jr[SP_STAGES - 1]);
         cp_async_commit();
         cp_async_wait<SP_STAGES - 1>();
         __syncwarp();
@@ -237,14 +242,14 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
         }
     }
     __syncthreads();
-    for (int u = tid; u < G * D; u += SP_WARPS * 32) {
+    for (int u = tid; u < G * D; u += W * 32) {
         const int hh = u / D, d = u % D;
         float mm = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < SP_WARPS; ++w) mm = fmaxf(mm, comb[w * (D * 8 + 16) + D * 8 + hh]);
+        for (int w = 0; w < W; ++w) mm = fmaxf(mm, comb[w * (D * 8 + 16) + D * 8 + hh]);
         float num = 0.f, den = 0.f;
 #pragma unroll
-        for (int w = 0; w < SP_WARPS; ++w) {
+        for (int w = 0; w < W; ++w) {
             const float* wb = comb + w * (D * 8 + 16);
             const float sc = ex2(wb[D * 8 + hh] - mm);
             num += sc * wb[d * 8 + hh];
@@ -254,21 +259,29 @@ __global__ void __launch_bounds__(SP_WARPS * 32) k3_sparse_kernel(Problem p, con
     }
 }
 
-template <int D, int G>
-cudaError_t launch_sparse_dg(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
-                             void* out, cudaStream_t st) {
-    using C = K3Cfg<D>;
+template <int D, int G, int W>
+cudaError_t launch_sparse_dgw(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
+                              void* out, cudaStream_t st) {
+    using C = K3Cfg<D, W>;
     const int smem = C::FIXED;
-    auto kern = k3_sparse_kernel<D, G>;
+    auto kern = k3_sparse_kernel<D, G, W>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(p.nq, p.hkv, p.B);
     prof_begin(KID_SPARSE, st);
-    kern<<<grid, SP_WARPS * 32, smem, st>>>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                           (const __nv_bfloat16*)v, idx, (__nv_bfloat16*)out);
+    kern<<<grid, W * 32, smem, st>>>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
+                                     idx, (__nv_bfloat16*)out);
     prof_end(st);
     count_launch();
     return cudaGetLastError();
+}
+
+template <int D, int G>
+cudaError_t launch_sparse_dg(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
+                             void* out, cudaStream_t st) {
+    const int64_t ctas = (int64_t)p.nq * p.hkv * p.B;
+    if (ctas < SP_SMALL_GRID) return launch_sparse_dgw<D, G, 4>(p, q, k, v, idx, out, st);
+    return launch_sparse_dgw<D, G, 1>(p, q, k, v, idx, out, st);
 }
 
 template <int D>
