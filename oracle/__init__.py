@@ -18,6 +18,9 @@ Method (HySparse2 pages: xiawanshe.com report, sections "两级KV共享" /
   causal probability, ties to the lower index, emitted ascending, -1 padded.
 * ``sparse`` -- one KV-reuse layer: softmax attention of the layer's own query
   over idx U window(t).
+* ``kv_bridge`` -- KV bridging (same report, section "两级KV共享", first
+  level): a token's Cross-Decoder K and V from its Self-Decoder hidden state by
+  one projection, output features [K heads | V heads], D per head.
 """
 from __future__ import annotations
 
@@ -61,6 +64,8 @@ def open_library(path: str):
     lib.hs2o_sparse.argtypes = [i32, i32, i32, i32, i32, ctypes.c_double,
                                 i64, P, P, P, P, i64, i64, P, P, i32]
     lib.hs2o_sparse.restype = i32
+    lib.hs2o_kv_bridge.argtypes = [i64, i32, i32, i32, P, P, P, P, i32]
+    lib.hs2o_kv_bridge.restype = i32
     lib.hs2o_max_threads.argtypes = []
     lib.hs2o_max_threads.restype = i32
     return lib
@@ -152,3 +157,20 @@ def sparse(q_rows, t, k, v, idx, *, window: int, scale: float | None = None,
     if rc != 0:
         raise RuntimeError(f"hs2o_sparse failed with code {rc}")
     return out
+
+
+def kv_bridge(hidden, w, *, h_kv: int, head_dim: int, n_threads: int = 0):
+    """K and V of each token from its hidden state: ``hidden`` [n_rows, d_model]
+    and ``w`` [2 * h_kv * head_dim, d_model] as bf16 bit patterns; returns
+    (k, v), each [n_rows, h_kv, head_dim] float64."""
+    x = _as_bits(hidden)
+    wb = _as_bits(w)
+    n_rows, d_model = x.shape
+    assert wb.shape == (2 * h_kv * head_dim, d_model)
+    k = np.empty((n_rows, h_kv, head_dim), dtype=np.float64)
+    v = np.empty_like(k)
+    rc = _load().hs2o_kv_bridge(n_rows, d_model, h_kv, head_dim, _ptr(x), _ptr(wb), _ptr(k), _ptr(v),
+                                int(n_threads))
+    if rc != 0:
+        raise ValueError(f"hs2o_kv_bridge: error {rc}")
+    return k, v

@@ -29,7 +29,12 @@
  *     (score descending, j ascending) -- ties go to the lower index -- and is
  *     emitted sorted ascending by j, padded with -1;
  *   - a sparse layer attends, per head, to the set idx_g(t) U window(t) with
- *     its own query, same K/V, same 1/sqrt(D) scale.
+ *     its own query, same K/V, same 1/sqrt(D) scale;
+ *   - "KV Bridging" (same report and section, first level) computes a token's
+ *     K and V from its Self-Decoder hidden state with one projection (no
+ *     bias, no normalisation or position encoding: the pages name none); the
+ *     projection's output features are [K heads 0..H_kv-1 | V heads], each
+ *     head D contiguous features.
  *
  * Every quantity is computed in double precision from the bf16 inputs widened
  * exactly (bf16 bits << 16 is an exact fp32, and fp32 -> fp64 is exact).
@@ -277,6 +282,33 @@ int hs2o_sparse(int h_q, int h_kv, int d, int window, int topk, double scale,
         free(s);
     }
     return err;
+}
+
+/* KV bridging (xiawanshe.com report, section "两级KV共享", first level "KV
+ * Bridging"): the Cross-Decoder's K and V of a token are computed from the
+ * Self-Decoder hidden state of that token by one projection,
+ *     kv[f] = sum_c hidden[c] * w[f][c],   f < 2 * h_kv * d,
+ * features [0, h_kv*d) being K (head f / d, dim f % d) and [h_kv*d, 2*h_kv*d)
+ * being V.  hidden [n_rows][d_model], w [2*h_kv*d][d_model] (bf16 bits);
+ * out_k, out_v [n_rows][h_kv][d] fp64. */
+int hs2o_kv_bridge(int64_t n_rows, int d_model, int h_kv, int d, const uint16_t* hidden, const uint16_t* w,
+                   double* out_k, double* out_v, int n_threads) {
+    if (n_rows < 0 || d_model <= 0 || h_kv <= 0 || d <= 0) return HS2O_EINVAL;
+    const int64_t hd = (int64_t)h_kv * d;
+#pragma omp parallel for schedule(dynamic, 4) num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const uint16_t* x = hidden + r * (int64_t)d_model;
+        for (int64_t f = 0; f < 2 * hd; ++f) {
+            const uint16_t* wf = w + f * (int64_t)d_model;
+            double acc = 0.0;
+            for (int c = 0; c < d_model; ++c) acc += bf16_to_double(x[c]) * bf16_to_double(wf[c]);
+            if (f < hd)
+                out_k[r * hd + f] = acc;
+            else
+                out_v[r * hd + (f - hd)] = acc;
+        }
+    }
+    return HS2O_OK;
 }
 
 int hs2o_max_threads(void) {

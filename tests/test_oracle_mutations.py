@@ -32,6 +32,12 @@ MUTATIONS = {
     "sparse_window_short": ("const int64_t w0 = tr - window + 1 > 0 ? tr - window + 1 : 0;",
                             "const int64_t w0 = tr - window + 2 > 0 ? tr - window + 2 : 0;", 0),
     "sparse_wrong_group": ("const int h = g * G + hh;", "const int h = hh * h_kv + g;", 2),
+    "bridge_k_v_swapped": ("                out_k[r * hd + f] = acc;\n            else\n                out_v[r * hd + (f - hd)] = acc;",
+                           "                out_v[r * hd + f] = acc;\n            else\n                out_k[r * hd + (f - hd)] = acc;", 0),
+    "bridge_weight_transposed": ("const uint16_t* wf = w + f * (int64_t)d_model;",
+                                 "const uint16_t* wf = w + f;", 0),
+    "bridge_drops_last_column": ("for (int c = 0; c < d_model; ++c) acc += bf16_to_double(x[c]) * bf16_to_double(wf[c]);",
+                                 "for (int c = 0; c + 1 < d_model; ++c) acc += bf16_to_double(x[c]) * bf16_to_double(wf[c]);", 0),
 }
 
 FAST_PINS = [
@@ -48,6 +54,10 @@ FAST_PINS = [
     pins.test_sparse_with_full_budget_equals_full_attention,
     pins.test_sparse_with_zero_budget_is_sliding_window,
     pins.test_short_context_selects_nothing,
+    pins.test_bridge_identity_weights_copy_the_hidden_state,
+    pins.test_bridge_feature_layout_by_permuted_one_hot_rows,
+    pins.test_bridge_one_hot_hidden_returns_a_weight_column,
+    pins.test_bridge_decimal_brute_force,
 ]
 
 

@@ -399,3 +399,70 @@ def test_oracle_is_deterministic_across_thread_counts():
     b = oracle.full_select(q, ts, k, v, window=16, topk=30, n_threads=4)
     for key in ("out", "lse", "idx", "kth"):
         np.testing.assert_array_equal(a[key], b[key])
+
+
+# ---------------------------------------------------------------------------
+# KV bridging (xiawanshe.com report, section "两级KV共享", first level): a
+# token's K and V come from its Self-Decoder hidden state by one projection.
+
+
+def test_bridge_identity_weights_copy_the_hidden_state():
+    """With W = I (d_model = 2 H_kv D), K is the first half of the hidden state and
+    V the second, head-major, exactly."""
+    rng = np.random.default_rng(21)
+    h_kv, d = 2, 4
+    x = rng.standard_normal((5, 2 * h_kv * d)).astype(np.float32)
+    k, v = oracle.kv_bridge(bits(x), bits(np.eye(2 * h_kv * d, dtype=np.float32)), h_kv=h_kv, head_dim=d)
+    xb = unbits(bits(x)).astype(np.float64)
+    assert np.array_equal(k, xb[:, :h_kv * d].reshape(5, h_kv, d))
+    assert np.array_equal(v, xb[:, h_kv * d:].reshape(5, h_kv, d))
+
+
+def test_bridge_feature_layout_by_permuted_one_hot_rows():
+    """Row f of W picks hidden column perm[f]: K[h][d] must equal hidden[perm[h D + d]]
+    and V[h][d] hidden[perm[H D + h D + d]] -- fixes which output feature is
+    which (K or V, head, dim)."""
+    rng = np.random.default_rng(22)
+    h_kv, d, d_model = 3, 2, 16
+    f_total = 2 * h_kv * d
+    perm = rng.permutation(d_model)[:f_total]
+    w = np.zeros((f_total, d_model), dtype=np.float32)
+    w[np.arange(f_total), perm] = 1.0
+    x = rng.standard_normal((4, d_model)).astype(np.float32)
+    xb = unbits(bits(x)).astype(np.float64)
+    k, v = oracle.kv_bridge(bits(x), bits(w), h_kv=h_kv, head_dim=d)
+    for h in range(h_kv):
+        for dd in range(d):
+            assert np.array_equal(k[:, h, dd], xb[:, perm[h * d + dd]])
+            assert np.array_equal(v[:, h, dd], xb[:, perm[h_kv * d + h * d + dd]])
+
+
+def test_bridge_one_hot_hidden_returns_a_weight_column():
+    rng = np.random.default_rng(23)
+    h_kv, d, d_model = 2, 8, 32
+    w = rng.standard_normal((2 * h_kv * d, d_model)).astype(np.float32)
+    wb = unbits(bits(w)).astype(np.float64)
+    x = np.zeros((3, d_model), dtype=np.float32)
+    cols = [0, 7, 31]
+    x[np.arange(3), cols] = 1.0
+    k, v = oracle.kv_bridge(bits(x), bits(w), h_kv=h_kv, head_dim=d)
+    for r, c in enumerate(cols):
+        assert np.array_equal(k[r].reshape(-1), wb[:h_kv * d, c])
+        assert np.array_equal(v[r].reshape(-1), wb[h_kv * d:, c])
+
+
+def test_bridge_decimal_brute_force():
+    """Every output feature as a 50-digit decimal dot product of the bf16 values."""
+    rng = np.random.default_rng(24)
+    h_kv, d, d_model = 2, 3, 10
+    x = rng.standard_normal((2, d_model)).astype(np.float32)
+    w = rng.standard_normal((2 * h_kv * d, d_model)).astype(np.float32)
+    xb, wb = unbits(bits(x)), unbits(bits(w))
+    k, v = oracle.kv_bridge(bits(x), bits(w), h_kv=h_kv, head_dim=d)
+    got = np.concatenate([k.reshape(2, -1), v.reshape(2, -1)], axis=1)
+    with decimal.localcontext() as ctx:
+        ctx.prec = 50
+        for r in range(2):
+            for f in range(2 * h_kv * d):
+                ref = sum(decimal.Decimal(float(xb[r, c])) * decimal.Decimal(float(wb[f, c])) for c in range(d_model))
+                assert abs(float(ref) - got[r, f]) <= 1e-12 * max(1.0, abs(float(ref)))
