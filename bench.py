@@ -130,6 +130,46 @@ def measure_ex2(dev, reps: int = 10) -> float:
     return n / (ms / 1e3)
 
 
+def bench_bridge(w: wl.Workload, dev, K: int, warmup: int, pk: dict) -> dict:
+    """The KV-bridging projection (a next row of the path) for the workload's new
+    tokens: prefill-shaped workloads project all n_q tokens of every sequence and
+    write them at q_pos0; decode workloads append one token per sequence.  Timed
+    on its own (CUDA events per call, hidden states > L2), not part of `value`."""
+    d_model = wl.BRIDGE_D_MODEL
+    n_new = 1 if w.decode else w.n_q
+    inp = wl.make_bridge_inputs(w.batch, n_new, d_model, w.h_kv, w.head_dim, dev, seed=w.seed)
+    cap = w.kv_len
+    k = torch.empty(w.batch, w.h_kv, cap, w.head_dim, dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    pos = None if not w.decode else torch.full((w.batch,), cap - 1, dtype=torch.int64, device=dev)
+    pos0 = 0 if w.decode else w.q_pos0
+    run = lambda: nv.kv_bridge(inp["hidden"], inp["w_kv"], k, v, pos0=pos0, seq_pos=pos)
+    for _ in range(warmup):
+        run()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    st = torch.cuda.current_stream()
+    torch.cuda.synchronize()
+    for e0, e1 in ev:
+        e0.record(st)
+        run()
+        e1.record(st)
+    torch.cuda.synchronize()
+    ms = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    feats = 2 * w.h_kv * w.head_dim
+    flops = 2.0 * w.batch * n_new * d_model * feats
+    note = "hidden [tokens, d_model] x W_kv^T -> bf16 K/V cache rows (synthetic weights)"
+    if w.decode:  # one token per sequence: streaming the weights is the cost
+        nbytes = 2.0 * feats * d_model + 2.0 * w.batch * (d_model + feats)
+        gbs = nbytes / (ms / 1e3) / 1e9
+        return {"ms": round(ms, 4), "tokens": w.batch * n_new, "d_model": d_model, "bound": "hbm",
+                "achieved": round(gbs, 2), "peak": pk["hbm"], "unit": "GB/s", "frac": round(gbs / pk["hbm"], 4),
+                "note": note}
+    tf = flops / (ms / 1e3) / 1e12
+    return {"ms": round(ms, 4), "tokens": w.batch * n_new, "d_model": d_model, "bound": "tensor",
+            "achieved": round(tf, 2), "peak": pk["tc_sustained"], "unit": "TFLOP/s",
+            "frac": round(tf / pk["tc_sustained"], 4), "note": note}
+
+
 def source_sha(path: str) -> str:
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
@@ -478,6 +518,7 @@ def run_ours(args):
     pk["l2_gather"] = l2_gather
     pk["ex2"] = ex2_rate
     rf, per_kernel = roofline(w, prof, args.steps, pk)
+    next_rows = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
 
@@ -500,6 +541,7 @@ def run_ours(args):
                        "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write, outside the events)"},
             "per_kernel": per_kernel,
             "roofline": rf,
+            "next_rows": next_rows,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,

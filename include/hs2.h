@@ -200,7 +200,8 @@ uint64_t hs2_launch_count(void);
  * (launches[u]); either array may be NULL.  Kernel ids: 1 full attention,
  * 2 selection scores, 3 top-k select, 4 sparse attention, 5 decode attention
  * partials, 6 decode combine, 7 fused attention + selection, 8 selection
- * threshold estimate, 9 filtered selection sweep, 10 selection retry. */
+ * threshold estimate, 9 filtered selection sweep, 10 selection retry,
+ * 11 KV bridging. */
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 
@@ -211,6 +212,40 @@ hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launche
  * softmax and selection kernels).  y holds 5n floats.  Asynchronous on
  * `stream`. */
 hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t stream);
+
+/* KV bridging (xiawanshe.com report, section "两级KV共享", first level "KV
+ * Bridging": the Cross-Decoder's K and V are computed from the Self-Decoder's
+ * hidden states).  For every new token (b, i) of the call:
+ *     kv[f] = sum_c hidden[b][i][c] * w_kv[f][c],        f < 2 * h_kv * D
+ *     k_cache[b][f / D][pos_b + i][f % D]        = bf16(kv[f])   f <  h_kv * D
+ *     v_cache[b][f / D - h_kv][pos_b + i][f % D] = bf16(kv[f])   otherwise
+ * with pos_b = seq_pos[b] (device int64 array of `batch`) or, if seq_pos is
+ * NULL, pos0 for every sequence.  Only those cache rows are written (this is
+ * also the decode-time cache append, n_new = 1).  fp32 accumulation, one
+ * rounding to bf16 (round to nearest even).  Layouts (device, caller-owned,
+ * 16-byte aligned): hidden [batch][n_new][d_model] bf16; w_kv
+ * [2 * h_kv * D][d_model] bf16 (row f = output feature); k_cache, v_cache
+ * [batch][h_kv][kv_cap][D] bf16.  Requires d_model > 0 a multiple of 64, D in
+ * {64, 128}, h_kv * D a multiple of 256 (so each 256-feature tile lies in K
+ * or in V), 0 <= pos0, pos0 + n_new <= kv_cap when seq_pos is NULL (else
+ * HS2_ERR_INVALID_ARG / HS2_ERR_UNSUPPORTED).  With seq_pos, a sequence whose
+ * rows would fall outside [0, kv_cap) writes nothing and is reported through
+ * the error word (HS2_ERR_DEVICE_CHECK, kernel id 11).  ws: at least
+ * hs2_workspace_size(..., HS2_ENTRY_SPARSE) bytes (the header), or NULL with
+ * ws_bytes == 0 (then no error word).  Asynchronous on `stream`. */
+typedef struct {
+    int32_t batch;     /* sequences */
+    int32_t n_new;     /* new tokens per sequence */
+    int32_t d_model;   /* hidden size of the Self-Decoder */
+    int32_t h_kv;      /* KV heads */
+    int32_t head_dim;  /* D */
+    int32_t reserved;  /* must be 0 */
+    int64_t pos0;      /* cache position of token 0 when seq_pos is NULL */
+    int64_t kv_cap;    /* cache rows per (sequence, head) */
+} hs2_bridge_shape;
+hs2_status hs2_kv_bridge(const hs2_bridge_shape* shape, const int64_t* seq_pos, const void* hidden,
+                         const void* w_kv, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
+                         hs2_stream_t stream);
 
 /* Diagnostics: the gather-bandwidth probe behind the sparse layer's roofline
  * (the sparse layer reads whole 256-byte K/V rows in data-dependent order).

@@ -275,6 +275,30 @@ hs2_status run_sparse(const hs2_shape* shape, const int64_t* seq_len, const void
 }  // namespace
 }  // namespace hs2
 
+hs2_status hs2_kv_bridge(const hs2_bridge_shape* s, const int64_t* seq_pos, const void* hidden, const void* w_kv,
+                         void* k_cache, void* v_cache, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    if (s == nullptr) return HS2_ERR_INVALID_ARG;
+    if (s->reserved != 0 || s->batch < 0 || s->n_new < 0 || s->d_model <= 0 || s->h_kv <= 0 || s->kv_cap <= 0 ||
+        s->pos0 < 0)
+        return HS2_ERR_INVALID_ARG;
+    if (s->d_model % 64 != 0 || (s->head_dim != 64 && s->head_dim != 128) || (s->h_kv * s->head_dim) % 256 != 0 ||
+        s->h_kv > 64)
+        return HS2_ERR_UNSUPPORTED;
+    const int64_t n_rows = (int64_t)s->batch * s->n_new;
+    if ((n_rows + 127) / 128 > 65535) return HS2_ERR_UNSUPPORTED;  // token tiles in one grid dimension
+    if (seq_pos == nullptr && s->pos0 + s->n_new > s->kv_cap) return HS2_ERR_INVALID_ARG;
+    if (n_rows == 0) return HS2_OK;
+    if (!hidden || !w_kv || !k_cache || !v_cache) return HS2_ERR_INVALID_ARG;
+    if (!aligned(hidden, 16) || !aligned(w_kv, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        (seq_pos && !aligned(seq_pos, 8)))
+        return HS2_ERR_INVALID_ARG;
+    if (ws != nullptr && (ws_bytes < kHeader || !aligned(ws, 256))) return HS2_ERR_WORKSPACE;
+    if (ws == nullptr && ws_bytes != 0) return HS2_ERR_INVALID_ARG;
+    WsHeader* err = ws ? reinterpret_cast<WsHeader*>(ws) : nullptr;
+    return cuda_status(launch_bridge(n_rows, s->n_new, s->d_model, s->h_kv, s->head_dim, s->pos0, s->kv_cap, seq_pos,
+                                     hidden, w_kv, k_cache, v_cache, err, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 hs2_status hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,
                            void* out, void* ws, size_t ws_bytes, hs2_stream_t stream) {
     return run_sparse(shape, nullptr, q, k, v, idx, out, ws, ws_bytes, stream);

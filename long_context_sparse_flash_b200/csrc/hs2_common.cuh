@@ -33,6 +33,7 @@ enum KernelId : uint32_t {
     KID_THRESH = 8,
     KID_FILTER = 9,
     KID_RETRY = 10,
+    KID_BRIDGE = 11,
 };
 
 __device__ __forceinline__ void report_error(WsHeader* h, uint32_t code, uint32_t kid, uint32_t a,

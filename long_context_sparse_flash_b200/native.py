@@ -27,11 +27,11 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
-           "hs2_gather_probe", "hs2_ex2_probe")
+           "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
-                10: "select_retry"}
+                10: "select_retry", 11: "kv_bridge"}
 
 
 class HS2Error(RuntimeError):
@@ -45,6 +45,12 @@ class hs2_shape(ctypes.Structure):
                 ("h_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("topk", ctypes.c_int32), ("reserved", ctypes.c_int32), ("q_pos0", ctypes.c_int64),
                 ("kv_len", ctypes.c_int64), ("softmax_scale", ctypes.c_float)]
+
+
+class hs2_bridge_shape(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_new", ctypes.c_int32), ("d_model", ctypes.c_int32),
+                ("h_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("pos0", ctypes.c_int64), ("kv_cap", ctypes.c_int64)]
 
 
 _libs = {}
@@ -87,10 +93,11 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     lib.hs2_gather_probe.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int32, P, P]
     lib.hs2_ex2_probe.argtypes = [ctypes.c_int32, P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.hs2_kv_bridge.argtypes = [ctypes.POINTER(hs2_bridge_shape), P, P, P, P, P, P, S, P]
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
-                 "hs2_gather_probe", "hs2_ex2_probe"):
+                 "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -220,6 +227,26 @@ def hs2_ex2_probe(iters: int, sink: torch.Tensor, stream=None) -> int:
     n = ctypes.c_int64(0)
     _check(load().hs2_ex2_probe(int(iters), _ptr(sink), _stream(stream), ctypes.byref(n)), "hs2_ex2_probe")
     return int(n.value)
+
+
+def hs2_kv_bridge(shape: hs2_bridge_shape, seq_pos, hidden, w_kv, k_cache, v_cache, ws=None, stream=None,
+                  checked=False):
+    _check(load(checked).hs2_kv_bridge(ctypes.byref(shape), _ptr(seq_pos), _ptr(hidden), _ptr(w_kv),
+                                       _ptr(k_cache), _ptr(v_cache), _ptr(ws),
+                                       0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
+           "hs2_kv_bridge")
+
+
+def kv_bridge(hidden: torch.Tensor, w_kv: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *,
+              pos0: int = 0, seq_pos: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+              stream=None, checked: bool = False) -> None:
+    """K/V of the new tokens, hidden [B, n_new, d_model] @ w_kv^T, written into the
+    caches [B, H_kv, kv_cap, D] at rows pos_b + i (pos_b = seq_pos[b] or pos0)."""
+    B, n_new, d_model = hidden.shape
+    _, h_kv, kv_cap, D = k_cache.shape
+    shape = hs2_bridge_shape(batch=B, n_new=n_new, d_model=d_model, h_kv=h_kv, head_dim=D, reserved=0,
+                             pos0=pos0, kv_cap=kv_cap)
+    hs2_kv_bridge(shape, seq_pos, hidden, w_kv, k_cache, v_cache, ws, stream, checked)
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):

@@ -73,6 +73,10 @@ WORKLOADS: Dict[str, Workload] = {
 
 # sub-seed offsets, one per drawn tensor: seed * 1000 + offset
 SUB_Q, SUB_K, SUB_V, SUB_QS, SUB_NEEDLE, SUB_SEG = 1, 2, 3, 10, 50, 60
+SUB_HIDDEN, SUB_WKV = 70, 71
+# hidden size of the Self-Decoder for the KV-bridging inputs (the pages give no
+# model dimensions; a common size for a model of this class)
+BRIDGE_D_MODEL = 4096
 
 
 def custom(name="custom", *, batch=1, n_q=256, q_pos0=0, kv_len=None, h_q=8, h_kv=2, head_dim=64,
@@ -192,6 +196,18 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
             q_sparse.append((torch.randn(B, Hq, nq, D, generator=g, device=device) * 0.5)
                             .to(torch.bfloat16))
     return dict(q=q, k=k, v=v, q_sparse=q_sparse, probes=probes_all)
+
+
+def make_bridge_inputs(batch: int, n_new: int, d_model: int, h_kv: int, head_dim: int, device="cpu",
+                       seed: int = 0) -> Dict[str, torch.Tensor]:
+    """Seeded inputs of the KV-bridging projection: hidden states
+    hidden [batch, n_new, d_model] ~ N(0, 1) and weights w_kv [2 h_kv D, d_model]
+    ~ N(0, 1/d_model) (so K and V come out near unit scale), both bf16."""
+    gh = _gen(device, seed * 1000 + SUB_HIDDEN)
+    gw = _gen(device, seed * 1000 + SUB_WKV)
+    hidden = torch.randn(batch, n_new, d_model, generator=gh, device=device).to(torch.bfloat16)
+    w = (torch.randn(2 * h_kv * head_dim, d_model, generator=gw, device=device) / math.sqrt(d_model)).to(torch.bfloat16)
+    return dict(hidden=hidden, w_kv=w)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

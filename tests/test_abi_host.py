@@ -160,3 +160,29 @@ def test_ex2_probe_argument_checks():
     assert L.hs2_ex2_probe(4, None, None, ctypes.byref(n)) == 1
     assert L.hs2_ex2_probe(4, FAKE, None, None) == 1
     assert nv.hs2_launch_count() == before
+
+
+def test_kv_bridge_validation_without_launch():
+    L = nv.load()
+    before = nv.hs2_launch_count()
+
+    def bs(**kw):
+        base = dict(batch=1, n_new=16, d_model=256, h_kv=4, head_dim=128, reserved=0, pos0=0, kv_cap=64)
+        base.update(kw)
+        return nv.hs2_bridge_shape(**base)
+
+    def call(s, seq=None, ws=None, ws_bytes=0):
+        return L.hs2_kv_bridge(ctypes.byref(s), seq, FAKE, FAKE, FAKE, FAKE, ws, ws_bytes, None)
+
+    assert L.hs2_kv_bridge(None, None, FAKE, FAKE, FAKE, FAKE, None, 0, None) == 1
+    assert call(bs(reserved=1)) == 1
+    assert call(bs(d_model=100)) == 2            # d_model not a multiple of 64
+    assert call(bs(head_dim=96)) == 2
+    assert call(bs(h_kv=1)) == 2                 # h_kv * D = 128: a 256-feature tile would span K and V
+    assert call(bs(pos0=60)) == 1                # pos0 + n_new > kv_cap
+    assert call(bs(pos0=-1)) == 1
+    assert call(bs(), ws=FAKE, ws_bytes=100) == 3  # workspace smaller than the header
+    assert call(bs(), ws=None, ws_bytes=256) == 1
+    assert call(bs(n_new=0)) == 0                # empty: no launch
+    assert call(bs(batch=0)) == 0
+    assert nv.hs2_launch_count() == before
