@@ -18,6 +18,8 @@ Method (HySparse2 pages: xiawanshe.com report, sections "两级KV共享" /
   causal probability, ties to the lower index, emitted ascending, -1 padded.
 * ``sparse`` -- one KV-reuse layer: softmax attention of the layer's own query
   over idx U window(t).
+* ``block_select`` -- the predecessor block-level selection at the same
+  budget: whole blocks of contiguous candidates, ranked by summed score.
 * ``kv_bridge`` -- KV bridging (same report, section "两级KV共享", first
   level): a token's Cross-Decoder K and V from its Self-Decoder hidden state by
   one projection, output features [K heads | V heads], D per head.
@@ -65,6 +67,8 @@ def open_library(path: str):
                                 i64, P, P, P, P, i64, i64, P, P, i32]
     lib.hs2o_sparse.restype = i32
     lib.hs2o_kv_bridge.argtypes = [i64, i32, i32, i32, P, P, P, P, i32]
+    lib.hs2o_block_select.argtypes = [i64, i32, i32, i32, i32, P, P, i64, P, P, P]
+    lib.hs2o_block_select.restype = i32
     lib.hs2o_kv_bridge.restype = i32
     lib.hs2o_max_threads.argtypes = []
     lib.hs2o_max_threads.restype = i32
@@ -174,3 +178,25 @@ def kv_bridge(hidden, w, *, h_kv: int, head_dim: int, n_threads: int = 0):
     if rc != 0:
         raise ValueError(f"hs2o_kv_bridge: error {rc}")
     return k, v
+
+
+def block_select(q_rows, t, k, v, *, window: int, topk: int, block: int, scale: float | None = None,
+                 n_threads: int = 0):
+    """Block-level selection from the same per-candidate scores as ``full_select``:
+    returns dict(idx [n_rows, h_kv, topk] token indices of the kept blocks,
+    ascending, -1 padded; kth_block / next_block [n_rows, h_kv]: score of the last
+    kept block and of the best block left out (-1 if none); and the full_select
+    result under "full")."""
+    full = full_select(q_rows, t, k, v, window=window, topk=0, scale=scale, want_scores=True,
+                       n_threads=n_threads)
+    t = np.ascontiguousarray(np.asarray(t, dtype=np.int64))
+    sc = np.ascontiguousarray(full["scores"], dtype=np.float64)
+    n_rows, h_kv = sc.shape[0], sc.shape[1]
+    idx = np.empty((n_rows, h_kv, topk), dtype=np.int32)
+    kth = np.empty((n_rows, h_kv), dtype=np.float64)
+    nxt = np.empty((n_rows, h_kv), dtype=np.float64)
+    rc = _load().hs2o_block_select(n_rows, h_kv, window, topk, block, _ptr(t), _ptr(sc), sc.shape[2],
+                                   _ptr(idx), _ptr(kth), _ptr(nxt))
+    if rc != 0:
+        raise ValueError(f"hs2o_block_select: error {rc}")
+    return dict(idx=idx, kth_block=kth, next_block=nxt, full=full)

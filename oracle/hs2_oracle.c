@@ -30,6 +30,9 @@
  *     emitted sorted ascending by j, padded with -1;
  *   - a sparse layer attends, per head, to the set idx_g(t) U window(t) with
  *     its own query, same K/V, same 1/sqrt(D) scale;
+ *   - block-level selection (the predecessor design the "Token级选择" section
+ *     contrasts with) keeps whole blocks of blk contiguous candidate tokens,
+ *     blocks ranked by the sum of their tokens' scores, at the same budget;
  *   - "KV Bridging" (same report and section, first level) computes a token's
  *     K and V from its Self-Decoder hidden state with one projection (no
  *     bias, no normalisation or position encoding: the pages name none); the
@@ -280,6 +283,59 @@ int hs2o_sparse(int h_q, int h_kv, int d, int window, int topk, double scale,
         }
         free(set);
         free(s);
+    }
+    return err;
+}
+
+/* Block-level selection, the predecessor design (xiawanshe.com report, section
+ * "Token级选择": the previous HySparse picked whole contiguous blocks of
+ * tokens).  From the per-candidate group scores written by hs2o_full_select:
+ * block b holds tokens [b*blk, (b+1)*blk); the candidate blocks are those lying
+ * entirely in [0, t-window], n_blk = (t - window + 1) / blk of them; a block's
+ * score is the sum of its tokens' scores; the first min(topk / blk, n_blk)
+ * blocks in the order (score desc, b asc) are kept and their tokens emitted
+ * ascending, -1 padded to topk.  kth_block (or NULL) gets the score of the last
+ * kept block in rank order (NAN when none is kept).
+ * scores [n_rows, h_kv, score_stride]; idx [n_rows, h_kv, topk]. */
+int hs2o_block_select(int64_t n_rows, int h_kv, int window, int topk, int blk, const int64_t* t,
+                      const double* scores, int64_t score_stride, int32_t* idx, double* kth_block,
+                      double* next_block) {
+    if (n_rows < 0 || h_kv <= 0 || window < 1 || topk < 0 || blk <= 0) return HS2O_EINVAL;
+    int err = HS2O_OK;
+    for (int64_t w = 0; w < n_rows * h_kv; ++w) {
+        const int64_t r = w / h_kv;
+        const int64_t n_cand = t[r] - window + 1 > 0 ? t[r] - window + 1 : 0;
+        const int64_t n_blk = n_cand / blk;
+        const int64_t keep = n_blk < topk / blk ? n_blk : topk / blk;
+        cand_t* cb = (cand_t*)malloc(sizeof(cand_t) * (size_t)(n_blk > 0 ? n_blk : 1));
+        if (!cb) {
+            err = HS2O_ENOMEM;
+            continue;
+        }
+        const double* row = scores + w * score_stride;
+        for (int64_t bb = 0; bb < n_blk; ++bb) {
+            double acc = 0.0;
+            for (int64_t u = 0; u < blk; ++u) acc += row[bb * blk + u];
+            cb[bb].score = acc;
+            cb[bb].j = bb;
+        }
+        qsort(cb, (size_t)n_blk, sizeof(cand_t), cand_cmp);
+        int32_t* row_idx = idx + w * (int64_t)topk;
+        int32_t* blocks = (int32_t*)malloc(sizeof(int32_t) * (size_t)(keep > 0 ? keep : 1));
+        if (!blocks) {
+            free(cb);
+            err = HS2O_ENOMEM;
+            continue;
+        }
+        for (int64_t i = 0; i < keep; ++i) blocks[i] = (int32_t)cb[i].j;
+        qsort(blocks, (size_t)keep, sizeof(int32_t), i32_cmp);
+        for (int64_t i = 0; i < keep; ++i)
+            for (int64_t u = 0; u < blk; ++u) row_idx[i * blk + u] = (int32_t)(blocks[i] * blk + u);
+        for (int64_t i = keep * blk; i < topk; ++i) row_idx[i] = -1;
+        if (kth_block) kth_block[w] = keep > 0 ? cb[keep - 1].score : NAN;
+        if (next_block) next_block[w] = keep < n_blk ? cb[keep].score : -1.0;
+        free(blocks);
+        free(cb);
     }
     return err;
 }

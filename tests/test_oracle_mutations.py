@@ -32,6 +32,11 @@ MUTATIONS = {
     "sparse_window_short": ("const int64_t w0 = tr - window + 1 > 0 ? tr - window + 1 : 0;",
                             "const int64_t w0 = tr - window + 2 > 0 ? tr - window + 2 : 0;", 0),
     "sparse_wrong_group": ("const int h = g * G + hh;", "const int h = hh * h_kv + g;", 2),
+    "block_partial_window": ("const int64_t n_blk = n_cand / blk;", "const int64_t n_blk = (n_cand + blk - 1) / blk;", 0),
+    "block_max_not_sum": ("for (int64_t u = 0; u < blk; ++u) acc += row[bb * blk + u];",
+                          "for (int64_t u = 0; u < blk; ++u) acc = fmax(acc, row[bb * blk + u]);", 0),
+    "block_budget_one_short": ("const int64_t keep = n_blk < topk / blk ? n_blk : topk / blk;",
+                               "const int64_t keep = n_blk < topk / blk ? n_blk : topk / blk - 1;", 0),
     "bridge_k_v_swapped": ("                out_k[r * hd + f] = acc;\n            else\n                out_v[r * hd + (f - hd)] = acc;",
                            "                out_v[r * hd + f] = acc;\n            else\n                out_k[r * hd + (f - hd)] = acc;", 0),
     "bridge_weight_transposed": ("const uint16_t* wf = w + f * (int64_t)d_model;",
@@ -54,6 +59,11 @@ FAST_PINS = [
     pins.test_sparse_with_full_budget_equals_full_attention,
     pins.test_sparse_with_zero_budget_is_sliding_window,
     pins.test_short_context_selects_nothing,
+    pins.test_block_of_one_token_is_the_token_selection,
+    pins.test_block_ties_take_the_lowest_blocks,
+    pins.test_blocks_lie_entirely_before_the_window,
+    pins.test_block_with_planted_key_is_kept,
+    pins.test_block_scores_sum_the_token_scores,
     pins.test_bridge_identity_weights_copy_the_hidden_state,
     pins.test_bridge_feature_layout_by_permuted_one_hot_rows,
     pins.test_bridge_one_hot_hidden_returns_a_weight_column,

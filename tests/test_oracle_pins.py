@@ -466,3 +466,77 @@ def test_bridge_decimal_brute_force():
             for f in range(2 * h_kv * d):
                 ref = sum(decimal.Decimal(float(xb[r, c])) * decimal.Decimal(float(wb[f, c])) for c in range(d_model))
                 assert abs(float(ref) - got[r, f]) <= 1e-12 * max(1.0, abs(float(ref)))
+
+
+# ---------------------------------------------------------------------------
+# Block-level selection (the predecessor design the "Token级选择" section of the
+# xiawanshe.com report contrasts with), at the same budget.
+
+
+def test_block_of_one_token_is_the_token_selection():
+    """Blocks of one token rank exactly like tokens: the same idx as full_select."""
+    rng = np.random.default_rng(31)
+    q, k, v = rand_qkv(rng, 6, 4, 2, 300, 16)
+    t = np.array([0, 130, 131, 200, 250, 299])
+    ref = oracle.full_select(q, t, k, v, window=16, topk=40)
+    got = oracle.block_select(q, t, k, v, window=16, topk=40, block=1)
+    assert np.array_equal(got["idx"], ref["idx"])
+
+
+def test_block_ties_take_the_lowest_blocks():
+    """q = 0: every candidate has the same score, so every block too; the tie rule
+    keeps the lowest-index blocks, i.e. tokens 0 .. K-1."""
+    rng = np.random.default_rng(32)
+    _, k, v = rand_qkv(rng, 1, 4, 2, 700, 8)
+    q = np.zeros((2, 4, 8), np.float32)
+    t = np.array([699, 600])
+    got = oracle.block_select(bits(q), t, k, v, window=128, topk=256, block=64)
+    assert np.array_equal(got["idx"], np.broadcast_to(np.arange(256, dtype=np.int32), (2, 2, 256)))
+
+
+def test_blocks_lie_entirely_before_the_window():
+    """With t - W + 1 = 3 * 64 + 10 candidates only blocks 0..2 are candidates; with
+    a budget of 8 blocks every candidate block is kept and the rest is -1."""
+    rng = np.random.default_rng(33)
+    W, blk = 32, 64
+    t_val = W - 1 + 3 * blk + 10
+    q, k, v = rand_qkv(rng, 1, 2, 1, t_val + 1, 8)
+    got = oracle.block_select(q, np.array([t_val]), k, v, window=W, topk=8 * blk, block=blk)
+    row = got["idx"][0, 0]
+    assert np.array_equal(row[:3 * blk], np.arange(3 * blk))
+    assert np.all(row[3 * blk:] == -1)
+
+
+def test_block_with_planted_key_is_kept():
+    """A key that dominates the probabilities selects its block (budget: 2 blocks of 64)."""
+    rng = np.random.default_rng(34)
+    q = rng.standard_normal((1, 2, 16))
+    qhat = q[0].sum(0) / np.linalg.norm(q[0].sum(0))
+    k = rng.standard_normal((1, 1000, 16)) * 0.3
+    v = rng.standard_normal((1, 1000, 16))
+    k[0, 517] = 200.0 * qhat
+    got = oracle.block_select(bits(q), np.array([999]), bits(k), bits(v), window=128, topk=128, block=64)
+    blocks = sorted(set((got["idx"][0, 0] // 64).tolist()))
+    assert 517 // 64 in blocks
+
+
+def test_block_scores_sum_the_token_scores():
+    """Every block's score equals the sum of its tokens' scores; the kept blocks are
+    the top ones and the best left-out block is below the last kept one."""
+    rng = np.random.default_rng(35)
+    q, k, v = rand_qkv(rng, 3, 4, 2, 900, 16)
+    t = np.array([899, 700, 560])
+    W, K, blk = 64, 256, 64
+    got = oracle.block_select(q, t, k, v, window=W, topk=K, block=blk)
+    sc = got["full"]["scores"]
+    for r in range(3):
+        n_blk = (t[r] - W + 1) // blk
+        for g in range(2):
+            bs = np.array([sc[r, g, b * blk:(b + 1) * blk].sum() for b in range(n_blk)])
+            kept = sorted(set((got["idx"][r, g][got["idx"][r, g] >= 0] // blk).tolist()))
+            order = np.lexsort((np.arange(n_blk), -bs))[:K // blk]
+            assert kept == sorted(order.tolist())
+            assert got["kth_block"][r, g] == pytest.approx(bs[order[-1]], rel=1e-12)
+            rest = np.setdiff1d(np.arange(n_blk), order)
+            if rest.size:
+                assert got["next_block"][r, g] == pytest.approx(bs[rest].max(), rel=1e-12)
