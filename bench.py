@@ -170,6 +170,49 @@ def bench_bridge(w: wl.Workload, dev, K: int, warmup: int, pk: dict) -> dict:
             "frac": round(tf / pk["tc_sustained"], 4), "note": note}
 
 
+def bench_block_select(w: wl.Workload, inp: dict, dev, K: int, warmup: int, pk: dict, flush: torch.Tensor,
+                       token_select_ms: float, blk: int = 64):
+    """Block-level selection at the same budget (a next row of the path: the
+    design token-level selection replaces), through its own C-ABI entry on the
+    same inputs, L2 flushed before every call; per-kernel times from the
+    library's event pairs.  Prefill-shaped workloads only; not part of `value`."""
+    if w.decode:
+        return None
+    shape = nv.shape_of(inp["q"], inp["k"], window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_BLOCK_SELECT, dev)
+    B, Hq, nq, D = inp["q"].shape
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty(B, Hq, nq, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, w.h_kv, nq, w.topk, dtype=torch.int32, device=dev)
+    run = lambda: nv.hs2_full_attn_block_select(shape, blk, inp["q"], inp["k"], inp["v"], out, lse, idx, ws)
+    for _ in range(warmup):
+        flush.zero_()
+        run()
+    torch.cuda.synchronize()
+    nv.hs2_profile_start()
+    for _ in range(K):
+        flush.zero_()
+        run()
+    prof = nv.hs2_profile_stop()
+    st, info = nv.hs2_get_device_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word after block selection: {st} {info}")
+    sweep_ms = prof.get("block_sweep", (0.0, 0))[0] / K
+    topk_ms = prof.get("block_topk", (0.0, 0))[0] / K
+    G = w.h_q // w.h_kv
+    ex2 = G * wl.flops_and_bytes(w)["cand"]
+    res = {"block": blk, "select_ms": round(sweep_ms + topk_ms, 4), "sweep_ms": round(sweep_ms, 4),
+           "topk_ms": round(topk_ms, 4), "token_select_ms": round(token_select_ms, 4),
+           "note": "chunk-sum sweep (every candidate's group probability, summed per 32 keys) + per-row block "
+                   "top-k; token_select_ms = the token-level selection kernels of the timed step"}
+    if sweep_ms > 0 and pk.get("ex2"):
+        achieved = ex2 / (sweep_ms / 1e3) / 1e9
+        res.update({"bound": "alu", "kernel": "block_sweep", "achieved": round(achieved, 2),
+                    "peak": round(pk["ex2"] / 1e9, 1), "unit": "Gex2/s",
+                    "frac": round(achieved / (pk["ex2"] / 1e9), 4)})
+    return res
+
+
 def source_sha(path: str) -> str:
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
@@ -519,6 +562,11 @@ def run_ours(args):
     pk["ex2"] = ex2_rate
     rf, per_kernel = roofline(w, prof, args.steps, pk)
     next_rows = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
+    sel_kernels = ("select_score", "select_thresh", "select_filter", "select_retry", "select_topk")
+    token_sel_ms = sum(per_kernel[n]["ms"] for n in sel_kernels if n in per_kernel)
+    blk = bench_block_select(w, inp, dev, args.steps, args.warmup, pk, flush, token_sel_ms)
+    if blk is not None:
+        next_rows["block_select"] = blk
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
 

@@ -88,7 +88,8 @@ enum {
     HS2_ENTRY_FULL_SELECT = 0,
     HS2_ENTRY_SPARSE = 1,
     HS2_ENTRY_PREFILL = 2,
-    HS2_ENTRY_DECODE = 3
+    HS2_ENTRY_DECODE = 3,
+    HS2_ENTRY_BLOCK_SELECT = 4
 };
 
 /* Bytes of workspace the entry point `entry` needs for `shape` (0 if the shape
@@ -119,6 +120,26 @@ hs2_status hs2_full_attn_select(const hs2_shape* shape, const void* q, const voi
 hs2_status hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v,
                            const int32_t* idx, void* out, void* ws, size_t ws_bytes,
                            hs2_stream_t stream);
+
+/* The full-attention layer with BLOCK-level selection at the same budget, the
+ * design token-level selection replaces (xiawanshe.com report, section
+ * "Token级选择": the earlier HySparse chose whole blocks of contiguous tokens).
+ * Same arguments, layouts and outputs as hs2_full_attn_select (any q_pos0, so
+ * it also serves prefill chunks), plus the block size.  Definitions:
+ *   block bb = keys [bb*block, (bb+1)*block), block in {32, 64, 128};
+ *   candidate blocks: those lying wholly in [0, t-window], n_blk(t) =
+ *   (t-window+1) / block of them (a partial block next to the window is not a
+ *   candidate);
+ *   block score = sum of score_{g,j} over the block's keys;
+ *   idx_g(t) = the keys of the first min(topk / block, n_blk) blocks in the
+ *   order (block score descending, bb ascending), stored ascending, then -1
+ *   padding up to topk entries.
+ * Any other block size returns HS2_ERR_UNSUPPORTED.  ws:
+ * hs2_workspace_size(shape, HS2_ENTRY_BLOCK_SELECT) bytes.  The output feeds
+ * hs2_sparse_attn unchanged. */
+hs2_status hs2_full_attn_block_select(const hs2_shape* shape, int32_t block, const void* q, const void* k,
+                                      const void* v, void* out, float* lse, int32_t* idx, void* ws,
+                                      size_t ws_bytes, hs2_stream_t stream);
 
 /* Prefill-chunk entry: the full-attention + selection layer for a chunk of
  * n_q new tokens appended to a cache of kv_len tokens (q_pos0 = kv_len - n_q
@@ -201,7 +222,7 @@ uint64_t hs2_launch_count(void);
  * 2 selection scores, 3 top-k select, 4 sparse attention, 5 decode attention
  * partials, 6 decode combine, 7 fused attention + selection, 8 selection
  * threshold estimate, 9 filtered selection sweep, 10 selection retry,
- * 11 KV bridging. */
+ * 11 KV bridging, 12 block-selection score sweep, 13 block top-k. */
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 

@@ -203,6 +203,65 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
     return HS2_OK;
 }
 
+// Block-level selection plan: chunk sums of every candidate tile, over chunks
+// of queries whose sums fit kScoreBudget.
+struct BlockPlan {
+    int64_t n_cand_max = 0;
+    int chunk = 0;
+    size_t bytes = 0;
+};
+
+BlockPlan block_plan(const Problem& p) {
+    BlockPlan bp;
+    const int64_t cand = p.q_pos0 + p.nq - p.window;  // candidates of the last query
+    if (cand <= 0 || p.nq == 0 || p.B == 0 || p.topk == 0) return bp;
+    bp.n_cand_max = cand;
+    const size_t per_q = block_tc_scratch_bytes(p, 1, cand);
+    int64_t chunk = (int64_t)(kScoreBudget / per_q) / 32 * 32;
+    if (chunk < 32) chunk = 32;
+    if (chunk > p.nq) chunk = p.nq;
+    bp.chunk = (int)chunk;
+    bp.bytes = block_tc_scratch_bytes(p, bp.chunk, cand);
+    return bp;
+}
+
+size_t block_body_bytes(const Problem& p) {
+    const size_t split = full_tc_split_scratch_bytes(p);
+    const size_t sel = block_plan(p).bytes;
+    return sel > split ? sel : split;
+}
+
+bool valid_block(int blk) { return blk == 32 || blk == 64 || blk == 128; }
+
+hs2_status run_block_select(const hs2_shape* shape, int blk, const void* q, const void* k, const void* v, void* out,
+                            float* lse, int32_t* idx, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (!valid_block(blk)) return HS2_ERR_UNSUPPORTED;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k || !v || !out || !lse || !ws) return HS2_ERR_INVALID_ARG;
+    if (p.topk > 0 && !idx) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(idx, 4) || !aligned(ws, 256))
+        return HS2_ERR_INVALID_ARG;
+    if (ws_bytes < kHeader + block_body_bytes(p)) return HS2_ERR_WORKSPACE;
+    p.err = reinterpret_cast<WsHeader*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* body = reinterpret_cast<uint8_t*>(ws) + kHeader;
+    cudaError_t e = launch_full(p, q, k, v, out, lse, body, ws_bytes - kHeader, st);
+    if (e != cudaSuccess) return HS2_ERR_CUDA;
+    if (p.topk == 0) return HS2_OK;
+    const BlockPlan bp = block_plan(p);
+    const int chunk = bp.chunk > 0 ? bp.chunk : p.nq;
+    for (int i0 = 0; i0 < p.nq; i0 += chunk) {
+        const int cnt = p.nq - i0 < chunk ? p.nq - i0 : chunk;
+        e = launch_block_select_tc(p, q, k, lse, idx, body, i0, cnt, bp.n_cand_max, blk, st);
+        if (e != cudaSuccess) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
 }  // namespace
 }  // namespace hs2
 
@@ -217,6 +276,7 @@ size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
         case HS2_ENTRY_SPARSE: return kHeader;
         case HS2_ENTRY_FULL_SELECT:
         case HS2_ENTRY_PREFILL: return kHeader + prefill_body_bytes(p, score_plan(p, false));
+        case HS2_ENTRY_BLOCK_SELECT: return kHeader + block_body_bytes(p);
         case HS2_ENTRY_DECODE: {
             if (p.nq != 1) return 0;
             return kHeader + (score_plan(p, true).bytes + 255) / 256 * 256 + decode_scratch_bytes(p);
@@ -233,6 +293,12 @@ hs2_status hs2_workspace_init(void* ws, size_t ws_bytes, hs2_stream_t stream) {
 hs2_status hs2_full_attn_select(const hs2_shape* shape, const void* q, const void* k, const void* v, void* out,
                                 float* lse, int32_t* idx, void* ws, size_t ws_bytes, hs2_stream_t stream) {
     return run_full_select(shape, nullptr, false, q, k, v, out, lse, idx, ws, ws_bytes, stream);
+}
+
+hs2_status hs2_full_attn_block_select(const hs2_shape* shape, int32_t block, const void* q, const void* k,
+                                      const void* v, void* out, float* lse, int32_t* idx, void* ws, size_t ws_bytes,
+                                      hs2_stream_t stream) {
+    return run_block_select(shape, block, q, k, v, out, lse, idx, ws, ws_bytes, stream);
 }
 
 hs2_status hs2_prefill_chunk(const hs2_shape* shape, const void* q, const void* k, const void* v, void* out,

@@ -34,6 +34,8 @@ enum KernelId : uint32_t {
     KID_FILTER = 9,
     KID_RETRY = 10,
     KID_BRIDGE = 11,
+    KID_BLOCK_SWEEP = 12,
+    KID_BLOCK_TOPK = 13,
 };
 
 __device__ __forceinline__ void report_error(WsHeader* h, uint32_t code, uint32_t kid, uint32_t a,

@@ -58,6 +58,13 @@ cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, 
 // K2 on tcgen05 for prefill-shaped calls: sampled threshold, filtered sweep
 // with on-chip survivor lists, exact final top-k, retry of underestimated rows.
 size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
+// Block-level selection (blocks of `blk` in {32, 64, 128} keys): the chunk-sum
+// sweep over the tensor cores, then the per-row block top-k.  Scratch: the
+// chunk sums, block_tc_scratch_bytes(p, i_count, n_cand_max) bytes.
+size_t block_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
+cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
+                                   void* scratch, int i_begin, int i_count, int64_t n_cand_max, int blk,
+                                   cudaStream_t st);
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
                              void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st);
 

@@ -56,7 +56,7 @@ constexpr int SL_CMAX = 4096;      // survivor list capacity per row
 constexpr int SL_SLOTS = 256;      // per-SM survivor slots (indexed by %smid)
 constexpr int SL_MIN_SMEM = 120 * 1024;  // keeps one CTA per SM (slots are per SM)
 
-enum { MODE_SAMPLE = 0, MODE_FILTER = 1, MODE_RETRY = 2 };
+enum { MODE_SAMPLE = 0, MODE_FILTER = 1, MODE_RETRY = 2, MODE_BLOCK = 3 };
 
 template <int D, int G>
 struct SlCfg {
@@ -95,6 +95,8 @@ struct SelArgs {
     int cmax;               // survivor list capacity per row
     int slot_by_block;      // 1: slot = block id (small grids); 0: slot = %smid (one CTA per SM)
     int64_t sample_stride;  // S: the sampling pass reads keys 0, S, 2S, ...
+    float* csum;            // block mode: [rows][cstride] sums of 32 consecutive candidate scores
+    int64_t cstride;
 };
 
 __device__ __forceinline__ uint32_t smid() {
@@ -239,7 +241,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         if (!need) return;
     }
     const uint32_t slot = a.slot_by_block ? (blockIdx.z * gridDim.y + blockIdx.y) * gridDim.x + blockIdx.x : smid();
-    if (MODE != MODE_SAMPLE && slot >= SL_SLOTS) {
+    if ((MODE == MODE_FILTER || MODE == MODE_RETRY) && slot >= SL_SLOTS) {
         if (tid == 0) report_error(p.err, HS2_ERR_DEVICE_CHECK, KID_SCORE, slot, 0);
         return;
     }
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 break;
             }
             tc::fence_after_sync();
-            if constexpr (MODE != MODE_SAMPLE) {
+            if constexpr (MODE == MODE_FILTER || MODE == MODE_RETRY) {
                 // rare: a list that could overflow on this tile is first cut to its exact
                 // top K; later keys (larger j) then need a score strictly above its K-th entry
                 // every warp reads the counts before any of them changes (uniform decision)
@@ -432,7 +434,27 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
             tc::fence_before_sync();
             tc::mbar_arrive(bar(SB_SEMPTY + sb));
 
-            if constexpr (MODE == MODE_SAMPLE) {
+            if constexpr (MODE == MODE_BLOCK) {
+                // sum of the warp's 32 keys for each of its QH = 8 queries, as a
+                // transposing butterfly: every exchange halves the values a lane holds,
+                // so lane l ends with query l >> 2 summed over all 32 lanes (9 shuffles
+                // instead of 8 x 5)
+                static_assert(QH == 8, "the butterfly below reduces 8 query columns");
+                float h4[4], h2[2], h1;
+                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                    h4[u] = (b4 ? sc[4 + u] : sc[u]) + __shfl_xor_sync(0xffffffffu, b4 ? sc[u] : sc[4 + u], 16);
+#pragma unroll
+                for (int u = 0; u < 2; ++u)
+                    h2[u] = (b3 ? h4[2 + u] : h4[u]) + __shfl_xor_sync(0xffffffffu, b3 ? h4[u] : h4[2 + u], 8);
+                h1 = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h2[0] : h2[1], 4);
+                h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
+                h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
+                const int q = wg * QH + (lane >> 2);
+                if ((lane & 3) == 0 && q < nq_here)
+                    a.csum[(row0 + q) * a.cstride + (jb >> 5) + kq] = h1;
+            } else if constexpr (MODE == MODE_SAMPLE) {
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
                     const int q = wg * QH + qq;
@@ -477,8 +499,10 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 }
             }
         }
-        if constexpr (MODE != MODE_SAMPLE) named_sync(barid, 128);  // every append is in place
-        if constexpr (MODE == MODE_SAMPLE) {
+        if constexpr (MODE == MODE_FILTER || MODE == MODE_RETRY) named_sync(barid, 128);  // every append is in place
+        if constexpr (MODE == MODE_BLOCK) {
+            // nothing after the sweep: the chunk sums are the output
+        } else if constexpr (MODE == MODE_SAMPLE) {
             // unused sample slots hold 0 (they rank below every valid sample)
             for (int it2 = n_tiles; it2 < SL_SAMPLE_TILES; ++it2)
                 for (int qq = 0; qq < QH; ++qq) {
@@ -571,6 +595,69 @@ __global__ void __launch_bounds__(128) k2_thresh_kernel(Problem p, SelArgs a) {
     if (lane == 0) a.tau[row] = tau;
 }
 
+// Block-level selection of one (query, group) row per warp from the chunk sums
+// of the block sweep.  Block bb of size blk covers keys [bb blk, (bb + 1) blk);
+// the candidate blocks are those lying wholly in [0, t - window], and the first
+// keep = min(topk / blk, n_blk) of them in the order (score desc, bb asc) are
+// kept, their keys written ascending, -1 padded to topk.  The warp first turns
+// the row's chunk sums into block sums in place (block bb's chunks sit at or
+// after position bb, so no unread chunk is overwritten), then runs the exact
+// radix select on them.
+__global__ void __launch_bounds__(128) k2_block_topk_kernel(Problem p, SelArgs a, int blk) {
+    __shared__ uint32_t hist[4][256];
+    __shared__ int32_t kept[4][64];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)p.B * p.hkv * a.i_count;
+    const int64_t row = (int64_t)blockIdx.x * 4 + warp;
+    if (row >= rows) return;
+    const int qi = (int)(row % a.i_count);
+    const int bg = (int)(row / a.i_count);  // b * H_kv + g
+    const int b = bg / p.hkv;
+    const int64_t t = seq_pos0(p, b, KID_TOPK) + a.i_begin + qi;
+    const int64_t n_cand = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
+    const int n_blk = (int)(n_cand / blk);
+    const int keep = min(p.topk / blk, n_blk);
+    int32_t* orow = a.idx + ((int64_t)bg * p.nq + a.i_begin + qi) * p.topk;
+    if (keep == n_blk || keep == 0) {  // every candidate block is kept (or none fits the budget)
+        for (int u = lane; u < p.topk; u += 32) orow[u] = u < keep * blk ? u : -1;
+        return;
+    }
+    float* cs = a.csum + row * a.cstride;
+    const int nc = blk / 32;  // chunks per block
+    if (nc > 1) {
+        for (int base = 0; base < n_blk; base += 32) {
+            const int bb = base + lane;
+            float acc = 0.f;
+            if (bb < n_blk)
+                for (int c = 0; c < nc; ++c) acc += cs[(int64_t)bb * nc + c];
+            __syncwarp();
+            if (bb < n_blk) cs[bb] = acc;
+            __syncwarp();
+        }
+    }
+    uint32_t kth, need_eq;
+    warp_kth(reinterpret_cast<const uint32_t*>(cs), 1, n_blk, (uint32_t)keep, hist[warp], kth, need_eq);
+    // ordered keep: blocks above the k-th score plus the lowest-index equal ones
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t eq_seen = 0, written = 0;
+    for (int base = 0; base < n_blk; base += 32) {
+        const int bb = base + lane;
+        const uint32_t x = bb < n_blk ? __float_as_uint(cs[bb]) : 0u;
+        const bool eq = bb < n_blk && x == kth;
+        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
+        const bool take = (bb < n_blk && x > kth) || (eq && eq_seen + __popc(eqb & lt) < need_eq);
+        const uint32_t tb = __ballot_sync(0xffffffffu, take);
+        if (take) kept[warp][written + __popc(tb & lt)] = bb;
+        eq_seen += __popc(eqb);
+        written += __popc(tb);
+    }
+    __syncwarp();
+    for (int u = lane; u < p.topk; u += 32) {
+        const int i = u / blk;
+        orow[u] = i < keep ? kept[warp][i] * blk + (u - i * blk) : -1;
+    }
+}
+
 // [B][H_q][n_q][D] bf16 seen as (D, H_q, n_q, B) with box (64, G, 32, 1): the
 // shared-memory tile rows come out ordered (query, head), 128 bytes each.
 bool make_q_map(CUtensorMap* m, const void* base, int D, int hq, int nq, int B, int G) {
@@ -594,7 +681,11 @@ cudaError_t launch_mode(const Problem& p, const CUtensorMap& mq, const CUtensorM
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     dim3 grid((a.i_count + SL_QT - 1) / SL_QT, p.hkv, p.B);
-    prof_begin(MODE == MODE_SAMPLE ? KID_SCORE : MODE == MODE_FILTER ? KID_FILTER : KID_RETRY, st);
+    prof_begin(MODE == MODE_SAMPLE   ? KID_SCORE
+               : MODE == MODE_FILTER ? KID_FILTER
+               : MODE == MODE_RETRY  ? KID_RETRY
+                                     : KID_BLOCK_SWEEP,
+               st);
     kern<<<grid, SL_THREADS, C::SMEM, st>>>(mq, mk, p, a);
     prof_end(st);
     count_launch();
@@ -631,6 +722,24 @@ cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, con
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = launch_mode<D, G, MODE_FILTER>(p, mq, mk, a, st)) != cudaSuccess) return e;
     return launch_mode<D, G, MODE_RETRY>(p, mq, mk, a, st);
+}
+
+template <int D, int G>
+cudaError_t launch_block_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+    CUtensorMap mq, mk;
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
+        return cudaErrorInvalidValue;
+    return launch_mode<D, G, MODE_BLOCK>(p, mq, mk, a, st);
+}
+
+template <int D>
+cudaError_t launch_block_d(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+    switch (p.hq / p.hkv) {
+        case 1: return launch_block_dg<D, 1>(p, q, k, a, st);
+        case 2: return launch_block_dg<D, 2>(p, q, k, a, st);
+        case 4: return launch_block_dg<D, 4>(p, q, k, a, st);
+        default: return launch_block_dg<D, 8>(p, q, k, a, st);
+    }
 }
 
 template <int D>
@@ -687,6 +796,37 @@ cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, con
     a.i_count = i_count;
     if (p.D == 64) return launch_select_d<64>(p, q, k, a, st);
     return launch_select_d<128>(p, q, k, a, st);
+}
+
+// Chunk sums: one float per 32 keys of every candidate tile, rows of cstride.
+static int64_t block_cstride(int64_t n_cand_max) { return (n_cand_max + SL_BN - 1) / SL_BN * (SL_BN / 32); }
+
+size_t block_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max) {
+    if (n_cand_max <= 0) return 0;
+    return (size_t)p.B * p.hkv * i_count * block_cstride(n_cand_max) * 4;
+}
+
+cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
+                                   void* scratch, int i_begin, int i_count, int64_t n_cand_max, int blk,
+                                   cudaStream_t st) {
+    SelArgs a{};
+    a.lse = lse;
+    a.idx = idx;
+    a.i_begin = i_begin;
+    a.i_count = i_count;
+    a.csum = reinterpret_cast<float*>(scratch);
+    a.cstride = block_cstride(n_cand_max);
+    // the sweep only runs when some row has more candidate blocks than the budget
+    if (n_cand_max / blk > p.topk / blk && p.topk >= blk) {
+        const cudaError_t e = p.D == 64 ? launch_block_d<64>(p, q, k, a, st) : launch_block_d<128>(p, q, k, a, st);
+        if (e != cudaSuccess) return e;
+    }
+    const int64_t rows = (int64_t)p.B * p.hkv * i_count;
+    prof_begin(KID_BLOCK_TOPK, st);
+    k2_block_topk_kernel<<<(unsigned)((rows + 3) / 4), 128, 0, st>>>(p, a, blk);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
 }
 
 }  // namespace hs2

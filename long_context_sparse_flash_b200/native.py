@@ -21,17 +21,18 @@ HS2_OK = 0
 STATUS = {0: "HS2_OK", 1: "HS2_ERR_INVALID_ARG", 2: "HS2_ERR_UNSUPPORTED", 3: "HS2_ERR_WORKSPACE",
           4: "HS2_ERR_CUDA", 5: "HS2_ERR_DEVICE_CHECK", 6: "HS2_ERR_TIMEOUT"}
 HS2_ENTRY_FULL_SELECT, HS2_ENTRY_SPARSE, HS2_ENTRY_PREFILL, HS2_ENTRY_DECODE = 0, 1, 2, 3
+HS2_ENTRY_BLOCK_SELECT = 4
 
 # every symbol include/hs2.h declares
 EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_sparse_attn",
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
-           "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge")
+           "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
-                10: "select_retry", 11: "kv_bridge"}
+                10: "select_retry", 11: "kv_bridge", 12: "block_sweep", 13: "block_topk"}
 
 
 class HS2Error(RuntimeError):
@@ -76,6 +77,7 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_workspace_init.argtypes = [P, S, P]
     lib.hs2_full_attn_select.argtypes = [sh, P, P, P, P, P, P, P, S, P]
     lib.hs2_prefill_chunk.argtypes = [sh, P, P, P, P, P, P, P, S, P]
+    lib.hs2_full_attn_block_select.argtypes = [sh, ctypes.c_int32, P, P, P, P, P, P, P, S, P]
     lib.hs2_decode.argtypes = [sh, P, P, P, P, P, P, P, P, S, P]
     lib.hs2_sparse_attn.argtypes = [sh, P, P, P, P, P, P, S, P]
     lib.hs2_decode_sparse.argtypes = [sh, P, P, P, P, P, P, P, S, P]
@@ -97,7 +99,7 @@ def load(checked: bool = False) -> ctypes.CDLL:
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
-                 "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge"):
+                 "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -167,6 +169,13 @@ def hs2_full_attn_select(shape, q, k, v, out, lse, idx, ws, stream=None, checked
     _check(load(checked).hs2_full_attn_select(ctypes.byref(shape), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                               _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
            "hs2_full_attn_select")
+
+
+def hs2_full_attn_block_select(shape, block, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_full_attn_block_select(ctypes.byref(shape), int(block), _ptr(q), _ptr(k), _ptr(v),
+                                                    _ptr(out), _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
+           "hs2_full_attn_block_select")
 
 
 def hs2_prefill_chunk(shape, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
@@ -298,6 +307,20 @@ def full_attn_select(q, k, v, *, window: int, topk: int, q_pos0: int = 0, ws=Non
     idx = torch.empty(B, k.shape[1], nq, topk, dtype=torch.int32, device=q.device)
     fn = hs2_prefill_chunk if entry == "prefill" else hs2_full_attn_select
     fn(shape, q, k, v, out, lse, idx, ws, stream, checked)
+    return out, lse, idx
+
+
+def full_attn_block_select(q, k, v, *, window: int, topk: int, block: int, q_pos0: int = 0, ws=None,
+                           stream=None, checked: bool = False):
+    """Allocate out/lse/idx and run hs2_full_attn_block_select."""
+    shape = shape_of(q, k, window=window, topk=topk, q_pos0=q_pos0)
+    if ws is None:
+        ws = alloc_workspace(shape, HS2_ENTRY_BLOCK_SELECT, q.device, checked, stream)
+    out = torch.empty_like(q)
+    B, Hq, nq, D = q.shape
+    lse = torch.empty(B, Hq, nq, dtype=torch.float32, device=q.device)
+    idx = torch.empty(B, k.shape[1], nq, topk, dtype=torch.int32, device=q.device)
+    hs2_full_attn_block_select(shape, block, q, k, v, out, lse, idx, ws, stream, checked)
     return out, lse, idx
 
 

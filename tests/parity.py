@@ -74,6 +74,47 @@ def check_idx(gpu_idx: np.ndarray, ores: dict, ts: np.ndarray, window: int, topk
     return stats
 
 
+def check_block_idx(gpu_idx: np.ndarray, ores: dict, ts: np.ndarray, window: int, topk: int, blk: int,
+                    what="block idx") -> dict:
+    """gpu_idx [n_rows, H_kv, topk]; ores from oracle.block_select.  Every row: the
+    first keep * blk entries are keep whole candidate blocks, ascending, then -1;
+    the GPU's block set equals the oracle's except for blocks whose oracle score
+    lies within min(blk * 1e-6, 2e-4 * kth) of the oracle's last kept block (the
+    token near-tie rule, scaled to a sum of blk token scores)."""
+    n_rows, h_kv, _ = gpu_idx.shape
+    stats = dict(rows=0, rows_differing=0, max_sym_diff=0)
+    sc = ores["full"]["scores"]
+    for r in range(n_rows):
+        t = int(ts[r])
+        n_blk = max(0, t - window + 1) // blk
+        keep = min(topk // blk, n_blk)
+        for g in range(h_kv):
+            row = gpu_idx[r, g]
+            assert np.all(row[keep * blk:] == -1), f"{what} row t={t} g={g}: bad padding"
+            body = row[:keep * blk].reshape(keep, blk) if keep else np.zeros((0, blk), np.int32)
+            starts = body[:, 0]
+            assert np.all(starts % blk == 0), f"{what} row t={t} g={g}: block not aligned"
+            assert np.array_equal(body, starts[:, None] + np.arange(blk)[None, :]), \
+                f"{what} row t={t} g={g}: block not contiguous"
+            if keep:
+                assert np.all(np.diff(starts) > 0), f"{what} row t={t} g={g}: blocks not ascending"
+                assert starts[-1] // blk < n_blk, f"{what} row t={t} g={g}: block beyond the candidates"
+            got = set((starts // blk).tolist())
+            want = set((ores["idx"][r, g, :keep * blk:blk] // blk).tolist())
+            stats["rows"] += 1
+            diff = got ^ want
+            if diff:
+                kth = float(ores["kth_block"][r, g])
+                margin = min(blk * IDX_ABS_MARGIN, IDX_REL_MARGIN * kth)
+                for bb in diff:
+                    gap = abs(float(sc[r, g, bb * blk:(bb + 1) * blk].sum()) - kth)
+                    assert gap <= margin, (f"{what} row t={t} g={g}: block {bb} differs with score gap "
+                                           f"{gap:.3g} > margin {margin:.3g} (kth {kth:.6g})")
+                stats["rows_differing"] += 1
+                stats["max_sym_diff"] = max(stats["max_sym_diff"], len(diff))
+    return stats
+
+
 def run_gpu(w: wl.Workload, inp: dict, entry: str = "full", checked: bool = False, seq_len=None):
     """Full-attention + selection layer, then every sparse layer, through the C ABI."""
     q, k, v = inp["q"], inp["k"], inp["v"]

@@ -186,3 +186,31 @@ def test_kv_bridge_validation_without_launch():
     assert call(bs(n_new=0)) == 0                # empty: no launch
     assert call(bs(batch=0)) == 0
     assert nv.hs2_launch_count() == before
+
+
+def test_block_select_validation_without_launch():
+    """Block-level selection entry: block size, workspace, pointers, empty calls."""
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    s = shape(n_q=4096, kv_len=4096)
+    need = nv.hs2_workspace_size(s, nv.HS2_ENTRY_BLOCK_SELECT)
+    # one float per 32 candidate keys of every 128-key tile, for every (query, group) row
+    cand = 4096 - 128
+    assert need == 256 + 4 * 4096 * (-(-cand // 128) * 4) * 4
+    args = [FAKE] * 7
+
+    def call(sh, blk, *a, ws_bytes=need):
+        return L.hs2_full_attn_block_select(ctypes.byref(sh) if sh is not None else None, blk, *a, ws_bytes, None)
+
+    for blk in (0, 16, 48, 96, 256, -64):
+        assert call(s, blk, *args) == 2
+    assert call(None, 64, *args) == 1
+    assert call(s, 64, None, *args[1:]) == 1
+    assert call(s, 64, *args, ws_bytes=need - 1) == 3
+    assert call(s, 64, ctypes.c_void_p((1 << 40) + 8), *args[1:]) == 1
+    assert call(shape(h_q=30), 64, *args) == 1
+    for kw in (dict(batch=0), dict(n_q=0)):
+        assert call(shape(**kw), 64, None, None, None, None, None, None, None, ws_bytes=0) == 0
+    # no candidate at all: the header only (plus the full layer's own split scratch, none here)
+    assert nv.hs2_workspace_size(shape(n_q=100, kv_len=100), nv.HS2_ENTRY_BLOCK_SELECT) == 256
+    assert nv.hs2_launch_count() == before
