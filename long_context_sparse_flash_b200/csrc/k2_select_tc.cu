@@ -370,11 +370,10 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 // top K; later keys (larger j) then need a score strictly above its K-th entry
                 // every warp reads the counts before any of them changes (uniform decision)
                 uint32_t need = 0;
-                int cnts[QH];
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
-                    cnts[qq] = r_cnt[(it & 1) * SL_QT + wg * QH + qq];
-                    if (cnts[qq] > cmax - SL_BN && cnts[qq] > p.topk) need |= 1u << qq;
+                    const int c = r_cnt[(it & 1) * SL_QT + wg * QH + qq];
+                    if (c > cmax - SL_BN && c > p.topk) need |= 1u << qq;
                 }
                 if (need) {
                     named_sync(barid, 128);
@@ -383,7 +382,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                         if (!((need >> qq) & 1u)) continue;
                         const int q = wg * QH + qq;
                         uint2* lst = lists + (int64_t)q * cmax;
-                        const int cnt = min(cnts[qq], cmax);
+                        const int cnt = min(r_cnt[(it & 1) * SL_QT + q], cmax);  // only this warp changes it
                         uint32_t kth, need_eq;
                         warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)p.topk, hist + warp * 256,
                                  kth, need_eq);

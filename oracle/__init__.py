@@ -20,6 +20,9 @@ Method (HySparse2 pages: xiawanshe.com report, sections "两级KV共享" /
   over idx U window(t).
 * ``block_select`` -- the predecessor block-level selection at the same
   budget: whole blocks of contiguous candidates, ranked by summed score.
+* ``branches`` -- the predecessor design's sparse layer: a sliding-window
+  branch over its own cache and a selected-tokens branch over the shared one,
+  each with its own softmax (outputs and LSEs, uncombined).
 * ``kv_bridge`` -- KV bridging (same report, section "两级KV共享", first
   level): a token's Cross-Decoder K and V from its Self-Decoder hidden state by
   one projection, output features [K heads | V heads], D per head.
@@ -70,6 +73,9 @@ def open_library(path: str):
     lib.hs2o_block_select.argtypes = [i64, i32, i32, i32, i32, P, P, i64, P, P, P]
     lib.hs2o_block_select.restype = i32
     lib.hs2o_kv_bridge.restype = i32
+    lib.hs2o_branches.argtypes = [i32, i32, i32, i32, i32, ctypes.c_double, i64, P, P, P, P, P, P, i64, P,
+                                  P, P, P, P, i32]
+    lib.hs2o_branches.restype = i32
     lib.hs2o_max_threads.argtypes = []
     lib.hs2o_max_threads.restype = i32
     return lib
@@ -200,3 +206,31 @@ def block_select(q_rows, t, k, v, *, window: int, topk: int, block: int, scale: 
     if rc != 0:
         raise ValueError(f"hs2o_block_select: error {rc}")
     return dict(idx=idx, kth_block=kth, next_block=nxt, full=full)
+
+
+def branches(q_rows, t, k_swa, v_swa, k, v, idx, *, window: int, scale: float | None = None,
+             n_threads: int = 0):
+    """The two branches of a predecessor-design sparse layer for query rows of ONE
+    sequence: returns dict(out_swa, lse_swa, out_sel, lse_sel); out [n, H_q, D]
+    f64, lse [n, H_q] f64 (natural log; -inf for a row with no selected key).
+    k_swa, v_swa: the window branch's own cache; k, v: the shared cache, all
+    uint16 [H_kv, kv_len, D]; idx int32 [n, H_kv, topk]."""
+    q_rows = _as_bits(q_rows)
+    k_swa, v_swa, k, v = _as_bits(k_swa), _as_bits(v_swa), _as_bits(k), _as_bits(v)
+    t = np.ascontiguousarray(t, dtype=np.int64)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    n, h_q, d = q_rows.shape
+    h_kv, kv_len, _ = k.shape
+    assert k_swa.shape == k.shape and v_swa.shape == k.shape and v.shape == k.shape
+    assert idx.shape[:2] == (n, h_kv)
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    res = dict(out_swa=np.zeros((n, h_q, d)), lse_swa=np.zeros((n, h_q)),
+               out_sel=np.zeros((n, h_q, d)), lse_sel=np.zeros((n, h_q)))
+    rc = _load().hs2o_branches(h_q, h_kv, d, window, idx.shape[2], float(scale), n, _ptr(t), _ptr(q_rows),
+                               _ptr(k_swa), _ptr(v_swa), _ptr(k), _ptr(v), kv_len, _ptr(idx),
+                               _ptr(res["out_swa"]), _ptr(res["lse_swa"]), _ptr(res["out_sel"]),
+                               _ptr(res["lse_sel"]), int(n_threads))
+    if rc != 0:
+        raise RuntimeError(f"hs2o_branches failed with code {rc}")
+    return res

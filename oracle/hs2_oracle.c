@@ -33,6 +33,10 @@
  *   - block-level selection (the predecessor design the "Token级选择" section
  *     contrasts with) keeps whole blocks of blk contiguous candidate tokens,
  *     blocks ranked by the sum of their tokens' scores, at the same budget;
+ *   - the predecessor design's sparse layer had two branches, a sliding-window
+ *     attention over its own cache and an attention over the selected tokens
+ *     of the shared cache; both are returned, uncombined (the pages do not
+ *     say how they were combined);
  *   - "KV Bridging" (same report and section, first level) computes a token's
  *     K and V from its Self-Decoder hidden state with one projection (no
  *     bias, no normalisation or position encoding: the pages name none); the
@@ -282,6 +286,115 @@ int hs2o_sparse(int h_q, int h_kv, int d, int window, int topk, double scale,
             }
         }
         free(set);
+        free(s);
+    }
+    return err;
+}
+
+/* Softmax attention of one fp64 query over the n rows set[] of one head's K/V:
+ * out = sum_u p_u v_{set[u]}, p_u = exp(s_u - lse), s_u = scale <q, k_{set[u]}>,
+ * lse = ln sum_u exp(s_u).  n = 0 gives out = 0 and lse = -inf. */
+static void attend_rows(const double* qd, const uint16_t* kg, const uint16_t* vg, const int64_t* set, int64_t n,
+                        int d, double scale, double* s, double* out, double* lse) {
+    for (int e = 0; e < d; ++e) out[e] = 0.0;
+    if (n == 0) {
+        *lse = -INFINITY;
+        return;
+    }
+    double m = -INFINITY;
+    for (int64_t u = 0; u < n; ++u) {
+        const uint16_t* kj = kg + set[u] * (int64_t)d;
+        double acc = 0.0;
+        for (int e = 0; e < d; ++e) acc += qd[e] * bf16_to_double(kj[e]);
+        s[u] = acc * scale;
+        m = s[u] > m ? s[u] : m;
+    }
+    double z = 0.0;
+    for (int64_t u = 0; u < n; ++u) z += exp(s[u] - m);
+    for (int64_t u = 0; u < n; ++u) {
+        const double pu = exp(s[u] - m) / z;
+        const uint16_t* vj = vg + set[u] * (int64_t)d;
+        for (int e = 0; e < d; ++e) out[e] += pu * bf16_to_double(vj[e]);
+    }
+    *lse = m + log(z);
+}
+
+/* The two attention branches of a sparse layer in the predecessor design
+ * (xiawanshe.com report, section "Token级选择": HySparse2 drops the separate
+ * sliding-window branch of the Cross-Decoder and keeps the recent tokens in
+ * the one shared cache instead).  Per row and head h (g = h / G):
+ *   window branch:   softmax attention over window(t) = [max(0, t-W+1), t] of
+ *                    the branch's OWN cache k_swa, v_swa;
+ *   selected branch: softmax attention over the selected set idx_g(t) alone
+ *                    (no window) of the shared cache k, v.
+ * Each writes its output [n_rows, h_q, d] and natural-log LSE [n_rows, h_q];
+ * a row with no selected key gets a zero output and LSE -inf.  The pages do
+ * not say how the predecessor combined the two branches, so both are
+ * returned.  idx entries are -1 or a candidate index in [0, t-W], no
+ * duplicates (HS2O_EIDX otherwise). */
+int hs2o_branches(int h_q, int h_kv, int d, int window, int topk, double scale, int64_t n_rows, const int64_t* t,
+                  const uint16_t* q, const uint16_t* k_swa, const uint16_t* v_swa, const uint16_t* k,
+                  const uint16_t* v, int64_t kv_len, const int32_t* idx, double* out_swa, double* lse_swa,
+                  double* out_sel, double* lse_sel, int n_threads) {
+    if (h_q <= 0 || h_kv <= 0 || h_q % h_kv != 0 || d <= 0 || d > 512 || window < 1 || topk < 0 || n_rows < 0)
+        return HS2O_EINVAL;
+    for (int64_t r = 0; r < n_rows; ++r)
+        if (t[r] < 0 || t[r] >= kv_len) return HS2O_EINVAL;
+    const int G = h_q / h_kv;
+    int err = HS2O_OK;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 1)
+#endif
+    for (int64_t w = 0; w < n_rows * h_kv; ++w) {
+        const int64_t r = w / h_kv;
+        const int g = (int)(w % h_kv);
+        const int64_t tr = t[r];
+        const int64_t w0 = tr - window + 1 > 0 ? tr - window + 1 : 0;
+        const int64_t cap = (topk > window ? topk : window) + 1;
+        int64_t* wset = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
+        int64_t* sset = (int64_t*)malloc(sizeof(int64_t) * (size_t)cap);
+        double* s = (double*)malloc(sizeof(double) * (size_t)cap);
+        if (!wset || !sset || !s) {
+            free(wset); free(sset); free(s);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = HS2O_ENOMEM;
+            continue;
+        }
+        int64_t nw = 0, ns = 0;
+        for (int64_t j = w0; j <= tr; ++j) wset[nw++] = j;
+        int bad = 0;
+        const int32_t* ir = idx + (r * h_kv + g) * (int64_t)topk;
+        for (int i = 0; i < topk && !bad; ++i) {
+            const int64_t j = ir[i];
+            if (j == -1) continue;
+            if (j < 0 || j > tr - window) bad = 1;
+            for (int64_t u = 0; u < ns && !bad; ++u)
+                if (sset[u] == j) bad = 1;
+            if (!bad) sset[ns++] = j;
+        }
+        if (bad) {
+            free(wset); free(sset); free(s);
+#ifdef _OPENMP
+#pragma omp atomic write
+#endif
+            err = HS2O_EIDX;
+            continue;
+        }
+        const int64_t off = (int64_t)g * kv_len * d;
+        for (int hh = 0; hh < G; ++hh) {
+            const int h = g * G + hh;
+            const uint16_t* qh = q + (r * h_q + h) * (int64_t)d;
+            double qd[512];
+            for (int e = 0; e < d; ++e) qd[e] = bf16_to_double(qh[e]);
+            const int64_t o = (r * h_q + h) * (int64_t)d;
+            attend_rows(qd, k_swa + off, v_swa + off, wset, nw, d, scale, s, out_swa + o, lse_swa + r * h_q + h);
+            attend_rows(qd, k + off, v + off, sset, ns, d, scale, s, out_sel + o, lse_sel + r * h_q + h);
+        }
+        free(wset);
+        free(sset);
         free(s);
     }
     return err;

@@ -32,6 +32,11 @@ MUTATIONS = {
     "sparse_window_short": ("const int64_t w0 = tr - window + 1 > 0 ? tr - window + 1 : 0;",
                             "const int64_t w0 = tr - window + 2 > 0 ? tr - window + 2 : 0;", 0),
     "sparse_wrong_group": ("const int h = g * G + hh;", "const int h = hh * h_kv + g;", 2),
+    "branch_window_on_shared_cache": ("attend_rows(qd, k_swa + off, v_swa + off, wset",
+                                      "attend_rows(qd, k + off, v_swa + off, wset", 0),
+    "branch_selected_attends_the_window": ("attend_rows(qd, k + off, v + off, sset, ns,",
+                                           "attend_rows(qd, k + off, v + off, wset, nw,", 0),
+    "branch_lse_without_max": ("    *lse = m + log(z);", "    *lse = log(z);", 0),
     "block_partial_window": ("const int64_t n_blk = n_cand / blk;", "const int64_t n_blk = (n_cand + blk - 1) / blk;", 0),
     "block_max_not_sum": ("for (int64_t u = 0; u < blk; ++u) acc += row[bb * blk + u];",
                           "for (int64_t u = 0; u < blk; ++u) acc = fmax(acc, row[bb * blk + u]);", 0),
@@ -68,6 +73,11 @@ FAST_PINS = [
     pins.test_bridge_feature_layout_by_permuted_one_hot_rows,
     pins.test_bridge_one_hot_hidden_returns_a_weight_column,
     pins.test_bridge_decimal_brute_force,
+    pins.test_branches_merged_by_lse_are_the_union_layer,
+    pins.test_window_branch_is_sliding_window_attention_of_its_own_cache,
+    pins.test_selected_branch_single_key_closed_form,
+    pins.test_selected_branch_without_keys_is_empty,
+    pins.test_each_branch_reads_only_its_own_cache,
 ]
 
 

@@ -540,3 +540,86 @@ def test_block_scores_sum_the_token_scores():
             rest = np.setdiff1d(np.arange(n_blk), order)
             if rest.size:
                 assert got["next_block"][r, g] == pytest.approx(bs[rest].max(), rel=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# The predecessor design's two-branch sparse layer (the "Token级选择" section of
+# the xiawanshe.com report: HySparse2 drops the separate sliding-window branch):
+# a window branch over its own cache and a selected-tokens branch over the
+# shared one, each with its own softmax.
+
+
+def _branch_inputs(seed, n_rows=6, h_q=4, h_kv=2, n=300, d=16, W=24, K=40):
+    rng = np.random.default_rng(seed)
+    ts = np.array([0, 5, W - 1, W, W + 7, n - 1])[:n_rows]
+    q, k, v = rand_qkv(rng, len(ts), h_q, h_kv, n, d, scale=1.0)
+    _, k2, v2 = rand_qkv(rng, 1, h_q, h_kv, n, d, scale=1.0)
+    idx = oracle.full_select(q, ts, k, v, window=W, topk=K)["idx"]
+    return ts, q, k, v, k2, v2, idx, W
+
+
+def test_branches_merged_by_lse_are_the_union_layer():
+    """Softmaxes over two disjoint sets, merged by their log-sum-exp, are the
+    softmax over the union: with the window branch on the shared cache the merge
+    is the HySparse2 sparse layer (idx U window) exactly."""
+    ts, q, k, v, _, _, idx, W = _branch_inputs(41)
+    br = oracle.branches(q, ts, k, v, k, v, idx, window=W)
+    union = oracle.sparse(q, ts, k, v, idx, window=W)
+    lse = np.logaddexp(br["lse_swa"], br["lse_sel"])
+    a = np.exp(br["lse_swa"] - lse)[..., None]
+    b = np.exp(br["lse_sel"] - lse)[..., None]
+    np.testing.assert_allclose(a * br["out_swa"] + b * br["out_sel"], union, atol=1e-12)
+
+
+def test_window_branch_is_sliding_window_attention_of_its_own_cache():
+    """The window branch against scipy's softmax over the window rows of k_swa."""
+    ts, q, k, v, k2, v2, idx, W = _branch_inputs(42)
+    br = oracle.branches(q, ts, k2, v2, k, v, idx, window=W)
+    qf, kf, vf = unbits(q), unbits(k2), unbits(v2)
+    d = q.shape[2]
+    for r, t in enumerate(ts):
+        lo = max(0, t - W + 1)
+        for h in range(q.shape[1]):
+            g = h // (q.shape[1] // k.shape[0])
+            s = kf[g, lo:t + 1] @ qf[r, h] / math.sqrt(d)
+            np.testing.assert_allclose(br["out_swa"][r, h], scipy.special.softmax(s) @ vf[g, lo:t + 1], atol=1e-12)
+            assert br["lse_swa"][r, h] == pytest.approx(scipy.special.logsumexp(s), abs=1e-12)
+
+
+def test_selected_branch_single_key_closed_form():
+    """One selected key j: the branch output is v_j and its LSE is the logit s_j."""
+    rng = np.random.default_rng(43)
+    h_q, h_kv, d, n, W = 4, 2, 16, 100, 8
+    q, k, v = rand_qkv(rng, 1, h_q, h_kv, n, d, scale=1.0)
+    t = np.array([60])
+    idx = np.full((1, h_kv, 3), -1, np.int32)
+    idx[0, 0, 0], idx[0, 1, 0] = 17, 40
+    br = oracle.branches(q, t, k, v, k, v, idx, window=W)
+    qf, kf, vf = unbits(q), unbits(k), unbits(v)
+    for h in range(h_q):
+        g = h // (h_q // h_kv)
+        j = idx[0, g, 0]
+        np.testing.assert_array_equal(br["out_sel"][0, h], vf[g, j])
+        assert br["lse_sel"][0, h] == pytest.approx(kf[g, j] @ qf[0, h] / math.sqrt(d), abs=1e-12)
+
+
+def test_selected_branch_without_keys_is_empty():
+    """Rows with no selected key (t < W, or an all -1 row): zero output, LSE -inf;
+    the window branch is unaffected."""
+    ts, q, k, v, k2, v2, idx, W = _branch_inputs(44)
+    idx[:] = -1
+    br = oracle.branches(q, ts, k2, v2, k, v, idx, window=W)
+    assert np.all(br["out_sel"] == 0.0) and np.all(np.isneginf(br["lse_sel"]))
+    assert np.all(np.isfinite(br["lse_swa"]))
+
+
+def test_each_branch_reads_only_its_own_cache():
+    """Changing the shared cache leaves the window branch unchanged, and changing
+    the window branch's cache leaves the selected branch unchanged."""
+    ts, q, k, v, k2, v2, idx, W = _branch_inputs(45)
+    a = oracle.branches(q, ts, k2, v2, k, v, idx, window=W)
+    b = oracle.branches(q, ts, k2, v2, v, k, idx, window=W)  # another shared cache
+    c = oracle.branches(q, ts, v2, k2, k, v, idx, window=W)  # another window cache
+    np.testing.assert_array_equal(a["out_swa"], b["out_swa"])
+    np.testing.assert_array_equal(a["out_sel"], c["out_sel"])
+    assert not np.allclose(a["out_sel"], b["out_sel"]) and not np.allclose(a["out_swa"], c["out_swa"])
