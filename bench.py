@@ -213,6 +213,53 @@ def bench_block_select(w: wl.Workload, inp: dict, dev, K: int, warmup: int, pk: 
     return res
 
 
+def bench_swa_comparator(w: wl.Workload, inp: dict, dev, K: int, warmup: int, flush: torch.Tensor,
+                         idx: torch.Tensor) -> dict:
+    """One sparse layer three ways on the workload's inputs (a next row of the
+    path: the cost comparison the pages make against the predecessor designs),
+    each call timed alone with CUDA events, L2 flushed before every call:
+      hysparse2   one softmax over idx U window, all from the shared cache
+                  (hs2_sparse_attn, the layer of the timed step);
+      two_branch  the predecessor's sparse layer: a sliding-window branch over
+                  its own cache plus the selected rows alone (hs2_swa_branches);
+      swa_only    a plain sliding-window layer over its own cache (the SWA layers
+                  of a hybrid full/SWA model: hs2_sparse_attn with top-k 0)."""
+    swa = wl.make_swa_cache(w, dev, seed=w.seed)
+    q = inp["q_sparse"][0] if inp["q_sparse"] else inp["q"]
+    q_pos0 = (w.kv_len - 1) if w.decode else w.q_pos0
+    shape = nv.shape_of(q, inp["k"], window=w.window, topk=w.topk, q_pos0=q_pos0)
+    shape0 = nv.shape_of(q, inp["k"], window=w.window, topk=0, q_pos0=q_pos0)
+    B, Hq, nq, D = q.shape
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    l1 = torch.empty(B, Hq, nq, dtype=torch.float32, device=dev)
+    l2 = torch.empty_like(l1)
+    calls = {
+        "hysparse2": lambda: nv.hs2_sparse_attn(shape, q, inp["k"], inp["v"], idx, o1, None),
+        "two_branch": lambda: nv.hs2_swa_branches(shape, q, swa["k_swa"], swa["v_swa"], inp["k"], inp["v"], idx,
+                                                  o1, l1, o2, l2),
+        "swa_only": lambda: nv.hs2_sparse_attn(shape0, q, swa["k_swa"], swa["v_swa"], None, o1, None),
+    }
+    st = torch.cuda.current_stream()
+    ms = {}
+    for name, fn in calls.items():
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(st)
+            fn()
+            e1.record(st)
+        torch.cuda.synchronize()
+        ms[name] = round(statistics.median(e0.elapsed_time(e1) for e0, e1 in ev), 4)
+    del swa
+    return {"ms_per_layer": ms, "two_branch_over_hysparse2": round(ms["two_branch"] / ms["hysparse2"], 3),
+            "kv_caches_per_layer": {"hysparse2": 1, "two_branch": 2, "swa_only": 1},
+            "note": "same q, idx and shared cache; the window branch's own cache is a seeded N(0,1)*0.5 draw "
+                    "of the same shape; L2 flushed before each call"}
+
+
 def source_sha(path: str) -> str:
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
@@ -567,6 +614,7 @@ def run_ours(args):
     blk = bench_block_select(w, inp, dev, args.steps, args.warmup, pk, flush, token_sel_ms)
     if blk is not None:
         next_rows["block_select"] = blk
+    next_rows["swa_comparator"] = bench_swa_comparator(w, inp, dev, args.steps, args.warmup, flush, step.idx)
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
 

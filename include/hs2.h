@@ -141,6 +141,29 @@ hs2_status hs2_full_attn_block_select(const hs2_shape* shape, int32_t block, con
                                       const void* v, void* out, float* lse, int32_t* idx, void* ws,
                                       size_t ws_bytes, hs2_stream_t stream);
 
+/* The two attention branches of a sparse layer in the predecessor design, as
+ * a cost comparator for hs2_sparse_attn (xiawanshe.com report, section
+ * "Token级选择": HySparse2 drops the Cross-Decoder's separate sliding-window
+ * branch and keeps the most recent tokens in the one shared cache instead).
+ * Per query t and head h (g = h / G), with the layer's own query q:
+ *   window branch:   out_swa, lse_swa = softmax attention over window(t) of the
+ *                    branch's OWN cache k_swa, v_swa ([batch, h_kv, kv_len,
+ *                    head_dim] bf16, laid out like k, v);
+ *   selected branch: out_sel, lse_sel = softmax attention over the selected
+ *                    rows idx_g(t) ALONE (no window) of the shared cache k, v;
+ *                    a row with no selected key gets out_sel = 0 and
+ *                    lse_sel = -inf.
+ * out_* [batch, h_q, n_q, head_dim] bf16; lse_* [batch, h_q, n_q] fp32,
+ * natural log.  The pages do not say how the predecessor combined the two
+ * outputs, so both are returned; merging them by their LSEs gives the softmax
+ * over idx U window.  idx rows as hs2_sparse_attn takes them (topk = 0 makes
+ * the selected branch empty).  ws may be NULL with ws_bytes == 0; with a
+ * workspace, the checked build reports invalid idx rows through its error
+ * word.  Two kernel launches (kernel id 4 each). */
+hs2_status hs2_swa_branches(const hs2_shape* shape, const void* q, const void* k_swa, const void* v_swa,
+                            const void* k, const void* v, const int32_t* idx, void* out_swa, float* lse_swa,
+                            void* out_sel, float* lse_sel, void* ws, size_t ws_bytes, hs2_stream_t stream);
+
 /* Prefill-chunk entry: the full-attention + selection layer for a chunk of
  * n_q new tokens appended to a cache of kv_len tokens (q_pos0 = kv_len - n_q
  * for an append; any q_pos0 with q_pos0 + n_q <= kv_len is accepted).  Same

@@ -381,6 +381,36 @@ hs2_status hs2_decode_sparse(const hs2_shape* shape, const int64_t* kv_len_per_s
     return run_sparse(&s, kv_len_per_seq, q, k, v, idx, out, ws, ws_bytes, stream);
 }
 
+hs2_status hs2_swa_branches(const hs2_shape* shape, const void* q, const void* k_swa, const void* v_swa,
+                            const void* k, const void* v, const int32_t* idx, void* out_swa, float* lse_swa,
+                            void* out_sel, float* lse_sel, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k_swa || !v_swa || !k || !v || !out_swa || !lse_swa || !out_sel || !lse_sel ||
+        (p.topk > 0 && !idx))
+        return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_swa, 16) || !aligned(v_swa, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(idx, 4) || !aligned(out_swa, 16) || !aligned(out_sel, 16) || !aligned(lse_swa, 4) ||
+        !aligned(lse_sel, 4))
+        return HS2_ERR_INVALID_ARG;
+    if (ws != nullptr) {
+        if (ws_bytes < kHeader || !aligned(ws, 256)) return HS2_ERR_WORKSPACE;
+        p.err = reinterpret_cast<WsHeader*>(ws);
+    } else if (ws_bytes != 0) {
+        return HS2_ERR_INVALID_ARG;
+    }
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    // selected branch: the selected rows of the shared cache alone
+    cudaError_t e = launch_sparse(p, q, k, v, idx, out_sel, st, 0, lse_sel);
+    if (e != cudaSuccess) return HS2_ERR_CUDA;
+    // window branch: the same kernel with no selection, over the branch's own cache
+    Problem pw = p;
+    pw.topk = 0;
+    return cuda_status(launch_sparse(pw, q, k_swa, v_swa, nullptr, out_swa, st, 1, lse_swa));
+}
+
 hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info) {
     if (ws == nullptr || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

@@ -76,8 +76,11 @@ cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const 
                           void* scratch, float* scores, int64_t sstride, cudaStream_t st);
 
 // K3: one sparse KV-reuse layer.
+// with_window = 0 attends to the selected rows alone; lse (nullable) receives
+// the natural-log LSE of the attended logits per (sequence, head, query).
 cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v,
-                          const int32_t* idx, void* out, cudaStream_t st);
+                          const int32_t* idx, void* out, cudaStream_t st, int with_window = 1,
+                          float* lse = nullptr);
 
 // Query position of query 0 of sequence b: q_pos0, or seq_len[b] - nq for decode
 // (clamped into [0, kv_len - nq]; a clamp is reported through the error word).

@@ -46,7 +46,8 @@ __global__ void __launch_bounds__(W * 32) k3_sparse_kernel(Problem p, const __nv
                                                                    const __nv_bfloat16* __restrict__ k,
                                                                    const __nv_bfloat16* __restrict__ v,
                                                                    const int32_t* __restrict__ idx,
-                                                                   __nv_bfloat16* __restrict__ out) {
+                                                                   __nv_bfloat16* __restrict__ out,
+                                                                   int with_window, float* __restrict__ lse) {
     using C = K3Cfg<D, W>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -54,7 +55,7 @@ __global__ void __launch_bounds__(W * 32) k3_sparse_kernel(Problem p, const __nv
     const int64_t pos0 = seq_pos0(p, b, KID_SPARSE);
     const int64_t t = pos0 + i;
     const int64_t w0 = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
-    const int nwin = (int)(t - w0 + 1);
+    const int nwin = with_window ? (int)(t - w0 + 1) : 0;  // 0: the selected rows alone
 
     // attended rows: the selection's valid prefix (its length counted here),
     // then the window
@@ -248,20 +249,25 @@ __global__ void __launch_bounds__(W * 32) k3_sparse_kernel(Problem p, const __nv
 #pragma unroll
         for (int w = 0; w < W; ++w) mm = fmaxf(mm, comb[w * (D * 8 + 16) + D * 8 + hh]);
         float num = 0.f, den = 0.f;
+        if (mm != -INFINITY) {  // else no attended row at all (the selected rows alone, none valid)
 #pragma unroll
-        for (int w = 0; w < W; ++w) {
-            const float* wb = comb + w * (D * 8 + 16);
-            const float sc = ex2(wb[D * 8 + hh] - mm);
-            num += sc * wb[d * 8 + hh];
-            den += sc * wb[D * 8 + 8 + hh];
+            for (int w = 0; w < W; ++w) {
+                const float* wb = comb + w * (D * 8 + 16);
+                const float sc = ex2(wb[D * 8 + hh] - mm);
+                num += sc * wb[d * 8 + hh];
+                den += sc * wb[D * 8 + 8 + hh];
+            }
         }
-        out[((int64_t)(b * p.hq + g * G + hh) * p.nq + i) * D + d] = __float2bfloat16_rn(num / den);
+        const int64_t oh = (int64_t)(b * p.hq + g * G + hh) * p.nq + i;
+        out[oh * D + d] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
+        // natural-log LSE of the attended logits: (m + log2 l) ln 2 in the kernel's log2 units
+        if (lse != nullptr && d == 0) lse[oh] = den > 0.f ? (mm + __log2f(den)) * kLn2 : -INFINITY;
     }
 }
 
 template <int D, int G, int W>
 cudaError_t launch_sparse_dgw(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
-                              void* out, cudaStream_t st) {
+                              void* out, int with_window, float* lse, cudaStream_t st) {
     using C = K3Cfg<D, W>;
     const int smem = C::FIXED;
     auto kern = k3_sparse_kernel<D, G, W>;
@@ -270,7 +276,7 @@ cudaError_t launch_sparse_dgw(const Problem& p, const void* q, const void* k, co
     dim3 grid(p.nq, p.hkv, p.B);
     prof_begin(KID_SPARSE, st);
     kern<<<grid, W * 32, smem, st>>>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k, (const __nv_bfloat16*)v,
-                                     idx, (__nv_bfloat16*)out);
+                                     idx, (__nv_bfloat16*)out, with_window, lse);
     prof_end(st);
     count_launch();
     return cudaGetLastError();
@@ -278,29 +284,29 @@ cudaError_t launch_sparse_dgw(const Problem& p, const void* q, const void* k, co
 
 template <int D, int G>
 cudaError_t launch_sparse_dg(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
-                             void* out, cudaStream_t st) {
+                             void* out, int with_window, float* lse, cudaStream_t st) {
     const int64_t ctas = (int64_t)p.nq * p.hkv * p.B;
-    if (ctas < SP_SMALL_GRID) return launch_sparse_dgw<D, G, 4>(p, q, k, v, idx, out, st);
-    return launch_sparse_dgw<D, G, 1>(p, q, k, v, idx, out, st);
+    if (ctas < SP_SMALL_GRID) return launch_sparse_dgw<D, G, 4>(p, q, k, v, idx, out, with_window, lse, st);
+    return launch_sparse_dgw<D, G, 1>(p, q, k, v, idx, out, with_window, lse, st);
 }
 
 template <int D>
 cudaError_t launch_sparse_d(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
-                            void* out, cudaStream_t st) {
+                            void* out, int with_window, float* lse, cudaStream_t st) {
     switch (p.hq / p.hkv) {
-        case 1: return launch_sparse_dg<D, 1>(p, q, k, v, idx, out, st);
-        case 2: return launch_sparse_dg<D, 2>(p, q, k, v, idx, out, st);
-        case 4: return launch_sparse_dg<D, 4>(p, q, k, v, idx, out, st);
-        default: return launch_sparse_dg<D, 8>(p, q, k, v, idx, out, st);
+        case 1: return launch_sparse_dg<D, 1>(p, q, k, v, idx, out, with_window, lse, st);
+        case 2: return launch_sparse_dg<D, 2>(p, q, k, v, idx, out, with_window, lse, st);
+        case 4: return launch_sparse_dg<D, 4>(p, q, k, v, idx, out, with_window, lse, st);
+        default: return launch_sparse_dg<D, 8>(p, q, k, v, idx, out, with_window, lse, st);
     }
 }
 
 }  // namespace
 
 cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v, const int32_t* idx,
-                          void* out, cudaStream_t st) {
-    if (p.D == 64) return launch_sparse_d<64>(p, q, k, v, idx, out, st);
-    return launch_sparse_d<128>(p, q, k, v, idx, out, st);
+                          void* out, cudaStream_t st, int with_window, float* lse) {
+    if (p.D == 64) return launch_sparse_d<64>(p, q, k, v, idx, out, with_window, lse, st);
+    return launch_sparse_d<128>(p, q, k, v, idx, out, with_window, lse, st);
 }
 
 }  // namespace hs2

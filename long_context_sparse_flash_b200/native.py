@@ -28,7 +28,8 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_prefill_chunk", "hs2_decode", "hs2_decode_sparse", "hs2_get_device_status", "hs2_status_string",
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
-           "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select")
+           "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
+           "hs2_swa_branches")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
@@ -78,6 +79,7 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_full_attn_select.argtypes = [sh, P, P, P, P, P, P, P, S, P]
     lib.hs2_prefill_chunk.argtypes = [sh, P, P, P, P, P, P, P, S, P]
     lib.hs2_full_attn_block_select.argtypes = [sh, ctypes.c_int32, P, P, P, P, P, P, P, S, P]
+    lib.hs2_swa_branches.argtypes = [sh, P, P, P, P, P, P, P, P, P, P, P, S, P]
     lib.hs2_decode.argtypes = [sh, P, P, P, P, P, P, P, P, S, P]
     lib.hs2_sparse_attn.argtypes = [sh, P, P, P, P, P, P, S, P]
     lib.hs2_decode_sparse.argtypes = [sh, P, P, P, P, P, P, P, S, P]
@@ -99,7 +101,8 @@ def load(checked: bool = False) -> ctypes.CDLL:
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
-                 "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select"):
+                 "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
+                 "hs2_swa_branches"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -176,6 +179,15 @@ def hs2_full_attn_block_select(shape, block, q, k, v, out, lse, idx, ws, stream=
     _check(load(checked).hs2_full_attn_block_select(ctypes.byref(shape), int(block), _ptr(q), _ptr(k), _ptr(v),
                                                     _ptr(out), _ptr(lse), _ptr(idx), wp, wn, _stream(stream)),
            "hs2_full_attn_block_select")
+
+
+def hs2_swa_branches(shape, q, k_swa, v_swa, k, v, idx, out_swa, lse_swa, out_sel, lse_sel, ws=None, stream=None,
+                     checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_swa_branches(ctypes.byref(shape), _ptr(q), _ptr(k_swa), _ptr(v_swa), _ptr(k), _ptr(v),
+                                          _ptr(idx), _ptr(out_swa), _ptr(lse_swa), _ptr(out_sel), _ptr(lse_sel),
+                                          wp, wn, _stream(stream)),
+           "hs2_swa_branches")
 
 
 def hs2_prefill_chunk(shape, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
@@ -322,6 +334,18 @@ def full_attn_block_select(q, k, v, *, window: int, topk: int, block: int, q_pos
     idx = torch.empty(B, k.shape[1], nq, topk, dtype=torch.int32, device=q.device)
     hs2_full_attn_block_select(shape, block, q, k, v, out, lse, idx, ws, stream, checked)
     return out, lse, idx
+
+
+def swa_branches(q, k_swa, v_swa, k, v, idx, *, window: int, q_pos0: int = 0, stream=None, ws=None,
+                 checked: bool = False):
+    """The predecessor design's two branches: returns (out_swa, lse_swa, out_sel, lse_sel)."""
+    shape = shape_of(q, k, window=window, topk=idx.shape[-1], q_pos0=q_pos0)
+    B, Hq, nq, D = q.shape
+    out_swa, out_sel = torch.empty_like(q), torch.empty_like(q)
+    lse_swa = torch.empty(B, Hq, nq, dtype=torch.float32, device=q.device)
+    lse_sel = torch.empty_like(lse_swa)
+    hs2_swa_branches(shape, q, k_swa, v_swa, k, v, idx, out_swa, lse_swa, out_sel, lse_sel, ws, stream, checked)
+    return out_swa, lse_swa, out_sel, lse_sel
 
 
 def decode(q, k, v, *, window: int, topk: int, kv_len_per_seq=None, ws=None, stream=None,

@@ -74,6 +74,7 @@ WORKLOADS: Dict[str, Workload] = {
 # sub-seed offsets, one per drawn tensor: seed * 1000 + offset
 SUB_Q, SUB_K, SUB_V, SUB_QS, SUB_NEEDLE, SUB_SEG = 1, 2, 3, 10, 50, 60
 SUB_HIDDEN, SUB_WKV = 70, 71
+SUB_KSWA, SUB_VSWA = 80, 81  # the sliding-window branch's own cache (comparator)
 # hidden size of the Self-Decoder for the KV-bridging inputs (the pages give no
 # model dimensions; a common size for a model of this class)
 BRIDGE_D_MODEL = 4096
@@ -208,6 +209,19 @@ def make_bridge_inputs(batch: int, n_new: int, d_model: int, h_kv: int, head_dim
     hidden = torch.randn(batch, n_new, d_model, generator=gh, device=device).to(torch.bfloat16)
     w = (torch.randn(2 * h_kv * head_dim, d_model, generator=gw, device=device) / math.sqrt(d_model)).to(torch.bfloat16)
     return dict(hidden=hidden, w_kv=w)
+
+
+def make_swa_cache(w: Workload, device="cpu", seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """The own K/V cache of a separate sliding-window branch (the predecessor
+    design's sparse layer), shaped like the shared cache: k_swa, v_swa bf16
+    [B, H_kv, kv_len, D] ~ N(0,1) * 0.5."""
+    seed = w.seed if seed is None else int(seed)
+    shape = (w.batch, w.h_kv, w.kv_len, w.head_dim)
+    gk = _gen(device, seed * 1000 + SUB_KSWA)
+    gv = _gen(device, seed * 1000 + SUB_VSWA)
+    k = (torch.randn(*shape, generator=gk, device=device) * 0.5).to(torch.bfloat16)
+    v = (torch.randn(*shape, generator=gv, device=device) * 0.5).to(torch.bfloat16)
+    return dict(k_swa=k, v_swa=v)
 
 
 def bf16_bits(t: torch.Tensor) -> np.ndarray:

@@ -214,3 +214,30 @@ def test_block_select_validation_without_launch():
     # no candidate at all: the header only (plus the full layer's own split scratch, none here)
     assert nv.hs2_workspace_size(shape(n_q=100, kv_len=100), nv.HS2_ENTRY_BLOCK_SELECT) == 256
     assert nv.hs2_launch_count() == before
+
+
+def test_swa_branches_validation_without_launch():
+    """The two-branch comparator entry: shape, pointers, alignment, workspace, empty calls."""
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    s = shape(n_q=512, kv_len=4096, q_pos0=3584)
+    ptrs = [FAKE] * 10  # q, k_swa, v_swa, k, v, idx, out_swa, lse_swa, out_sel, lse_sel
+
+    def call(sh, *a, ws=None, ws_bytes=0):
+        return L.hs2_swa_branches(ctypes.byref(sh) if sh is not None else None, *a, ws, ws_bytes, None)
+
+    assert call(None, *ptrs) == 1
+    assert call(shape(h_q=30), *ptrs) == 1
+    assert call(shape(head_dim=96), *ptrs) == 2
+    for i in range(10):
+        bad = list(ptrs)
+        bad[i] = None
+        assert call(s, *bad) == 1, i
+    mis = list(ptrs)
+    mis[1] = ctypes.c_void_p((1 << 40) + 8)  # k_swa not 16-byte aligned
+    assert call(s, *mis) == 1
+    assert call(s, *ptrs, ws=FAKE, ws_bytes=100) == 3
+    assert call(s, *ptrs, ws=None, ws_bytes=256) == 1
+    for kw in (dict(batch=0), dict(n_q=0)):
+        assert call(shape(**kw), *([None] * 10)) == 0
+    assert nv.hs2_launch_count() == before
