@@ -89,7 +89,10 @@ enum {
     HS2_ENTRY_SPARSE = 1,
     HS2_ENTRY_PREFILL = 2,
     HS2_ENTRY_DECODE = 3,
-    HS2_ENTRY_BLOCK_SELECT = 4
+    HS2_ENTRY_BLOCK_SELECT = 4,
+    HS2_ENTRY_CP_ATTN = 5,     /* slice calls: sized by hs2_cp_workspace_size */
+    HS2_ENTRY_CP_SELECT = 6,
+    HS2_ENTRY_CP_SPARSE = 7
 };
 
 /* Bytes of workspace the entry point `entry` needs for `shape` (0 if the shape
@@ -163,6 +166,73 @@ hs2_status hs2_full_attn_block_select(const hs2_shape* shape, int32_t block, con
 hs2_status hs2_swa_branches(const hs2_shape* shape, const void* q, const void* k_swa, const void* v_swa,
                             const void* k, const void* v, const int32_t* idx, void* out_swa, float* lse_swa,
                             void* out_sel, float* lse_sel, void* ws, size_t ws_bytes, hs2_stream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * Context parallelism: the KV cache of one long context is cut into P
+ * contiguous slices, slice p holding keys [kv_off_p, kv_off_p + len_p) on its
+ * own GPU (offsets ascending, slices adjacent).  The layers of the pages
+ * (xiawanshe.com report, sections "两级KV共享" and "Token级选择") are computed
+ * exactly, with one exchange of per-slice results after each step:
+ *   1. hs2_cp_attn_partial on every slice -> out_p, lse_p (attention over the
+ *      slice's causal keys); exchange; hs2_cp_combine -> out, lse.
+ *   2. hs2_cp_select_local on every slice with the combined lse -> the slice's
+ *      top-K candidates and their scores; exchange; hs2_cp_select_merge -> idx
+ *      (the same rows hs2_full_attn_select selects from the whole cache).
+ *   3. per sparse layer: hs2_cp_sparse_partial on every slice -> out_p, lse_p
+ *      (the layer over the rows of idx U window the slice holds); exchange;
+ *      hs2_cp_combine -> out.
+ * The exchange itself (an all-gather of the per-slice buffers, stacked along
+ * a new leading axis in slice order) is the caller's; the library only
+ * computes.  Slice calls take a `shape` describing the slice: kv_len = len_p
+ * rows (the row stride of k, v), q_pos0 = the ABSOLUTE position of query 0
+ * (any q_pos0 >= 0: a query may sit before the slice -- it has no key there,
+ * out_p = 0 and lse_p = -inf -- or after it -- every key of the slice is
+ * causal for it); n_q >= 64 (HS2_ERR_UNSUPPORTED below).  Candidates are still
+ * the keys j <= t - window in absolute positions.  Slice calls need a
+ * workspace of hs2_cp_workspace_size(shape, kv_off, entry) bytes. */
+
+/* Bytes of workspace a slice call needs (0 if the shape or entry is invalid). */
+size_t hs2_cp_workspace_size(const hs2_shape* shape, int64_t kv_off, int entry);
+
+/* Step 1 on one slice: out [batch, h_q, n_q, head_dim] bf16 and lse [batch,
+ * h_q, n_q] fp32 (natural log) of the attention over the slice's keys
+ * j <= t.  Entry HS2_ENTRY_CP_ATTN. */
+hs2_status hs2_cp_attn_partial(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k, const void* v,
+                               void* out, float* lse, void* ws, size_t ws_bytes, hs2_stream_t stream);
+
+/* Step 2 on one slice: with lse the COMBINED (whole-context) LSE, the slice's
+ * top-min(topk, its candidates) keys by (score desc, j asc): idx [batch,
+ * h_kv, n_q, topk] int32 as LOCAL rows of the slice (ascending, -1 padded) and
+ * score [batch, h_kv, n_q, topk] fp32 (the group-summed probability, -1 for
+ * padding).  Entry HS2_ENTRY_CP_SELECT. */
+hs2_status hs2_cp_select_local(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k,
+                               const float* lse, int32_t* idx, float* score, void* ws, size_t ws_bytes,
+                               hs2_stream_t stream);
+
+/* Step 3 on one slice: one sparse layer (q its own query) over the rows of
+ * idx U window(t) that the slice holds; idx is the whole-context selection
+ * (absolute rows, as hs2_cp_select_merge writes it).  out bf16, lse fp32
+ * (natural log; -inf and out = 0 for a query with no such row in the slice).
+ * Entry HS2_ENTRY_CP_SPARSE. */
+hs2_status hs2_cp_sparse_partial(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes,
+                                 hs2_stream_t stream);
+
+/* The merge of steps 1 and 3: out_parts [n_parts][n_rows][head_dim] bf16 and
+ * lse_parts [n_parts][n_rows] fp32 (n_rows = batch * h_q * n_q) -> out, lse:
+ * lse = ln sum_p e^(lse_p), out = sum_p e^(lse_p - lse) out_p; a row whose parts
+ * are all -inf gets 0 and -inf.  Device buffers; stream-ordered. */
+hs2_status hs2_cp_combine(int32_t n_parts, int64_t n_rows, int32_t head_dim, const void* out_parts,
+                          const float* lse_parts, void* out, float* lse, hs2_stream_t stream);
+
+/* The merge of step 2: shape is the WHOLE context's (kv_len = total keys, the
+ * usual q_pos0 rule); kv_offs is a HOST array of the n_parts slices' first keys
+ * (strictly ascending; n_parts <= 16); idx_parts / score_parts stack the
+ * slices' hs2_cp_select_local outputs in slice order.  Writes idx [batch, h_kv,
+ * n_q, topk]: the whole-context selection, absolute rows ascending, -1 padded. */
+hs2_status hs2_cp_select_merge(const hs2_shape* shape, int32_t n_parts, const int64_t* kv_offs,
+                               const int32_t* idx_parts, const float* score_parts, int32_t* idx,
+                               hs2_stream_t stream);
 
 /* Prefill-chunk entry: the full-attention + selection layer for a chunk of
  * n_q new tokens appended to a cache of kv_len tokens (q_pos0 = kv_len - n_q
@@ -245,7 +315,9 @@ uint64_t hs2_launch_count(void);
  * 2 selection scores, 3 top-k select, 4 sparse attention, 5 decode attention
  * partials, 6 decode combine, 7 fused attention + selection, 8 selection
  * threshold estimate, 9 filtered selection sweep, 10 selection retry,
- * 11 KV bridging, 12 block-selection score sweep, 13 block top-k. */
+ * 11 KV bridging, 12 block-selection score sweep, 13 block top-k,
+ * 14 context-parallel combine, 15 context-parallel selection merge,
+ * 16 context-parallel selection slicing. */
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 

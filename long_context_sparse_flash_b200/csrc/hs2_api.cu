@@ -262,6 +262,63 @@ hs2_status run_block_select(const hs2_shape* shape, int blk, const void* q, cons
     return HS2_OK;
 }
 
+// Context parallelism: a call over one slice of the context's KV cache.  The
+// shape describes the slice (kv_len = its rows, q_pos0 = the absolute position
+// of query 0) and kv_off is the absolute position of the slice's first key; a
+// query may sit before the slice (no key there) or after it (all its keys).
+// The kernels see positions shifted by -kv_off.  Prefill-shaped calls only
+// (n_q >= 64, the tensor-core paths).
+hs2_status check_slice(const hs2_shape* shape, int64_t kv_off, Problem* p) {
+    if (shape == nullptr || kv_off < 0) return HS2_ERR_INVALID_ARG;
+    if (shape->kv_len < 1 || shape->q_pos0 < 0) return HS2_ERR_INVALID_ARG;
+    hs2_shape s = *shape;
+    s.q_pos0 = 0;  // the slice rule replaces q_pos0 + n_q <= kv_len
+    if (s.kv_len < s.n_q) s.kv_len = s.n_q;
+    const hs2_status st = check_shape(&s, p);
+    if (st != HS2_OK) return st;
+    if (shape->n_q > 0 && shape->n_q < 64) return HS2_ERR_UNSUPPORTED;
+    if (shape->q_pos0 + (int64_t)shape->n_q > (int64_t)INT32_MAX + 1) return HS2_ERR_UNSUPPORTED;
+    p->kv_len = shape->kv_len;
+    p->q_pos0 = shape->q_pos0 - kv_off;
+    return HS2_OK;
+}
+
+// Selection plan of a slice: candidates of the last query inside the slice.
+// The selection runs even when no query has a candidate in the slice (it then
+// writes -1 rows and -1 scores), so the plan never has zero candidates.
+ScorePlan slice_plan(const Problem& p) {
+    ScorePlan sp;
+    if (p.nq == 0 || p.B == 0 || p.topk == 0) return sp;
+    int64_t cand = p.q_pos0 + p.nq - p.window;  // t_max - window + 1 in slice rows
+    if (cand > p.kv_len) cand = p.kv_len;
+    if (cand < 1) cand = 1;
+    sp.tc = true;
+    sp.n_cand_max = cand;
+    const size_t per_q = (size_t)p.B * p.hkv * (1024 * 4 + 12);
+    int64_t chunk = (int64_t)(kSampleBudget / per_q) / 32 * 32;
+    if (chunk < 32) chunk = 32;
+    if (chunk > p.nq) chunk = p.nq;
+    sp.chunk = (int)chunk;
+    sp.bytes = select_tc_scratch_bytes(p, sp.chunk, cand);
+    return sp;
+}
+
+size_t cp_body_bytes(const Problem& p, int entry) {
+    switch (entry) {
+        case HS2_ENTRY_CP_ATTN: return full_tc_split_scratch_bytes(p);
+        case HS2_ENTRY_CP_SELECT: return slice_plan(p).bytes;
+        case HS2_ENTRY_CP_SPARSE: return (size_t)p.B * p.hkv * p.nq * p.topk * 4;
+        default: return 0;
+    }
+}
+
+// Slice calls need a workspace: the error word, then `need` bytes of scratch.
+hs2_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
+    if (ws_bytes < kHeader + need) return HS2_ERR_WORKSPACE;
+    return HS2_OK;
+}
+
 }  // namespace
 }  // namespace hs2
 
@@ -277,6 +334,9 @@ size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
         case HS2_ENTRY_FULL_SELECT:
         case HS2_ENTRY_PREFILL: return kHeader + prefill_body_bytes(p, score_plan(p, false));
         case HS2_ENTRY_BLOCK_SELECT: return kHeader + block_body_bytes(p);
+        case HS2_ENTRY_CP_ATTN:
+        case HS2_ENTRY_CP_SELECT:
+        case HS2_ENTRY_CP_SPARSE: return 0;  // slices: hs2_cp_workspace_size
         case HS2_ENTRY_DECODE: {
             if (p.nq != 1) return 0;
             return kHeader + (score_plan(p, true).bytes + 255) / 256 * 256 + decode_scratch_bytes(p);
@@ -409,6 +469,103 @@ hs2_status hs2_swa_branches(const hs2_shape* shape, const void* q, const void* k
     Problem pw = p;
     pw.topk = 0;
     return cuda_status(launch_sparse(pw, q, k_swa, v_swa, nullptr, out_swa, st, 1, lse_swa));
+}
+
+size_t hs2_cp_workspace_size(const hs2_shape* shape, int64_t kv_off, int entry) {
+    Problem p;
+    if (check_slice(shape, kv_off, &p) != HS2_OK) return 0;
+    if (entry != HS2_ENTRY_CP_ATTN && entry != HS2_ENTRY_CP_SELECT && entry != HS2_ENTRY_CP_SPARSE) return 0;
+    return kHeader + cp_body_bytes(p, entry);
+}
+
+hs2_status hs2_cp_attn_partial(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k, const void* v,
+                               void* out, float* lse, void* ws, size_t ws_bytes, hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_slice(shape, kv_off, &p);
+    if (s != HS2_OK) return s;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k || !v || !out || !lse) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4))
+        return HS2_ERR_INVALID_ARG;
+    if ((s = check_ws(ws, ws_bytes, cp_body_bytes(p, HS2_ENTRY_CP_ATTN))) != HS2_OK) return s;
+    p.err = reinterpret_cast<WsHeader*>(ws);
+    return cuda_status(launch_full_tc(p, q, k, v, out, lse, reinterpret_cast<uint8_t*>(ws) + kHeader,
+                                      ws_bytes - kHeader, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_cp_select_local(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k,
+                               const float* lse, int32_t* idx, float* score, void* ws, size_t ws_bytes,
+                               hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_slice(shape, kv_off, &p);
+    if (s != HS2_OK) return s;
+    if (p.B == 0 || p.nq == 0 || p.topk == 0) return HS2_OK;
+    if (!q || !k || !lse || !idx || !score) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(lse, 4) || !aligned(idx, 4) || !aligned(score, 4))
+        return HS2_ERR_INVALID_ARG;
+    const ScorePlan sp = slice_plan(p);
+    if ((s = check_ws(ws, ws_bytes, sp.bytes)) != HS2_OK) return s;
+    p.err = reinterpret_cast<WsHeader*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    void* scratch = reinterpret_cast<uint8_t*>(ws) + kHeader;
+    const int chunk = sp.chunk > 0 ? sp.chunk : p.nq;
+    for (int i0 = 0; i0 < p.nq; i0 += chunk) {
+        const int cnt = p.nq - i0 < chunk ? p.nq - i0 : chunk;
+        const cudaError_t e = launch_select_tc(p, q, k, lse, idx, scratch, i0, cnt, sp.n_cand_max, st, score);
+        if (e != cudaSuccess) return HS2_ERR_CUDA;
+    }
+    return HS2_OK;
+}
+
+hs2_status hs2_cp_sparse_partial(const hs2_shape* shape, int64_t kv_off, const void* q, const void* k,
+                                 const void* v, const int32_t* idx, void* out, float* lse, void* ws, size_t ws_bytes,
+                                 hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_slice(shape, kv_off, &p);
+    if (s != HS2_OK) return s;
+    if (p.B == 0 || p.nq == 0) return HS2_OK;
+    if (!q || !k || !v || !out || !lse || (p.topk > 0 && !idx)) return HS2_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(lse, 4) ||
+        !aligned(idx, 4))
+        return HS2_ERR_INVALID_ARG;
+    if ((s = check_ws(ws, ws_bytes, cp_body_bytes(p, HS2_ENTRY_CP_SPARSE))) != HS2_OK) return s;
+    p.err = reinterpret_cast<WsHeader*>(ws);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int32_t* local = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + kHeader);
+    const int64_t rows = (int64_t)p.B * p.hkv * p.nq;
+    cudaError_t e = launch_cp_idx_local(rows, p.topk, idx, kv_off, p.kv_len, local, st);
+    if (e != cudaSuccess) return HS2_ERR_CUDA;
+    return cuda_status(launch_sparse(p, q, k, v, p.topk > 0 ? local : nullptr, out, st, 1, lse));
+}
+
+hs2_status hs2_cp_combine(int32_t n_parts, int64_t n_rows, int32_t head_dim, const void* out_parts,
+                          const float* lse_parts, void* out, float* lse, hs2_stream_t stream) {
+    if (n_parts < 1 || n_rows < 0) return HS2_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return HS2_ERR_UNSUPPORTED;
+    if (n_rows == 0) return HS2_OK;
+    if (!out_parts || !lse_parts || !out || !lse) return HS2_ERR_INVALID_ARG;
+    if (!aligned(out_parts, 16) || !aligned(out, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+        return HS2_ERR_INVALID_ARG;
+    return cuda_status(launch_cp_combine(n_parts, n_rows, head_dim, out_parts, lse_parts, out, lse,
+                                         reinterpret_cast<cudaStream_t>(stream)));
+}
+
+hs2_status hs2_cp_select_merge(const hs2_shape* shape, int32_t n_parts, const int64_t* kv_offs,
+                               const int32_t* idx_parts, const float* score_parts, int32_t* idx,
+                               hs2_stream_t stream) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (n_parts < 1 || kv_offs == nullptr) return HS2_ERR_INVALID_ARG;
+    if (n_parts > cp_max_parts()) return HS2_ERR_UNSUPPORTED;
+    for (int i = 0; i < n_parts; ++i)
+        if (kv_offs[i] < 0 || (i > 0 && kv_offs[i] <= kv_offs[i - 1])) return HS2_ERR_INVALID_ARG;
+    if (p.B == 0 || p.nq == 0 || p.topk == 0) return HS2_OK;
+    if (!idx_parts || !score_parts || !idx) return HS2_ERR_INVALID_ARG;
+    if (!aligned(idx_parts, 4) || !aligned(score_parts, 4) || !aligned(idx, 4)) return HS2_ERR_INVALID_ARG;
+    const int64_t rows = (int64_t)p.B * p.hkv * p.nq;
+    return cuda_status(launch_cp_select_merge(n_parts, rows, p.topk, idx_parts, score_parts, kv_offs, idx,
+                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
 hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info) {

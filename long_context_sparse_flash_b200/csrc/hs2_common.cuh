@@ -36,6 +36,9 @@ enum KernelId : uint32_t {
     KID_BRIDGE = 11,
     KID_BLOCK_SWEEP = 12,
     KID_BLOCK_TOPK = 13,
+    KID_CP_COMBINE = 14,
+    KID_CP_MERGE = 15,
+    KID_CP_IDX = 16,
 };
 
 __device__ __forceinline__ void report_error(WsHeader* h, uint32_t code, uint32_t kid, uint32_t a,

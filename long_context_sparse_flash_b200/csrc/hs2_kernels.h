@@ -66,7 +66,8 @@ cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* 
                                    void* scratch, int i_begin, int i_count, int64_t n_cand_max, int blk,
                                    cudaStream_t st);
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
-                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st);
+                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st,
+                             float* sel_score = nullptr);
 
 // Decode (one query per sequence): split-KV partial attention that also stores
 // the candidates' logits, exact combine -> out/lse, and (scores != nullptr)
@@ -81,6 +82,22 @@ cudaError_t launch_decode(const Problem& p, const void* q, const void* k, const 
 cudaError_t launch_sparse(const Problem& p, const void* q, const void* k, const void* v,
                           const int32_t* idx, void* out, cudaStream_t st, int with_window = 1,
                           float* lse = nullptr);
+
+// Context parallelism (cp_kernels.cu): the merges of per-slice results.
+//   launch_cp_combine: P partial (out bf16 [P][rows][D], natural-log lse [P][rows])
+//     -> out, lse over the union of the slices' keys;
+//   launch_cp_select_merge: P per-slice top-K lists (local rows [P][rows][K],
+//     ascending, -1 padded; scores [P][rows][K]) with the slices' first keys
+//     offs[P] (ascending, host array) -> the whole-context top-K, ascending;
+//   launch_cp_idx_local: whole-context idx -> the rows in [off, off + len),
+//     shifted by -off, in order, -1 padded.
+int cp_max_parts();
+cudaError_t launch_cp_combine(int n_parts, int64_t rows, int head_dim, const void* out_parts, const float* lse_parts,
+                              void* out, float* lse, cudaStream_t st);
+cudaError_t launch_cp_select_merge(int n_parts, int64_t rows, int topk, const int32_t* idx_parts,
+                                   const float* score_parts, const int64_t* offs, int32_t* idx, cudaStream_t st);
+cudaError_t launch_cp_idx_local(int64_t rows, int topk, const int32_t* idx, int64_t off, int64_t len, int32_t* out,
+                                cudaStream_t st);
 
 // Query position of query 0 of sequence b: q_pos0, or seq_len[b] - nq for decode
 // (clamped into [0, kv_len - nq]; a clamp is reported through the error word).

@@ -186,7 +186,10 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
     // key tiles of the causal range; with a split, this CTA takes the split-th of
     // n_split contiguous parts, tiles jt0 .. jt0 + n_tiles - 1 (loop indices below
     // are local, tile jt0 + j is read)
-    const int n_all = (int)((pos0 + i_last + PP_BN) / PP_BN);
+    // (a query may sit before the buffer's first key or past its last one when the
+    // buffer holds one slice of a longer context: its keys are those of the slice)
+    const int64_t t_last = min(pos0 + i_last, p.kv_len - 1);
+    const int n_all = t_last < 0 ? 0 : (int)((t_last + PP_BN) / PP_BN);
     const int per = (n_all + n_split - 1) / n_split;
     const int jt0 = min(split * per, n_all);
     const int n_tiles = min(per, n_all - jt0);
@@ -326,7 +329,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
         // ------------------------------------------------------------ softmax (warps 0-7)
         const int x = warp >> 2;                // query tile of this warpgroup
         const int r = tid & 127;                // row within the tile == TMEM lane
-        const int64_t t = pos0 + min(i0 + x * PP_BM + r, p.nq - 1);
+        const int64_t t = min(pos0 + min(i0 + x * PP_BM + r, p.nq - 1), p.kv_len - 1);  // last key of the row
         const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         const uint32_t s_addr = tmem + lane_off + x * PP_BN, o_addr = tmem + lane_off + C::O_COL + x * D;
         float m = -INFINITY, l = 0.f;
@@ -396,13 +399,18 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
         } else if (ok) {
             tc::fence_after_sync();
             const int i = i0 + x * PP_BM + r;
-            const float inv = 1.f / l;
+            const float inv = l > 0.f ? 1.f / l : 0.f;  // l = 0: the row has no key in the buffer
             __nv_bfloat16* orow = out + ((int64_t)(b * p.hq + h) * p.nq + i) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
-                tc::tmem_ld32(o_addr + c * 32, o);
-                tc::tmem_wait_ld();
+                if (n_tiles > 0) {
+                    tc::tmem_ld32(o_addr + c * 32, o);
+                    tc::tmem_wait_ld();
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) o[e] = 0.f;
+                }
                 if (i < p.nq) {
 #pragma unroll
                     for (int e = 0; e < 32; e += 8) {
@@ -415,7 +423,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                     }
                 }
             }
-            if (i < p.nq) lse[(int64_t)(b * p.hq + h) * p.nq + i] = (m + log2f(l)) * kLn2;
+            if (i < p.nq) lse[(int64_t)(b * p.hq + h) * p.nq + i] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
         }
     }
 
@@ -470,7 +478,7 @@ __global__ void __launch_bounds__(256) k1_split_combine_kernel(Problem p, int n_
     } else {
         *reinterpret_cast<uint32_t*>(orow) = pack_bf16(acc[0] * inv, acc[1] * inv);
     }
-    if (lane == 0) lse[row] = (M + log2f(L)) * kLn2;
+    if (lane == 0) lse[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
 }
 
 template <int D>
@@ -516,7 +524,9 @@ cudaError_t launch_full_tc_d(const Problem& p, const void* q, const void* k, con
 int full_tc_splits(const Problem& p) {
     if (p.seq_len != nullptr || p.nq < 64) return 1;
     const int64_t ctas = (int64_t)((p.nq + PP_QT * PP_BM - 1) / (PP_QT * PP_BM)) * p.hq * p.B;
-    const int64_t min_tiles = (p.q_pos0 + (p.nq < PP_QT * PP_BM ? p.nq : PP_QT * PP_BM) + PP_BN - 1) / PP_BN;
+    // key tiles of the shortest query block (keys past the buffer's end do not exist)
+    const int64_t first_keys = min(p.q_pos0 + (p.nq < PP_QT * PP_BM ? p.nq : PP_QT * PP_BM), p.kv_len);
+    const int64_t min_tiles = first_keys > 0 ? (first_keys + PP_BN - 1) / PP_BN : 0;
     auto idle = [](int64_t n) {
         const int64_t waves = (n + 147) / 148;
         return (double)(waves * 148 - n) / (double)(waves * 148);

@@ -97,7 +97,15 @@ struct SelArgs {
     int64_t sample_stride;  // S: the sampling pass reads keys 0, S, 2S, ...
     float* csum;            // block mode: [rows][cstride] sums of 32 consecutive candidate scores
     int64_t cstride;
+    float* sel_score;       // optional [B, H_kv, n_q, K]: the score of every selected key (-1 padding)
 };
+
+// Last candidate key of the query at t: t - window, and not past the buffer's
+// last key (when the buffer holds one slice of a longer context, a query may
+// sit past its end, or before its start: then it has no candidate here).
+__device__ __forceinline__ int64_t last_cand(const Problem& p, int64_t t) {
+    return min(t - p.window, p.kv_len - 1);
+}
 
 __device__ __forceinline__ uint32_t smid() {
     uint32_t r;
@@ -168,8 +176,10 @@ __device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uin
 
 // Keep, in list order, the entries with key > kth plus the first need_eq with
 // key == kth.  compact: write kept entries to the front of `list`; otherwise
-// write their j to `out`.  Returns the number kept.
-__device__ int warp_keep(uint2* list, int n, uint32_t kth, uint32_t need_eq, int32_t* out, bool compact) {
+// write their j to `out` (and their scores to `sout` unless it is null).
+// Returns the number kept.
+__device__ int warp_keep(uint2* list, int n, uint32_t kth, uint32_t need_eq, int32_t* out, bool compact,
+                         float* sout = nullptr) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
     uint32_t eq_seen = 0, written = 0;
@@ -185,8 +195,12 @@ __device__ int warp_keep(uint2* list, int n, uint32_t kth, uint32_t need_eq, int
         const uint32_t pos = written + __popc(tb & lt);
         __syncwarp();
         if (take) {
-            if (compact) list[pos] = e;
-            else out[pos] = (int32_t)e.y;
+            if (compact) {
+                list[pos] = e;
+            } else {
+                out[pos] = (int32_t)e.y;
+                if (sout) sout[pos] = __uint_as_float(e.x);
+            }
         }
         eq_seen += __popc(eqb);
         written += __popc(tb);
@@ -229,7 +243,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     const int nq_here = min(SL_QT, a.i_count - q0);
     const int64_t pos0 = seq_pos0(p, b, KID_SCORE) + a.i_begin;
     const int64_t t_max = pos0 + q0 + nq_here - 1;
-    const int64_t cand_end = t_max - p.window + 1;  // candidate keys are j < cand_end
+    const int64_t cand_end = last_cand(p, t_max) + 1;  // candidate keys are j < cand_end
     const int64_t row0 = (int64_t)(b * p.hkv + g) * a.i_count + q0;  // chunk row of query q0
     if (cand_end <= 0 && MODE != MODE_FILTER) return;
     const int n_ct = cand_end > 0 ? (int)((cand_end + SL_BN - 1) / SL_BN) : 0;
@@ -258,7 +272,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         const int q = tid;
         const bool live = q < nq_here;
         const int64_t t = pos0 + q0 + q;
-        const int64_t n = t - p.window + 1;
+        const int64_t n = last_cand(p, t) + 1;
         float bs = 0.f;
         int32_t act = live && n > 0;
         if (MODE == MODE_FILTER && act) bs = a.tau[row0 + q];
@@ -266,7 +280,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         r_cnt[q] = 0;
         r_cnt[SL_QT + q] = 0;
         r_lo[q] = act ? bs : INFINITY;
-        r_tlim[q] = (int32_t)(t - p.window);
+        r_tlim[q] = (int32_t)max(last_cand(p, t), (int64_t)-1);
         r_act[q] = act;
     }
     for (int c = tid; c < N; c += SL_THREADS) {
@@ -459,14 +473,14 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     const int q = wg * QH + qq;
                     if (q < nq_here) {
                         const int64_t t = pos0 + q0 + q;
-                        a.samples[(row0 + q) * SL_SPR + it * SL_BN + et] = (j <= t - p.window) ? sc[qq] : 0.f;
+                        a.samples[(row0 + q) * SL_SPR + it * SL_BN + et] = (j <= last_cand(p, t)) ? sc[qq] : 0.f;
                     }
                 }
             } else {
                 // FILTER / RETRY: ordered append (ascending j) of the candidates at or
                 // above each row's bound; key quarter kq's entries follow quarters < kq.
                 // Tiles entirely below every row's candidate limit skip the per-row test.
-                const bool all_valid = (int64_t)jb + SL_BN - 1 <= pos0 + q0 - p.window;
+                const bool all_valid = (int64_t)jb + SL_BN - 1 <= last_cand(p, pos0 + q0);
                 uint32_t bal[QH];
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
@@ -513,7 +527,8 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 const int q = wg * QH + et;
                 const int64_t t = pos0 + q0 + q;
                 // sampled keys S b <= t - window among the n_tiles * 128 read
-                const int64_t nv = t >= p.window ? (t - p.window) / S + 1 : 0;
+                const int64_t lc = last_cand(p, t);
+                const int64_t nv = lc >= 0 ? lc / S + 1 : 0;
                 a.s_valid[row0 + q] = (int)min(nv, (int64_t)n_tiles * SL_BN);
             }
         } else if (ok) {
@@ -521,16 +536,21 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
             for (int qq = kq; qq < QH; qq += 4) {
                 const int q = wg * QH + qq;
                 if (q >= nq_here) continue;
-                int32_t* orow = a.idx + ((int64_t)(b * p.hkv + g) * p.nq + a.i_begin + q0 + q) * p.topk;
+                const int64_t orow_off = ((int64_t)(b * p.hkv + g) * p.nq + a.i_begin + q0 + q) * p.topk;
+                int32_t* orow = a.idx + orow_off;
+                float* srow = a.sel_score ? a.sel_score + orow_off : nullptr;
                 if (!r_act[q]) {
                     if (MODE == MODE_FILTER) {  // no candidates at all (t < window)
-                        for (int u = lane; u < p.topk; u += 32) orow[u] = -1;
+                        for (int u = lane; u < p.topk; u += 32) {
+                            orow[u] = -1;
+                            if (srow) srow[u] = -1.f;
+                        }
                         if (lane == 0) a.status[row0 + q] = 0;
                     }
                     continue;
                 }
                 const int64_t t = pos0 + q0 + q;
-                const int64_t n = t - p.window + 1;
+                const int64_t n = last_cand(p, t) + 1;
                 const int n_sel = (int)(n < p.topk ? n : p.topk);
                 const int cnt = min(r_cnt[(n_tiles & 1) * SL_QT + q], cmax);
                 uint2* lst = lists + (int64_t)q * cmax;
@@ -540,15 +560,22 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 }
                 int written;
                 if (cnt == n_sel) {
-                    for (int u = lane; u < cnt; u += 32) orow[u] = (int32_t)lst[u].y;
+                    for (int u = lane; u < cnt; u += 32) {
+                        const uint2 e = lst[u];
+                        orow[u] = (int32_t)e.y;
+                        if (srow) srow[u] = __uint_as_float(e.x);
+                    }
                     written = cnt;
                 } else {
                     uint32_t kth, need_eq;
                     warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)n_sel, hist + warp * 256, kth,
                              need_eq);
-                    written = warp_keep(lst, cnt, kth, need_eq, orow, false);
+                    written = warp_keep(lst, cnt, kth, need_eq, orow, false, srow);
                 }
-                for (int u = written + lane; u < p.topk; u += 32) orow[u] = -1;
+                for (int u = written + lane; u < p.topk; u += 32) {
+                    orow[u] = -1;
+                    if (srow) srow[u] = -1.f;
+                }
                 if (lane == 0) a.status[row0 + q] = 0;
             }
         }
@@ -574,7 +601,7 @@ __global__ void __launch_bounds__(128) k2_thresh_kernel(Problem p, SelArgs a) {
     const int qi = (int)(row % a.i_count);
     const int b = (int)(row / ((int64_t)p.hkv * a.i_count));
     const int64_t t = seq_pos0(p, b, KID_TOPK) + a.i_begin + qi;
-    const int64_t n = t - p.window + 1;
+    const int64_t n = last_cand(p, t) + 1;
     const int s = a.s_valid[row];
     float tau = 0.f;
     if (n > a.cmax / 2 && s > 0) {
@@ -613,7 +640,7 @@ __global__ void __launch_bounds__(128) k2_block_topk_kernel(Problem p, SelArgs a
     const int bg = (int)(row / a.i_count);  // b * H_kv + g
     const int b = bg / p.hkv;
     const int64_t t = seq_pos0(p, b, KID_TOPK) + a.i_begin + qi;
-    const int64_t n_cand = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
+    const int64_t n_cand = last_cand(p, t) + 1 > 0 ? last_cand(p, t) + 1 : 0;
     const int n_blk = (int)(n_cand / blk);
     const int keep = min(p.topk / blk, n_blk);
     int32_t* orow = a.idx + ((int64_t)bg * p.nq + a.i_begin + qi) * p.topk;
@@ -773,15 +800,17 @@ size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max
 }
 
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
-                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st) {
+                             void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st,
+                             float* sel_score) {
     const int64_t rows = (int64_t)p.B * p.hkv * i_count;
     uint8_t* base = reinterpret_cast<uint8_t*>(scratch);
-    SelArgs a;
+    SelArgs a{};
     int n_slots;
     select_tc_geometry(p, i_count, n_cand_max, a.cmax, n_slots, a.slot_by_block);
     a.sample_stride = p.kv_len / (SL_SAMPLE_TILES * SL_BN) > 1 ? p.kv_len / (SL_SAMPLE_TILES * SL_BN) : 1;
     a.lse = lse;
     a.idx = idx;
+    a.sel_score = sel_score;
     a.slots = reinterpret_cast<uint2*>(base);
     base += (size_t)n_slots * SL_QT * a.cmax * sizeof(uint2);
     a.samples = reinterpret_cast<float*>(base);

@@ -55,7 +55,10 @@ __global__ void __launch_bounds__(W * 32) k3_sparse_kernel(Problem p, const __nv
     const int64_t pos0 = seq_pos0(p, b, KID_SPARSE);
     const int64_t t = pos0 + i;
     const int64_t w0 = t - p.window + 1 > 0 ? t - p.window + 1 : 0;
-    const int nwin = with_window ? (int)(t - w0 + 1) : 0;  // 0: the selected rows alone
+    // last window key held by the buffer (a slice of a longer context may end
+    // before t, or start after it: then fewer or no window rows are here)
+    const int64_t w_hi = min(t, p.kv_len - 1);
+    const int nwin = (with_window && w_hi >= w0) ? (int)(w_hi - w0 + 1) : 0;  // 0: the selected rows alone
 
     // attended rows: the selection's valid prefix (its length counted here),
     // then the window

@@ -22,6 +22,7 @@ STATUS = {0: "HS2_OK", 1: "HS2_ERR_INVALID_ARG", 2: "HS2_ERR_UNSUPPORTED", 3: "H
           4: "HS2_ERR_CUDA", 5: "HS2_ERR_DEVICE_CHECK", 6: "HS2_ERR_TIMEOUT"}
 HS2_ENTRY_FULL_SELECT, HS2_ENTRY_SPARSE, HS2_ENTRY_PREFILL, HS2_ENTRY_DECODE = 0, 1, 2, 3
 HS2_ENTRY_BLOCK_SELECT = 4
+HS2_ENTRY_CP_ATTN, HS2_ENTRY_CP_SELECT, HS2_ENTRY_CP_SPARSE = 5, 6, 7
 
 # every symbol include/hs2.h declares
 EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "hs2_sparse_attn",
@@ -29,11 +30,13 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_launch_count", "hs2_is_checked_build", "hs2_profile_start", "hs2_profile_stop",
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
            "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
-           "hs2_swa_branches")
+           "hs2_swa_branches", "hs2_cp_workspace_size", "hs2_cp_attn_partial", "hs2_cp_select_local",
+           "hs2_cp_sparse_partial", "hs2_cp_combine", "hs2_cp_select_merge")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
-                10: "select_retry", 11: "kv_bridge", 12: "block_sweep", 13: "block_topk"}
+                10: "select_retry", 11: "kv_bridge", 12: "block_sweep", 13: "block_topk",
+                14: "cp_combine", 15: "cp_select_merge", 16: "cp_idx_local"}
 
 
 class HS2Error(RuntimeError):
@@ -80,6 +83,14 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_prefill_chunk.argtypes = [sh, P, P, P, P, P, P, P, S, P]
     lib.hs2_full_attn_block_select.argtypes = [sh, ctypes.c_int32, P, P, P, P, P, P, P, S, P]
     lib.hs2_swa_branches.argtypes = [sh, P, P, P, P, P, P, P, P, P, P, P, S, P]
+    I64, I32 = ctypes.c_int64, ctypes.c_int32
+    lib.hs2_cp_workspace_size.argtypes = [sh, I64, ctypes.c_int]
+    lib.hs2_cp_workspace_size.restype = S
+    lib.hs2_cp_attn_partial.argtypes = [sh, I64, P, P, P, P, P, P, S, P]
+    lib.hs2_cp_select_local.argtypes = [sh, I64, P, P, P, P, P, P, S, P]
+    lib.hs2_cp_sparse_partial.argtypes = [sh, I64, P, P, P, P, P, P, P, S, P]
+    lib.hs2_cp_combine.argtypes = [I32, I64, I32, P, P, P, P, P]
+    lib.hs2_cp_select_merge.argtypes = [sh, I32, ctypes.POINTER(ctypes.c_int64), P, P, P, P]
     lib.hs2_decode.argtypes = [sh, P, P, P, P, P, P, P, P, S, P]
     lib.hs2_sparse_attn.argtypes = [sh, P, P, P, P, P, P, S, P]
     lib.hs2_decode_sparse.argtypes = [sh, P, P, P, P, P, P, P, S, P]
@@ -102,7 +113,8 @@ def load(checked: bool = False) -> ctypes.CDLL:
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
                  "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
-                 "hs2_swa_branches"):
+                 "hs2_swa_branches", "hs2_cp_attn_partial", "hs2_cp_select_local", "hs2_cp_sparse_partial",
+                 "hs2_cp_combine", "hs2_cp_select_merge"):
         getattr(lib, name).restype = ctypes.c_int
     _libs[checked] = lib
     return lib
@@ -188,6 +200,40 @@ def hs2_swa_branches(shape, q, k_swa, v_swa, k, v, idx, out_swa, lse_swa, out_se
                                           _ptr(idx), _ptr(out_swa), _ptr(lse_swa), _ptr(out_sel), _ptr(lse_sel),
                                           wp, wn, _stream(stream)),
            "hs2_swa_branches")
+
+
+def hs2_cp_workspace_size(shape, kv_off: int, entry: int, checked=False) -> int:
+    return int(load(checked).hs2_cp_workspace_size(ctypes.byref(shape), int(kv_off), int(entry)))
+
+
+def hs2_cp_attn_partial(shape, kv_off, q, k, v, out, lse, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_cp_attn_partial(ctypes.byref(shape), int(kv_off), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                             _ptr(lse), wp, wn, _stream(stream)), "hs2_cp_attn_partial")
+
+
+def hs2_cp_select_local(shape, kv_off, q, k, lse, idx, score, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_cp_select_local(ctypes.byref(shape), int(kv_off), _ptr(q), _ptr(k), _ptr(lse),
+                                             _ptr(idx), _ptr(score), wp, wn, _stream(stream)), "hs2_cp_select_local")
+
+
+def hs2_cp_sparse_partial(shape, kv_off, q, k, v, idx, out, lse, ws, stream=None, checked=False) -> None:
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_cp_sparse_partial(ctypes.byref(shape), int(kv_off), _ptr(q), _ptr(k), _ptr(v), _ptr(idx),
+                                               _ptr(out), _ptr(lse), wp, wn, _stream(stream)),
+           "hs2_cp_sparse_partial")
+
+
+def hs2_cp_combine(n_parts, n_rows, head_dim, out_parts, lse_parts, out, lse, stream=None, checked=False) -> None:
+    _check(load(checked).hs2_cp_combine(int(n_parts), int(n_rows), int(head_dim), _ptr(out_parts), _ptr(lse_parts),
+                                        _ptr(out), _ptr(lse), _stream(stream)), "hs2_cp_combine")
+
+
+def hs2_cp_select_merge(shape, kv_offs, idx_parts, score_parts, idx, stream=None, checked=False) -> None:
+    offs = (ctypes.c_int64 * len(kv_offs))(*[int(o) for o in kv_offs])
+    _check(load(checked).hs2_cp_select_merge(ctypes.byref(shape), len(kv_offs), offs, _ptr(idx_parts),
+                                             _ptr(score_parts), _ptr(idx), _stream(stream)), "hs2_cp_select_merge")
 
 
 def hs2_prefill_chunk(shape, q, k, v, out, lse, idx, ws, stream=None, checked=False) -> None:
@@ -291,7 +337,7 @@ def hs2_profile_start(checked=False) -> None:
 
 def hs2_profile_stop(checked=False) -> dict:
     """{kernel name: (total ms, launches)} recorded since hs2_profile_start."""
-    n = 16
+    n = 24
     ms = (ctypes.c_float * n)()
     cnt = (ctypes.c_uint64 * n)()
     _check(load(checked).hs2_profile_stop(n, ms, cnt), "hs2_profile_stop")

@@ -241,3 +241,44 @@ def test_swa_branches_validation_without_launch():
     for kw in (dict(batch=0), dict(n_q=0)):
         assert call(shape(**kw), *([None] * 10)) == 0
     assert nv.hs2_launch_count() == before
+
+
+def test_context_parallel_validation_without_launch():
+    """Slice calls and merges: shapes, offsets, workspace, sizes -- checked on the host."""
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    s = shape(n_q=256, q_pos0=5000, kv_len=2000)  # a slice of 2000 keys; queries after it
+    for e in (nv.HS2_ENTRY_CP_ATTN, nv.HS2_ENTRY_CP_SELECT, nv.HS2_ENTRY_CP_SPARSE):
+        assert nv.hs2_cp_workspace_size(s, 1000, e) >= 256
+        assert nv.hs2_cp_workspace_size(s, -1, e) == 0
+    assert nv.hs2_cp_workspace_size(s, 0, nv.HS2_ENTRY_FULL_SELECT) == 0
+    assert nv.hs2_workspace_size(s, nv.HS2_ENTRY_CP_ATTN) == 0  # slices are sized by the slice call
+    # local rows of the sparse step: one int32 per selected entry
+    assert nv.hs2_cp_workspace_size(s, 0, nv.HS2_ENTRY_CP_SPARSE) == 256 + 4 * 256 * 1024 * 4
+    need = nv.hs2_cp_workspace_size(s, 1000, nv.HS2_ENTRY_CP_ATTN)
+    assert L.hs2_cp_attn_partial(ctypes.byref(s), 1000, FAKE, FAKE, FAKE, FAKE, FAKE, None, 0, None) == 1
+    assert L.hs2_cp_attn_partial(ctypes.byref(s), 1000, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need - 1, None) == 3
+    assert L.hs2_cp_attn_partial(ctypes.byref(s), -5, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 1
+    small = shape(n_q=32, q_pos0=5000, kv_len=2000)
+    assert L.hs2_cp_attn_partial(ctypes.byref(small), 0, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, need, None) == 2
+    need_sel = nv.hs2_cp_workspace_size(s, 1000, nv.HS2_ENTRY_CP_SELECT)
+    assert L.hs2_cp_select_local(ctypes.byref(s), 1000, FAKE, FAKE, FAKE, None, FAKE, FAKE, need_sel, None) == 1
+    # merges
+    assert L.hs2_cp_combine(0, 10, 128, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert L.hs2_cp_combine(2, 10, 96, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert L.hs2_cp_combine(2, 0, 128, None, None, None, None, None) == 0
+    whole = shape(n_q=256, q_pos0=4000, kv_len=4256)
+    offs = (ctypes.c_int64 * 3)(0, 2000, 1000)  # not ascending
+    assert L.hs2_cp_select_merge(ctypes.byref(whole), 3, offs, FAKE, FAKE, FAKE, None) == 1
+    many = (ctypes.c_int64 * 17)(*range(0, 17 * 100, 100))
+    assert L.hs2_cp_select_merge(ctypes.byref(whole), 17, many, FAKE, FAKE, FAKE, None) == 2
+    assert nv.hs2_launch_count() == before
+
+
+def test_slice_offsets():
+    from long_context_sparse_flash_b200 import cp
+    assert cp.slice_offsets(10, 3) == [0, 4, 7]
+    assert cp.slice_offsets(8, 4) == [0, 2, 4, 6]
+    assert cp.slice_offsets(5, 1) == [0]
+    with pytest.raises(ValueError):
+        cp.slice_offsets(2, 3)
