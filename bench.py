@@ -260,6 +260,65 @@ def bench_swa_comparator(w: wl.Workload, inp: dict, dev, K: int, warmup: int, fl
                     "of the same shape; L2 flushed before each call"}
 
 
+def bench_context_parallel(w: wl.Workload, inp: dict, dev, K: int, warmup: int, flush: torch.Tensor,
+                           n_slices: int = 4):
+    """Context parallelism (a next row of the path) on one GPU: the cache cut into
+    n_slices slices, every slice's steps and every merge timed alone with CUDA
+    events (median of K, L2 flushed before each).  A rank of an n-GPU run would
+    execute one slice's steps plus every merge, so the per-rank time is the
+    slowest slice per step plus the merges; the exchanges (all-gathers) cannot
+    run on one GPU and are given as bytes received per rank and the time they
+    take at the measured 770 GB/s NVLink peer bandwidth."""
+    if w.decode or w.n_q < 64:
+        return None
+    from long_context_sparse_flash_b200 import cp
+    st = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(warmup):
+            flush.zero_()
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        res = None
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(st)
+            res = fn()
+            e1.record(st)
+        torch.cuda.synchronize()
+        return statistics.median(e0.elapsed_time(e1) for e0, e1 in ev), res
+
+    offs, ks, vs = cp.split_cache(inp["k"], inp["v"], n_slices)
+    q, W, Kk, p0 = inp["q"], w.window, w.topk, w.q_pos0
+    t1, parts = zip(*[timed(lambda s=s: cp.attn_partial(q, ks[s], vs[s], kv_off=offs[s], window=W, topk=Kk,
+                                                        q_pos0=p0)) for s in range(n_slices)])
+    O, L = torch.stack([x[0] for x in parts]), torch.stack([x[1] for x in parts])
+    tc1, (out, lse) = timed(lambda: cp.combine(O, L))
+    t2, sel = zip(*[timed(lambda s=s: cp.select_local(q, ks[s], lse, kv_off=offs[s], window=W, topk=Kk, q_pos0=p0))
+                    for s in range(n_slices)])
+    I, S = torch.stack([x[0] for x in sel]), torch.stack([x[1] for x in sel])
+    shape = nv.make_shape(w.batch, w.n_q, w.h_q, w.h_kv, w.head_dim, W, Kk, p0, w.kv_len)
+    tm, idx = timed(lambda: cp.select_merge(I, S, offs, shape=shape))
+    t3, sp = zip(*[timed(lambda s=s: cp.sparse_partial(inp["q_sparse"][0], ks[s], vs[s], idx, kv_off=offs[s],
+                                                       window=W, q_pos0=p0)) for s in range(n_slices)])
+    O3, L3 = torch.stack([x[0] for x in sp]), torch.stack([x[1] for x in sp])
+    tc3, _ = timed(lambda: cp.combine(O3, L3))
+    layers = w.n_sparse
+    per_rank = max(t1) + tc1 + max(t2) + tm + layers * (max(t3) + tc3)
+    rows_q = w.batch * w.h_q * w.n_q
+    rows_g = w.batch * w.h_kv * w.n_q
+    recv = (n_slices - 1) * (rows_q * (w.head_dim * 2 + 4) * (1 + layers) + rows_g * w.topk * 8)
+    nvlink_ms = recv / 770e9 * 1e3
+    del ks, vs
+    return {"slices": n_slices, "ms": {"attn_partial_max": round(max(t1), 4), "combine": round(tc1, 4),
+                                       "select_local_max": round(max(t2), 4), "select_merge": round(tm, 4),
+                                       "sparse_partial_max": round(max(t3), 4), "sparse_combine": round(tc3, 4)},
+            "per_rank_compute_ms": round(per_rank, 4), "bytes_received_per_rank": int(recv),
+            "exchange_ms_at_770GBs": round(nvlink_ms, 4),
+            "note": "slices run one after another on one GPU; per rank = slowest slice per step + the merges "
+                    "(every rank runs them); exchanges not run (one GPU), given as bytes and NVLink time"}
+
+
 def source_sha(path: str) -> str:
     return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
 
@@ -608,13 +667,18 @@ def run_ours(args):
     pk["l2_gather"] = l2_gather
     pk["ex2"] = ex2_rate
     rf, per_kernel = roofline(w, prof, args.steps, pk)
-    next_rows = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
-    sel_kernels = ("select_score", "select_thresh", "select_filter", "select_retry", "select_topk")
-    token_sel_ms = sum(per_kernel[n]["ms"] for n in sel_kernels if n in per_kernel)
-    blk = bench_block_select(w, inp, dev, args.steps, args.warmup, pk, flush, token_sel_ms)
-    if blk is not None:
-        next_rows["block_select"] = blk
-    next_rows["swa_comparator"] = bench_swa_comparator(w, inp, dev, args.steps, args.warmup, flush, step.idx)
+    next_rows = None
+    if not args.no_next_rows:
+        next_rows = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
+        sel_kernels = ("select_score", "select_thresh", "select_filter", "select_retry", "select_topk")
+        token_sel_ms = sum(per_kernel[n]["ms"] for n in sel_kernels if n in per_kernel)
+        blk = bench_block_select(w, inp, dev, args.steps, args.warmup, pk, flush, token_sel_ms)
+        if blk is not None:
+            next_rows["block_select"] = blk
+        next_rows["swa_comparator"] = bench_swa_comparator(w, inp, dev, args.steps, args.warmup, flush, step.idx)
+        cpr = bench_context_parallel(w, inp, dev, args.steps, args.warmup, flush)
+        if cpr is not None:
+            next_rows["context_parallel"] = cpr
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
 
@@ -693,6 +757,9 @@ def main():
     ap.add_argument("--workload", default="prefill_32k", choices=sorted(wl.WORKLOADS))
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="skip the next-row measurements (KV bridging, block selection, SWA comparator, "
+                         "context parallelism) that run after the timed steps")
     ap.add_argument("--cpu-rows", type=int, default=1536, help="query rows in the oracle baseline sample (about 10 s of host work)")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference-arm step")
     args = ap.parse_args()
