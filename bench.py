@@ -144,7 +144,8 @@ def bench_bridge(w: wl.Workload, dev, K: int, warmup: int, pk: dict) -> dict:
     v = torch.empty_like(k)
     pos = None if not w.decode else torch.full((w.batch,), cap - 1, dtype=torch.int64, device=dev)
     pos0 = 0 if w.decode else w.q_pos0
-    run = lambda: nv.kv_bridge(inp["hidden"], inp["w_kv"], k, v, pos0=pos0, seq_pos=pos)
+    ws = nv.kv_bridge_workspace(inp["hidden"], k)  # enables the split path for the decode append
+    run = lambda: nv.kv_bridge(inp["hidden"], inp["w_kv"], k, v, pos0=pos0, seq_pos=pos, ws=ws)
     for _ in range(warmup):
         run()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]

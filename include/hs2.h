@@ -348,7 +348,10 @@ hs2_status hs2_selftest_exp2(const float* x, float* y, int n, hs2_stream_t strea
  * rows would fall outside [0, kv_cap) writes nothing and is reported through
  * the error word (HS2_ERR_DEVICE_CHECK, kernel id 11).  ws: at least
  * hs2_workspace_size(..., HS2_ENTRY_SPARSE) bytes (the header), or NULL with
- * ws_bytes == 0 (then no error word).  Asynchronous on `stream`. */
+ * ws_bytes == 0 (then no error word).  With hs2_kv_bridge_workspace_size(shape)
+ * bytes, a call with few tokens (e.g. the decode append) splits d_model over
+ * more CTAs and sums fp32 partials in a second kernel (kernel id 11 too): the
+ * same rows, the fp32 sum taken in another order.  Asynchronous on `stream`. */
 typedef struct {
     int32_t batch;     /* sequences */
     int32_t n_new;     /* new tokens per sequence */
@@ -362,6 +365,11 @@ typedef struct {
 hs2_status hs2_kv_bridge(const hs2_bridge_shape* shape, const int64_t* seq_pos, const void* hidden,
                          const void* w_kv, void* k_cache, void* v_cache, void* ws, size_t ws_bytes,
                          hs2_stream_t stream);
+
+/* Workspace bytes that enable hs2_kv_bridge's split path for `shape` (the
+ * 256-byte header alone when the call has enough tokens not to need it; 0 for
+ * an invalid shape). */
+size_t hs2_kv_bridge_workspace_size(const hs2_bridge_shape* shape);
 
 /* Diagnostics: the gather-bandwidth probe behind the sparse layer's roofline
  * (the sparse layer reads whole 256-byte K/V rows in data-dependent order).

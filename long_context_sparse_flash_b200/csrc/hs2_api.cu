@@ -421,8 +421,20 @@ hs2_status hs2_kv_bridge(const hs2_bridge_shape* s, const int64_t* seq_pos, cons
     if (ws != nullptr && (ws_bytes < kHeader || !aligned(ws, 256))) return HS2_ERR_WORKSPACE;
     if (ws == nullptr && ws_bytes != 0) return HS2_ERR_INVALID_ARG;
     WsHeader* err = ws ? reinterpret_cast<WsHeader*>(ws) : nullptr;
+    // a workspace large enough for the split partials enables the split path
+    const size_t split = bridge_split_bytes(n_rows, s->d_model, s->h_kv, s->head_dim);
+    float* part = (ws != nullptr && split > 0 && ws_bytes >= kHeader + split)
+                      ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kHeader)
+                      : nullptr;
     return cuda_status(launch_bridge(n_rows, s->n_new, s->d_model, s->h_kv, s->head_dim, s->pos0, s->kv_cap, seq_pos,
-                                     hidden, w_kv, k_cache, v_cache, err, reinterpret_cast<cudaStream_t>(stream)));
+                                     hidden, w_kv, k_cache, v_cache, err, reinterpret_cast<cudaStream_t>(stream), part));
+}
+
+size_t hs2_kv_bridge_workspace_size(const hs2_bridge_shape* s) {
+    if (s == nullptr || s->batch < 0 || s->n_new < 0 || s->d_model <= 0 || s->d_model % 64 != 0 || s->h_kv <= 0 ||
+        (s->head_dim != 64 && s->head_dim != 128))
+        return 0;
+    return kHeader + bridge_split_bytes((int64_t)s->batch * s->n_new, s->d_model, s->h_kv, s->head_dim);
 }
 
 hs2_status hs2_sparse_attn(const hs2_shape* shape, const void* q, const void* k, const void* v, const int32_t* idx,

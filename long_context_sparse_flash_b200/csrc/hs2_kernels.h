@@ -26,10 +26,14 @@ void prof_begin(uint32_t kid, cudaStream_t st);
 void prof_end(cudaStream_t st);
 
 // K0: KV bridging -- kv = hidden W_kv^T written as bf16 into k_cache / v_cache
-// rows pos_b + i (see hs2_kv_bridge in hs2.h); err may be null.
+// rows pos_b + i (see hs2_kv_bridge in hs2.h); err may be null.  With `part`
+// (bridge_split_bytes(...) bytes, or null) a call with few tokens splits d_model
+// over more CTAs and sums the fp32 partials in a second kernel.
+int bridge_splits(int64_t n_rows, int d_model, int h_kv, int head_dim);
+size_t bridge_split_bytes(int64_t n_rows, int d_model, int h_kv, int head_dim);
 cudaError_t launch_bridge(int64_t n_rows, int n_new, int d_model, int h_kv, int head_dim, int64_t pos0,
                           int64_t kv_cap, const int64_t* seq_pos, const void* hidden, const void* w_kv,
-                          void* k_cache, void* v_cache, WsHeader* err, cudaStream_t st);
+                          void* k_cache, void* v_cache, WsHeader* err, cudaStream_t st, float* part = nullptr);
 
 // K1 on tcgen05/TMEM/TMA (prefill-shaped calls: 128-row query tiles).  When
 // full_tc_splits(p) > 1 and `scratch` holds full_tc_split_scratch_bytes(p),

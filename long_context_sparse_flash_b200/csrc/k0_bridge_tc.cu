@@ -18,6 +18,11 @@
 //              both K-major, accumulator in 256 TMEM columns
 // Operand tiles are 128-byte swizzled (TMA SWIZZLE_128B).  Every wait is
 // bounded; a stalled CTA reports HS2_ERR_TIMEOUT, drains and exits.
+//
+// Few tokens (the decode-time append: one token per sequence) leave only a few
+// CTAs to stream all of W_kv.  Then the d_model range is split over blockIdx.z:
+// each CTA accumulates its slice of the K-steps and writes an fp32 partial
+// tile, and k0_bridge_reduce_kernel sums the partials and writes the cache rows.
 #include <cudaTypedefs.h>
 
 #include "hs2_kernels.h"
@@ -53,7 +58,22 @@ struct BridgeArgs {
     __nv_bfloat16* k_cache;
     __nv_bfloat16* v_cache;
     WsHeader* err;
+    int k_per;            // K-steps per split (all of them without a split)
+    float* part;          // split: fp32 partials [split][n_rows][features], else null
 };
+
+// Cache row of token m, or -1 if its sequence's rows would leave the cache
+// (then the first token of the sequence reports it).
+__device__ __forceinline__ int64_t bridge_row(const BridgeArgs& a, int64_t m, int64_t& b, bool report) {
+    b = m / a.n_new;
+    const int64_t i = m - b * a.n_new;
+    const int64_t pb = a.seq_pos ? a.seq_pos[b] : a.pos0;
+    if (pb < 0 || pb + a.n_new > a.kv_cap) {
+        if (report) report_error(a.err, HS2_ERR_DEVICE_CHECK, KID_BRIDGE, (uint32_t)b, (uint32_t)i);
+        return -1;
+    }
+    return pb + i;
+}
 
 __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                                   const __grid_constant__ CUtensorMap tm_w,
@@ -70,7 +90,9 @@ __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_c
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t m0 = (int64_t)blockIdx.y * BR_BM;  // first token row
     const int n0 = blockIdx.x * BR_BN;               // first output feature
-    const int n_k = a.d_model / BR_BK;
+    const int split = blockIdx.z;
+    const int kb0 = split * a.k_per;                 // first K-step of this CTA
+    const int n_k = min(a.d_model / BR_BK - kb0, a.k_per);
 
     if (tid == 0) {
         for (int i = 0; i < BB_COUNT; ++i) tc::mbar_init(bar(i), 1);
@@ -93,8 +115,8 @@ __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_c
                     !tc::mbar_wait(bar(BB_EMPTY + s), ((kk - BR_NS) / BR_NS) & 1, ab, a.err, KID_BRIDGE, 1))
                     break;
                 tc::mbar_expect_tx(bar(BB_FULL + s), BR_ABLK + BR_BBLK);
-                tc::tma_load_3d(sA + s * BR_ABLK, &tm_x, bar(BB_FULL + s), kk * BR_BK, (int)m0, 0);
-                tc::tma_load_3d(sB + s * BR_BBLK, &tm_w, bar(BB_FULL + s), kk * BR_BK, n0, 0);
+                tc::tma_load_3d(sA + s * BR_ABLK, &tm_x, bar(BB_FULL + s), (kb0 + kk) * BR_BK, (int)m0, 0);
+                tc::tma_load_3d(sB + s * BR_BBLK, &tm_w, bar(BB_FULL + s), (kb0 + kk) * BR_BK, n0, 0);
                 issued = kk + 1;
             }
             if (ab->flag) {  // drain: every issued load lands before the CTA exits
@@ -136,18 +158,13 @@ __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_c
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const bool ok = __all_sync(~0u, tc::mbar_wait(bar(BB_DONE), 0, ab, a.err, KID_BRIDGE, 3));
         tc::fence_after_sync();
-        // destination of this token: sequence b, cache row pos_b + i
+        // destination of this token: sequence b, cache row pos_b + i (a split
+        // writes its fp32 partial row instead; the reduce places it)
         bool write = ok && m < a.n_rows;
         int64_t b = 0, row = 0;
-        if (write) {
-            b = m / a.n_new;
-            const int64_t i = m - b * a.n_new;
-            const int64_t pb = a.seq_pos ? a.seq_pos[b] : a.pos0;
-            row = pb + i;
-            if (pb < 0 || pb + a.n_new > a.kv_cap) {  // the whole sequence is skipped
-                report_error(a.err, HS2_ERR_DEVICE_CHECK, KID_BRIDGE, (uint32_t)b, (uint32_t)i);
-                write = false;
-            }
+        if (write && a.part == nullptr) {
+            row = bridge_row(a, m, b, true);
+            write = row >= 0;  // the whole sequence is skipped
         }
         const int hd = a.h_kv * a.head_dim;
         const bool is_v = n0 >= hd;
@@ -160,7 +177,11 @@ __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_c
                 tc::tmem_ld32(tmem + lane_off + c * 32, o);
                 tc::tmem_wait_ld();
             }
-            if (write) {
+            if (write && a.part != nullptr) {
+                float* dst = a.part + ((int64_t)split * a.n_rows + m) * (2 * a.h_kv * a.head_dim) + n0 + c * 32;
+#pragma unroll
+                for (int e = 0; e < 32; e += 4) *reinterpret_cast<float4*>(dst + e) = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
+            } else if (write) {
                 const int f = f0 + c * 32;  // 32 features of one head
                 const int h = f / a.head_dim, d = f - h * a.head_dim;
                 __nv_bfloat16* dst = cache + (((int64_t)b * a.h_kv + h) * a.kv_cap + row) * a.head_dim + d;
@@ -185,11 +206,60 @@ __global__ void __launch_bounds__(BR_THREADS, 1) k0_bridge_kernel(const __grid_c
     }
 }
 
+// Sum of the n_split fp32 partials of 8 features of one token, written as bf16
+// into its cache row.
+__global__ void __launch_bounds__(256) k0_bridge_reduce_kernel(BridgeArgs a, int n_split) {
+    const int features = 2 * a.h_kv * a.head_dim;
+    const int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t m = u / (features / 8);
+    if (m >= a.n_rows) return;
+    const int f = (int)(u - m * (features / 8)) * 8;
+    int64_t b;
+    const int64_t row = bridge_row(a, m, b, f == 0);
+    if (row < 0) return;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int s = 0; s < n_split; ++s) {
+        const float* src = a.part + ((int64_t)s * a.n_rows + m) * features + f;
+        const float4 x = *reinterpret_cast<const float4*>(src);
+        const float4 y = *reinterpret_cast<const float4*>(src + 4);
+        acc[0] += x.x, acc[1] += x.y, acc[2] += x.z, acc[3] += x.w;
+        acc[4] += y.x, acc[5] += y.y, acc[6] += y.z, acc[7] += y.w;
+    }
+    const int hd = a.h_kv * a.head_dim;
+    const bool is_v = f >= hd;
+    const int fl = is_v ? f - hd : f;
+    const int h = fl / a.head_dim, d = fl - h * a.head_dim;
+    __nv_bfloat16* cache = is_v ? a.v_cache : a.k_cache;
+    uint4 v;
+    v.x = pack_bf16(acc[0], acc[1]);
+    v.y = pack_bf16(acc[2], acc[3]);
+    v.z = pack_bf16(acc[4], acc[5]);
+    v.w = pack_bf16(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(cache + ((b * a.h_kv + h) * a.kv_cap + row) * a.head_dim + d) = v;
+}
+
 }  // namespace
+
+// Split of the K-steps for a call of n_rows tokens: enough CTAs to stream the
+// weights with most SMs; 1 when the token and feature tiles already fill them.
+int bridge_splits(int64_t n_rows, int d_model, int h_kv, int head_dim) {
+    const int64_t ctas = (int64_t)(2 * h_kv * head_dim / BR_BN) * ((n_rows + BR_BM - 1) / BR_BM);
+    const int n_k = d_model / BR_BK;
+    if (ctas >= 74 || n_k < 2) return 1;
+    int want = (int)(148 / ctas);
+    if (want > n_k) want = n_k;
+    const int per = (n_k + want - 1) / want;
+    return (n_k + per - 1) / per;  // every split gets at least one K-step
+}
+
+size_t bridge_split_bytes(int64_t n_rows, int d_model, int h_kv, int head_dim) {
+    const int S = bridge_splits(n_rows, d_model, h_kv, head_dim);
+    return S > 1 ? (size_t)S * n_rows * 2 * h_kv * head_dim * 4 : 0;
+}
 
 cudaError_t launch_bridge(int64_t n_rows, int n_new, int d_model, int h_kv, int head_dim, int64_t pos0,
                           int64_t kv_cap, const int64_t* seq_pos, const void* hidden, const void* w_kv,
-                          void* k_cache, void* v_cache, WsHeader* err, cudaStream_t st) {
+                          void* k_cache, void* v_cache, WsHeader* err, cudaStream_t st, float* part) {
     if (n_rows == 0) return cudaSuccess;
     const int features = 2 * h_kv * head_dim;
     CUtensorMap mx, mw;
@@ -210,10 +280,22 @@ cudaError_t launch_bridge(int64_t n_rows, int n_new, int d_model, int h_kv, int 
     a.k_cache = reinterpret_cast<__nv_bfloat16*>(k_cache);
     a.v_cache = reinterpret_cast<__nv_bfloat16*>(v_cache);
     a.err = err;
+    const int n_k = d_model / BR_BK;
+    const int S = part != nullptr ? bridge_splits(n_rows, d_model, h_kv, head_dim) : 1;
+    a.k_per = (n_k + S - 1) / S;
+    a.part = S > 1 ? part : nullptr;
     // feature tiles fastest: CTAs of one token tile run together and share it in L2
-    dim3 grid(features / BR_BN, (unsigned)((n_rows + BR_BM - 1) / BR_BM));
+    dim3 grid(features / BR_BN, (unsigned)((n_rows + BR_BM - 1) / BR_BM), (unsigned)S);
     prof_begin(KID_BRIDGE, st);
     k0_bridge_kernel<<<grid, BR_THREADS, BR_SMEM, st>>>(mx, mw, a);
+    prof_end(st);
+    count_launch();
+    if (S == 1) return cudaGetLastError();
+    cudaError_t e2 = cudaGetLastError();
+    if (e2 != cudaSuccess) return e2;
+    const int64_t threads = n_rows * (features / 8);
+    prof_begin(KID_BRIDGE, st);
+    k0_bridge_reduce_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(a, S);
     prof_end(st);
     count_launch();
     return cudaGetLastError();

@@ -31,7 +31,8 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_full_attn_select_static", "hs2_static_scratch_bytes", "hs2_selftest_exp2",
            "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
            "hs2_swa_branches", "hs2_cp_workspace_size", "hs2_cp_attn_partial", "hs2_cp_select_local",
-           "hs2_cp_sparse_partial", "hs2_cp_combine", "hs2_cp_select_merge")
+           "hs2_cp_sparse_partial", "hs2_cp_combine", "hs2_cp_select_merge",
+           "hs2_kv_bridge_workspace_size")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
@@ -109,6 +110,8 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_gather_probe.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int32, P, P]
     lib.hs2_ex2_probe.argtypes = [ctypes.c_int32, P, P, ctypes.POINTER(ctypes.c_int64)]
     lib.hs2_kv_bridge.argtypes = [ctypes.POINTER(hs2_bridge_shape), P, P, P, P, P, P, S, P]
+    lib.hs2_kv_bridge_workspace_size.argtypes = [ctypes.POINTER(hs2_bridge_shape)]
+    lib.hs2_kv_bridge_workspace_size.restype = S
     for name in ("hs2_workspace_init", "hs2_full_attn_select", "hs2_prefill_chunk", "hs2_decode",
                  "hs2_sparse_attn", "hs2_decode_sparse", "hs2_get_device_status", "hs2_is_checked_build",
                  "hs2_profile_start", "hs2_profile_stop", "hs2_full_attn_select_static", "hs2_selftest_exp2",
@@ -314,6 +317,20 @@ def kv_bridge(hidden: torch.Tensor, w_kv: torch.Tensor, k_cache: torch.Tensor, v
     shape = hs2_bridge_shape(batch=B, n_new=n_new, d_model=d_model, h_kv=h_kv, head_dim=D, reserved=0,
                              pos0=pos0, kv_cap=kv_cap)
     hs2_kv_bridge(shape, seq_pos, hidden, w_kv, k_cache, v_cache, ws, stream, checked)
+
+
+def kv_bridge_workspace(hidden: torch.Tensor, k_cache: torch.Tensor, stream=None, checked: bool = False):
+    """A workspace of hs2_kv_bridge_workspace_size bytes (enables the split path), initialised."""
+    B, n_new, d_model = hidden.shape
+    _, h_kv, kv_cap, D = k_cache.shape
+    shape = hs2_bridge_shape(batch=B, n_new=n_new, d_model=d_model, h_kv=h_kv, head_dim=D, reserved=0, pos0=0,
+                             kv_cap=kv_cap)
+    n = int(load(checked).hs2_kv_bridge_workspace_size(ctypes.byref(shape)))
+    if n == 0:
+        raise HS2Error(1, "hs2_kv_bridge_workspace_size")
+    ws = torch.empty(n, dtype=torch.uint8, device=hidden.device)
+    hs2_workspace_init(ws, stream=stream, checked=checked)
+    return ws
 
 
 def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):

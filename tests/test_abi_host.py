@@ -185,6 +185,11 @@ def test_kv_bridge_validation_without_launch():
     assert call(bs(), ws=None, ws_bytes=256) == 1
     assert call(bs(n_new=0)) == 0                # empty: no launch
     assert call(bs(batch=0)) == 0
+    # workspace for the split path: fp32 partials of every split when few CTAs would stream W_kv
+    ws_size = lambda sh: L.hs2_kv_bridge_workspace_size(ctypes.byref(sh))
+    assert ws_size(bs(batch=64, n_new=1, d_model=4096, kv_cap=300)) == 256 + 32 * 64 * 1024 * 4
+    assert ws_size(bs(batch=1, n_new=32768, d_model=4096, kv_cap=32768)) == 256  # enough token tiles
+    assert ws_size(bs(d_model=100)) == 0
     assert nv.hs2_launch_count() == before
 
 

@@ -100,3 +100,45 @@ def test_bridge_out_of_range_position_reported_and_skipped():
     assert torch.all(k[1] == 7.0) and torch.all(v[1] == -3.0)  # nothing of sequence 1 is written
     _check({"hidden": inp["hidden"][[0, 2]], "w_kv": inp["w_kv"]}, k[[0, 2]], v[[0, 2]],
            [[3, 4], [10, 11]], h_kv, d)
+
+
+@pytest.mark.parametrize("batch,n_new,d_model,h_kv,d", [
+    (64, 1, wl.BRIDGE_D_MODEL, 4, 128),   # the 128K decode step's append: 4 CTAs without the split
+    (8, 1, 448, 2, 128),                  # 7 K-steps: a split into uneven parts
+    (3, 40, 1024, 4, 64),                 # several tokens per sequence, D = 64
+])
+def test_bridge_split_path(batch, n_new, d_model, h_kv, d):
+    """With hs2_kv_bridge_workspace_size bytes, few-token calls split d_model over
+    more CTAs and sum fp32 partials in a second kernel; same rows, oracle parity."""
+    from long_context_sparse_flash_b200 import native
+    inp = wl.make_bridge_inputs(batch, n_new, d_model, h_kv, d, "cuda", seed=8)
+    kv_cap = 300
+    k, v = _sentinel_caches(batch, h_kv, kv_cap, d)
+    ws = native.kv_bridge_workspace(inp["hidden"], k)
+    assert ws.numel() > 256  # the split path is taken
+    pos = torch.tensor([(37 * b) % (kv_cap - n_new + 1) for b in range(batch)], dtype=torch.int64, device="cuda")
+    before = nv.hs2_launch_count()
+    nv.kv_bridge(inp["hidden"], inp["w_kv"], k, v, seq_pos=pos, ws=ws)
+    rc, info = nv.hs2_get_device_status(ws)
+    assert rc == 0, info
+    assert nv.hs2_launch_count() == before + 2  # partials + reduce
+    _check(inp, k, v, [list(range(p, p + n_new)) for p in pos.tolist()], h_kv, d)
+    # the split and the one-pass kernels agree to fp32 rounding (bf16 outputs within one ulp)
+    k2, v2 = _sentinel_caches(batch, h_kv, kv_cap, d)
+    nv.kv_bridge(inp["hidden"], inp["w_kv"], k2, v2, seq_pos=pos)
+    torch.cuda.synchronize()
+    P.assert_close(P.to_f64(k), P.to_f64(k2), "split vs one-pass K", atol=1e-2, rtol=1e-2)
+
+
+def test_bridge_split_path_reports_out_of_range_sequences():
+    batch, d_model, h_kv, d, kv_cap = 4, 512, 4, 64, 16
+    inp = wl.make_bridge_inputs(batch, 1, d_model, h_kv, d, "cuda", seed=9)
+    k, v = _sentinel_caches(batch, h_kv, kv_cap, d)
+    ws = nv.kv_bridge_workspace(inp["hidden"], k)
+    pos = torch.tensor([0, 16, 5, -1], dtype=torch.int64, device="cuda")  # sequences 1 and 3 out of range
+    nv.kv_bridge(inp["hidden"], inp["w_kv"], k, v, seq_pos=pos, ws=ws)
+    rc, info = nv.hs2_get_device_status(ws)
+    assert rc == 5 and info[1] == 11, (rc, info)
+    for b in (1, 3):
+        assert torch.all(k[b] == 7.0) and torch.all(v[b] == -3.0)
+    _check({"hidden": inp["hidden"][[0, 2]], "w_kv": inp["w_kv"]}, k[[0, 2]], v[[0, 2]], [[0], [5]], h_kv, d)
