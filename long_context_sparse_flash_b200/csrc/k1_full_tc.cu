@@ -23,6 +23,12 @@
 // Operand tiles are 128-byte swizzled (TMA SWIZZLE_128B), rows of 64 bf16.
 // Every wait is bounded (tc::mbar_wait): a stalled CTA reports HS2_ERR_TIMEOUT
 // through the error word, drains its own copies, frees its TMEM and exits.
+//
+// The K/V buffer may hold one slice of a longer context (context parallelism:
+// positions shifted by the slice's first key).  A query past the buffer's last
+// key sees all of it; a query before its first key sees none (output 0, LSE
+// -inf).  Long causal rows with few CTAs split their key range over blockIdx.z
+// and merge the parts exactly (k1_split_combine_kernel).
 #include <cudaTypedefs.h>
 
 #include "exp2_poly.cuh"

@@ -29,7 +29,18 @@
 //           candidates passed (tau overestimated), the row is marked,
 //   RETRY   re-runs only the tiles with a marked row, with bound 0.
 // Ordering of equal scores: the survivor lists are ascending in j, and every
-// selection step keeps the first (lowest-j) entries among equal keys.
+// selection step keeps the first (lowest-j) entries among equal keys.  The
+// exact select can also write each selected key's score (used to merge the
+// selections of several slices of one context).
+//
+// The same sweep in MODE_BLOCK serves block-level selection (the design
+// token-level selection replaces, same report and section): the epilogue sums
+// each warp's 32 keys per query and writes one float per 32 candidate keys,
+// and k2_block_topk_kernel ranks whole blocks from those sums.
+//
+// The buffer may hold one slice of a longer context (context parallelism):
+// positions are then shifted by the slice's first key, and every candidate
+// range is cut at the slice's last key (last_cand).
 #include <cudaTypedefs.h>
 
 #include "hs2_kernels.h"
@@ -265,7 +276,6 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     const int64_t S = a.sample_stride;
     const int64_t n_sb = cand_end > 0 ? (cand_end + S - 1) / S : 0;  // sampled keys below the candidate limit
     const int n_tiles = MODE == MODE_SAMPLE ? (int)min((int64_t)SL_SAMPLE_TILES, (n_sb + SL_BN - 1) / SL_BN) : n_ct;
-    auto tile_of = [&](int it) -> int { return it; };
 
     // row state
     if (tid < SL_QT) {
@@ -312,7 +322,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 if (it >= SL_NS && !tc::mbar_wait(bar(SB_KEMPTY + s), ((it - SL_NS) / SL_NS) & 1, ab, p.err, KID_SCORE, 1))
                     break;
                 tc::mbar_expect_tx(bar(SB_KFULL + s), C::KB * C::KBLK);
-                const int kt = tile_of(it);
+                const int kt = it;
                 for (int kb = 0; kb < C::KB; ++kb)
                     tc::tma_load_3d(sK + (s * C::KB + kb) * C::KBLK, &tm_k, bar(SB_KFULL + s), kb * 64, kt * SL_BN,
                                     b * p.hkv + g);
@@ -368,7 +378,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         }
         for (int it = 0; it < n_tiles; ++it) {
             const int sb = it & 1;
-            const int64_t jb = (int64_t)tile_of(it) * SL_BN;
+            const int64_t jb = (int64_t)it * SL_BN;
             const int64_t j = MODE == MODE_SAMPLE ? S * (jb + et) : jb + et;
             // one thread per warpgroup waits (bounded) and the named barrier hands
             // the result to its four warps, so they leave the loop together

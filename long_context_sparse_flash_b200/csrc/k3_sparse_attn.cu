@@ -18,7 +18,13 @@
 //                                             B = P^T via movmatrix.trans
 // The group's heads sit in the MMA's N = 8 columns (padded when G < 8), so no
 // tensor-core work is spent on padding rows of M.  With W > 1 warps per CTA the
-// warps' partial (max, sum, O) would be merged exactly at the end.
+// warps' partial (max, sum, O) are merged exactly at the end.
+//
+// Two further uses share the kernel: with_window = 0 attends to the selected
+// rows alone (the selected branch of the predecessor design's two-branch layer),
+// and a non-null lse receives the natural-log LSE of the attended logits (both
+// branches, and the per-slice partials of context parallelism, are merged by
+// it).  A query with no attended row writes 0 and LSE -inf.
 #include "hs2_kernels.h"
 
 namespace hs2 {
