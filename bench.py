@@ -353,20 +353,74 @@ def dram_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
+    """SM clocks and clock-event reasons of this process's GPU while the timed
+    region runs: read through NVML every 5 ms on a background thread (so a short
+    region still gets samples), or through `nvidia-smi -lms 200` if NVML is not
+    available.  Read-only: no clock or other GPU setting is changed."""
     FIELDS = ("uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
               "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
               "clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
     def __init__(self, device: int):
         self.proc = None
         self.uuid = None
+        self.nvml = None
+        self.handle = None
+        self.thread = None
+        self.samples = []
         try:
             u = str(torch.cuda.get_device_properties(device).uuid)
             self.uuid = u if u.startswith("GPU-") else "GPU-" + u
         except Exception:
             pass
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            # this process's GPU: by PCI address (CUDA and NVML number GPUs differently)
+            pr = torch.cuda.get_device_properties(device)
+            bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.handle = None
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    uid = pynvml.nvmlDeviceGetUUID(h)
+                    uid = uid.decode() if isinstance(uid, bytes) else uid
+                    if self.uuid is not None and uid == self.uuid:
+                        self.handle = h
+                        break
+            if self.handle is not None:
+                self.nvml = pynvml
+            else:
+                self.error = f"no NVML device at {bus} or {self.uuid}"
+        except Exception as e:
+            self.nvml = None
+            self.error = f"NVML: {type(e).__name__}: {e}"
+
+    def _run_nvml(self):
+        nv_ = self.nvml
+        bits = [nv_.nvmlClocksEventReasonHwSlowdown, nv_.nvmlClocksEventReasonHwThermalSlowdown,
+                nv_.nvmlClocksEventReasonSwThermalSlowdown, nv_.nvmlClocksEventReasonSwPowerCap]
+        mx = nv_.nvmlDeviceGetMaxClockInfo(self.handle, nv_.NVML_CLOCK_SM)
+        while not self._stop.is_set():
+            try:
+                sm = nv_.nvmlDeviceGetClockInfo(self.handle, nv_.NVML_CLOCK_SM)
+                r = nv_.nvmlDeviceGetCurrentClocksEventReasons(self.handle)
+                self.samples.append((float(sm), float(mx), [n for n, b in zip(self.NAMES, bits) if r & b]))
+            except Exception:
+                pass
+            self._stop.wait(0.005)
 
     def start(self):
+        if self.nvml is not None:
+            import threading
+            self._stop = threading.Event()
+            self.thread = threading.Thread(target=self._run_nvml, daemon=True)
+            self.thread.start()
+            return
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                                           "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
@@ -374,33 +428,34 @@ class ClockSampler:
             self.proc = None
 
     def stop(self):
-        if self.proc is None:
-            return None
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=10)
-        except Exception:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
-        if self.uuid:
-            mine = [r for r in rows if r[0] == self.uuid]
-            rows = mine or rows
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+            rows = self.samples
+        elif self.proc is not None:
+            self.proc.terminate()
             try:
-                sm.append(float(r[1]))
-                mx.append(float(r[2]))
-                for name, val in zip(names, r[4:8]):
-                    if val.strip().lower() == "active":
-                        reasons.add(name)
-            except (ValueError, IndexError):
-                continue
-        if not sm:
+                out, _ = self.proc.communicate(timeout=10)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            rows = []
+            for r in (x.split(", ") for x in out.strip().splitlines() if x.strip()):
+                if self.uuid and r[0] != self.uuid:
+                    continue
+                try:
+                    rows.append((float(r[1]), float(r[2]),
+                                 [n for n, v in zip(self.NAMES, r[4:8]) if v.strip().lower() == "active"]))
+                except (ValueError, IndexError):
+                    continue
+        else:
             return None
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not rows:
+            return {"samples": 0, "error": self.error or "no sample during the timed region"}
+        reasons = sorted({n for _, _, rs in rows for n in rs})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows),
+                "source": "nvml" if self.thread is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
