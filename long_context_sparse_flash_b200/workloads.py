@@ -120,11 +120,13 @@ def _segment_keys(w: Workload, device, gen: torch.Generator) -> torch.Tensor:
 
 
 def _plant(w: Workload, q_seq: torch.Tensor, k_seq: torch.Tensor, probes: List[int],
-           gen: torch.Generator) -> None:
+           gen: torch.Generator) -> Dict[int, List[int]]:
     """Plant w.needles keys per probe query i (absolute t = q_pos0 + i) at distinct
     older positions j <= t - window not used by an earlier plant:
-    k_{g,j} = 2 * normalize(sum_{h in g} q_{h,t}) + 0.1 * N(0,1)."""
+    k_{g,j} = 2 * normalize(sum_{h in g} q_{h,t}) + 0.1 * N(0,1).
+    Returns the planted positions of each probe query."""
     m = w.needles
+    planted: Dict[int, List[int]] = {}
     dev = k_seq.device
     used = torch.zeros(w.kv_len, dtype=torch.bool, device=dev)
     G = w.group
@@ -152,6 +154,8 @@ def _plant(w: Workload, q_seq: torch.Tensor, k_seq: torch.Tensor, probes: List[i
         qd = qd / qd.norm(dim=-1, keepdim=True).clamp_min(1e-12)
         noise = torch.randn(w.h_kv, m, w.head_dim, generator=gen, device=dev)
         k_seq[:, pos, :] = (2.0 * qd[:, None, :] + 0.1 * noise).to(torch.bfloat16)
+        planted[i] = seen
+    return planted
 
 
 def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
@@ -163,6 +167,7 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
       k, v     bf16 [B, H_kv, kv_len, D] the shared Cross-Decoder cache
       q_sparse list of n_sparse bf16 [B, H_q, n_q, D] (fresh draw per layer)
       probes   list (per sequence) of query indices that got planted needles
+      needles  list (per sequence) of {probe query index: planted key positions}
     """
     seed = w.seed if seed is None else int(seed)
     B, Hq, Hk, D, N, nq = w.batch, w.h_q, w.h_kv, w.head_dim, w.kv_len, w.n_q
@@ -173,19 +178,22 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
     gn = _gen(device, seed * 1000 + SUB_NEEDLE)
     k = torch.empty(B, Hk, N, D, dtype=torch.bfloat16, device=device)
     probes_all = []
+    needles_all = []
     for b in range(B):
         if w.keys == "segments":
             k[b] = _segment_keys(w, device, gs)
         else:
             k[b] = (torch.randn(Hk, N, D, generator=gk, device=device) * 0.5).to(torch.bfloat16)
         probes = []
+        planted = {}
         if w.needles > 0:
             n_probe = min(nq, max(1, N // (8 * w.needles)))
             # probe queries: seeded, distinct, increasing
             perm = torch.randperm(nq, generator=gn, device=device)[:n_probe]
             probes = sorted(int(x) for x in perm.tolist())
-            _plant(w, q[b], k[b], probes, gn)
+            planted = _plant(w, q[b], k[b], probes, gn)
         probes_all.append(probes)
+        needles_all.append(planted)
     gv = _gen(device, seed * 1000 + SUB_V)
     v = torch.empty(B, Hk, N, D, dtype=torch.bfloat16, device=device)
     for b in range(B):
@@ -196,7 +204,7 @@ def make_inputs(w: Workload, device="cpu", seed: Optional[int] = None,
             g = _gen(device, seed * 1000 + SUB_QS + layer)
             q_sparse.append((torch.randn(B, Hq, nq, D, generator=g, device=device) * 0.5)
                             .to(torch.bfloat16))
-    return dict(q=q, k=k, v=v, q_sparse=q_sparse, probes=probes_all)
+    return dict(q=q, k=k, v=v, q_sparse=q_sparse, probes=probes_all, needles=needles_all)
 
 
 def make_bridge_inputs(batch: int, n_new: int, d_model: int, h_kv: int, head_dim: int, device="cpu",
