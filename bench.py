@@ -85,8 +85,26 @@ def kernel_work(w: wl.Workload):
         # and takes one 2^x per (candidate, head): the special-function unit's ex2 rate is
         # the binding limit ("alu"); the tensor-core fraction is reported beside it
         G = w.h_q // w.h_kv
-        work["select_filter"] = dict(bound="alu", ex2=G * cand, flops=f["select_qk_flops"])
+        work["select_filter"] = dict(bound="alu", ex2=G * cand, flops=f["select_qk_flops"],
+                                     stream_bytes=select_stream_bytes(w))
     return work
+
+
+def select_stream_bytes(w: wl.Workload) -> float:
+    """Bytes the filtered sweep streams per call: every CTA (32 queries of one KV
+    group) reads the K rows of its candidate tiles (128 keys each) once, plus the
+    queries, the LSE and the written selection.  The fraction of HBM bandwidth
+    this gives is the one usually quoted for a select pass; most of
+    the K reads are L2 hits, and the binding unit is the ex2 rate."""
+    D = w.head_dim
+    tiles = 0
+    for q0 in range(0, w.n_q, 32):
+        t_max = w.q_pos0 + min(q0 + 32, w.n_q) - 1
+        cand_end = t_max - w.window + 1
+        tiles += max(0, -(-cand_end // 128))
+    k_bytes = tiles * 128 * D * 2 * w.h_kv * w.batch
+    f = wl.flops_and_bytes(w)
+    return float(k_bytes + f["q_bytes"] + 4.0 * w.batch * w.h_q * w.n_q + f["idx_bytes"])
 
 
 def measure_l2_gather(dev, reps: int = 10) -> float:
@@ -675,6 +693,8 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
                          achieved=round(achieved, 2), peak=peak, unit=unit, frac=round(achieved / peak, 4))
         if wk["bound"] == "alu" and "flops" in wk:  # the contraction's share of the tensor peak, for reference
             per[name]["tensor_frac"] = round(wk["flops"] * calls / (ms / 1e3) / 1e12 / pk["tc_sustained"], 4)
+        if "stream_bytes" in wk:  # the bytes it streams against HBM bandwidth, for reference
+            per[name]["hbm_frac"] = round(wk["stream_bytes"] * calls / (ms / 1e3) / 1e9 / pk["hbm"], 4)
     if not per:
         return None, per
     top = max((n for n in per if "bound" in per[n]), key=lambda n: per[n]["ms"])
