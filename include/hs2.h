@@ -96,8 +96,10 @@ enum {
 };
 
 /* Bytes of workspace the entry point `entry` needs for `shape` (0 if the shape
- * is invalid).  The first 256 bytes of every workspace hold the device error
- * word; hs2_workspace_init() must zero them once before first use. */
+ * is invalid, and 0 for the context-parallel slice entries, which
+ * hs2_cp_workspace_size sizes).  The first 256 bytes of every workspace hold
+ * the device error word; hs2_workspace_init() must zero them once before first
+ * use. */
 size_t hs2_workspace_size(const hs2_shape* shape, int entry);
 
 /* Zero the workspace header (error word) on `stream`.  Asynchronous. */
