@@ -162,7 +162,7 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
         !aligned(idx, 4) || !aligned(ws, 256) || (seq_len && !aligned(seq_len, 8)))
         return HS2_ERR_INVALID_ARG;
     const ScorePlan sp = score_plan(p, decode);
-    const size_t extra = decode ? decode_scratch_bytes(p) : 0;
+    const size_t extra = decode ? decode_scratch_bytes(p) + topk_chunk_bytes(p, sp.n_cand_max) : 0;
     const size_t body = decode ? (sp.bytes + 255) / 256 * 256 + extra : prefill_body_bytes(p, sp);
     if (ws_bytes < kHeader + body) return HS2_ERR_WORKSPACE;
     p.seq_len = seq_len;
@@ -176,7 +176,12 @@ hs2_status run_full_select(const hs2_shape* shape, const int64_t* seq_len, bool 
         cudaError_t e = launch_decode(p, q, k, v, out, lse, scratch, sel ? scores : nullptr, sp.sstride, st);
         if (e != cudaSuccess) return HS2_ERR_CUDA;
         if (p.topk == 0) return HS2_OK;
-        e = launch_topk(p, scores, sp.sstride, idx, 0, 1, st);
+        // the chunk lists of the selection sit after the decode attention's scratch
+        void* chunk = topk_chunk_bytes(p, sp.n_cand_max) > 0
+                          ? reinterpret_cast<uint8_t*>(scratch) + decode_scratch_bytes(p)
+                          : nullptr;
+        e = sel ? launch_topk_decode(p, scores, sp.sstride, sp.n_cand_max, idx, chunk, st)
+                : launch_topk(p, scores, sp.sstride, idx, 0, 1, st);
         return e == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
     }
     // the full layer's split parts (if any) use the selection scratch, which is
@@ -339,7 +344,8 @@ size_t hs2_workspace_size(const hs2_shape* shape, int entry) {
         case HS2_ENTRY_CP_SPARSE: return 0;  // slices: hs2_cp_workspace_size
         case HS2_ENTRY_DECODE: {
             if (p.nq != 1) return 0;
-            return kHeader + (score_plan(p, true).bytes + 255) / 256 * 256 + decode_scratch_bytes(p);
+            const ScorePlan sp = score_plan(p, true);
+            return kHeader + (sp.bytes + 255) / 256 * 256 + decode_scratch_bytes(p) + topk_chunk_bytes(p, sp.n_cand_max);
         }
         default: return 0;
     }

@@ -62,6 +62,12 @@ cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, 
 // K2 on tcgen05 for prefill-shaped calls: sampled threshold, filtered sweep
 // with on-chip survivor lists, exact final top-k, retry of underestimated rows.
 size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
+// Decode selection over few, long rows: each row cut into key chunks (each
+// chunk's exact top-K with scores on its own CTA, then a per-row merge);
+// chunk_scratch holds topk_chunk_bytes(p, n_cand_max) bytes (0: one CTA per row).
+size_t topk_chunk_bytes(const Problem& p, int64_t n_cand_max);
+cudaError_t launch_topk_decode(const Problem& p, const float* scores, int64_t sstride, int64_t n_cand_max,
+                               int32_t* idx, void* chunk_scratch, cudaStream_t st);
 // Block-level selection (blocks of `blk` in {32, 64, 128} keys): the chunk-sum
 // sweep over the tensor cores, then the per-row block top-k.  Scratch: the
 // chunk sums, block_tc_scratch_bytes(p, i_count, n_cand_max) bytes.

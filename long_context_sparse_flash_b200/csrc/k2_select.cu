@@ -206,7 +206,7 @@ __device__ __forceinline__ void digit_of(int pass, int& shift, uint32_t& mask) {
 // Exact top-k of one row over all n keys in global memory (the fallback):
 // 3-pass radix select for the k-th key, then an ordered pass, indices ascending.
 __device__ void topk_exact_global(const uint32_t* __restrict__ key, int n, int topk, int32_t* __restrict__ orow,
-                                  TopkSmem& sm) {
+                                  TopkSmem& sm, float* __restrict__ srow = nullptr) {
     const int tid = threadIdx.x, lane = tid & 31;
     const int n4 = n / 4;  // rows start 16-byte aligned (sstride is a multiple of 4)
     // radix select: the key value of the topk-th largest (non-negative floats
@@ -308,7 +308,10 @@ __device__ void topk_exact_global(const uint32_t* __restrict__ key, int n, int t
         uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-            if (take[u]) orow[pos++] = j0 + u;
+            if (take[u]) {
+                if (srow) srow[pos] = __uint_as_float(x[u]);
+                orow[pos++] = j0 + u;
+            }
         eq_seen += eq_tot;
         written += take_tot;
         __syncthreads();
@@ -376,6 +379,47 @@ __device__ void block_kth_shared(const uint32_t* keys, int n, uint32_t K, TopkSm
     need_eq = k_rem;
 }
 
+// Exact top K of the n (key, index) pairs in shared memory, which are in index
+// order: the K-th key, then one ordered pass that writes the indices of the keys
+// above it and of the first keys equal to it, ascending, to orow.
+__device__ void block_topk_ordered(const uint32_t* lk, const uint32_t* lj, int n, int topk, int32_t* orow,
+                                   TopkSmem& sm) {
+    const int tid = threadIdx.x;
+    uint32_t kth, need_eq;
+    block_kth_shared(lk, n, (uint32_t)topk, sm, kth, need_eq);
+    uint32_t eq_seen = 0, written = 0;
+    for (int base = 0; base < n; base += 4 * TK_THREADS) {
+        const int e0 = base + 4 * tid;
+        uint32_t x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) x[u] = (e0 + u < n) ? lk[e0 + u] : 0u;
+        uint32_t neq = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) neq += (e0 + u < n && x[u] == kth) ? 1u : 0u;
+        uint32_t eq_tot;
+        uint32_t eq_rank = eq_seen + block_excl_sum(neq, sm.warp_tot, eq_tot);
+        bool take[4];
+        uint32_t ntake = 0;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const bool valid = e0 + u < n;
+            const bool eq = valid && x[u] == kth;
+            take[u] = (valid && x[u] > kth) || (eq && eq_rank < need_eq);
+            eq_rank += eq ? 1u : 0u;
+            ntake += take[u] ? 1u : 0u;
+        }
+        __syncthreads();
+        uint32_t take_tot;
+        uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            if (take[u]) orow[pos++] = (int32_t)lj[e0 + u];
+        eq_seen += eq_tot;
+        written += take_tot;
+        __syncthreads();
+    }
+}
+
 // One row per CTA.  Fast path: a threshold tau from 8192 keys sampled at a
 // fixed stride (the r-th largest, r = L + 4.5 sqrt(L) + 2 with L = K s / n the
 // expected number of samples above the K-th best key; tau = 0 when n fits the
@@ -383,26 +427,41 @@ __device__ void block_kth_shared(const uint32_t* keys, int n, uint32_t K, TopkSm
 // order, into shared memory, then the exact select over those survivors.  A
 // row with fewer than K survivors (tau too high) or more than the buffer holds
 // (e.g. many equal scores) takes the exact passes over the whole row instead.
+//
+// Chunk mode (chunk_len > 0, one query per sequence): blockIdx.x is a chunk of
+// chunk_len candidates of the row; the CTA writes the chunk's exact top-min(K, n)
+// as LOCAL indices, ascending, with their scores, to cidx / cscore [row][chunk][K]
+// (-1 padded), and k2_chunk_merge_kernel gives the row's top K.
 __global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const float* __restrict__ scores,
                                                              int64_t sstride, int32_t* __restrict__ idx,
-                                                             int i_begin, int i_count) {
+                                                             int i_begin, int i_count, int64_t chunk_len,
+                                                             int32_t* __restrict__ cidx, float* __restrict__ cscore) {
     __shared__ TopkSmem sm;
     extern __shared__ __align__(16) uint32_t tk_dyn[];
     uint32_t* lk = tk_dyn;            // survivor keys (also the samples, before the compaction)
     uint32_t* lj = tk_dyn + TK_CAP;   // survivor indices
     const int tid = threadIdx.x;
-    const int qi = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const bool chunked = chunk_len > 0;
+    const int qi = chunked ? 0 : blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int i = i_begin + qi;
     const int64_t pos0 = seq_pos0(p, b, KID_TOPK);
     const int64_t t = pos0 + i;
     const int64_t n64 = t - p.window + 1;
-    const int n = n64 > 0 ? (int)n64 : 0;
-    int32_t* orow = idx + ((int64_t)(b * p.hkv + g) * p.nq + i) * p.topk;
+    const int64_t c0 = chunked ? (int64_t)blockIdx.x * chunk_len : 0;  // first candidate of the chunk
+    int64_t n_here = n64 - c0;
+    if (chunked && n_here > chunk_len) n_here = chunk_len;
+    const int n = n_here > 0 ? (int)n_here : 0;
+    const int64_t row = (int64_t)(b * p.hkv + g);
+    int32_t* orow = chunked ? cidx + (row * gridDim.x + blockIdx.x) * p.topk : idx + (row * p.nq + i) * p.topk;
+    float* srow = chunked ? cscore + (row * gridDim.x + blockIdx.x) * p.topk : nullptr;
+    const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + (row * i_count + qi) * sstride + c0);
     if (n <= p.topk) {
-        for (int r = tid; r < p.topk; r += TK_THREADS) orow[r] = r < n ? r : -1;
+        for (int r = tid; r < p.topk; r += TK_THREADS) {
+            orow[r] = r < n ? r : -1;
+            if (srow) srow[r] = r < n ? __uint_as_float(key[r]) : -1.f;
+        }
         return;
     }
-    const uint32_t* key = reinterpret_cast<const uint32_t*>(scores + ((int64_t)(b * p.hkv + g) * i_count + qi) * sstride);
 
     // threshold
     uint32_t tau = 0u;
@@ -457,44 +516,100 @@ __global__ void __launch_bounds__(TK_THREADS) k2_topk_kernel(Problem p, const fl
         __syncthreads();  // warp_tot is reused by the next step
     }
     if (cnt < (uint32_t)p.topk || cnt > (uint32_t)TK_CAP) {
-        topk_exact_global(key, n, p.topk, orow, sm);
+        topk_exact_global(key, n, p.topk, orow, sm, srow);
         return;
     }
 
     // exact top K among the survivors, then an ordered keep (they are in j order)
-    uint32_t kth, need_eq;
-    block_kth_shared(lk, (int)cnt, (uint32_t)p.topk, sm, kth, need_eq);
-    uint32_t eq_seen = 0, written = 0;
-    for (int base = 0; base < (int)cnt; base += 4 * TK_THREADS) {
-        const int e0 = base + 4 * tid;
-        uint32_t x[4];
+    if (srow) {  // chunk mode also records the kept keys' scores
+        uint32_t kth, need_eq;
+        block_kth_shared(lk, (int)cnt, (uint32_t)p.topk, sm, kth, need_eq);
+        __syncthreads();
+        uint32_t eq_seen = 0, written = 0;
+        for (int base = 0; base < (int)cnt; base += 4 * TK_THREADS) {
+            const int e0 = base + 4 * tid;
+            uint32_t x[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) x[u] = (e0 + u < (int)cnt) ? lk[e0 + u] : 0u;
-        uint32_t neq = 0;
+            for (int u = 0; u < 4; ++u) x[u] = (e0 + u < (int)cnt) ? lk[e0 + u] : 0u;
+            uint32_t neq = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) neq += (e0 + u < (int)cnt && x[u] == kth) ? 1u : 0u;
-        uint32_t eq_tot;
-        uint32_t eq_rank = eq_seen + block_excl_sum(neq, sm.warp_tot, eq_tot);
-        bool take[4];
-        uint32_t ntake = 0;
+            for (int u = 0; u < 4; ++u) neq += (e0 + u < (int)cnt && x[u] == kth) ? 1u : 0u;
+            uint32_t eq_tot;
+            uint32_t eq_rank = eq_seen + block_excl_sum(neq, sm.warp_tot, eq_tot);
+            bool take[4];
+            uint32_t ntake = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const bool valid = e0 + u < (int)cnt;
-            const bool eq = valid && x[u] == kth;
-            take[u] = (valid && x[u] > kth) || (eq && eq_rank < need_eq);
-            eq_rank += eq ? 1u : 0u;
-            ntake += take[u] ? 1u : 0u;
+            for (int u = 0; u < 4; ++u) {
+                const bool valid = e0 + u < (int)cnt;
+                const bool eq = valid && x[u] == kth;
+                take[u] = (valid && x[u] > kth) || (eq && eq_rank < need_eq);
+                eq_rank += eq ? 1u : 0u;
+                ntake += take[u] ? 1u : 0u;
+            }
+            __syncthreads();
+            uint32_t take_tot;
+            uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+                if (take[u]) {
+                    srow[pos] = __uint_as_float(x[u]);
+                    orow[pos++] = (int32_t)lj[e0 + u];
+                }
+            eq_seen += eq_tot;
+            written += take_tot;
+            __syncthreads();
         }
-        __syncthreads();
-        uint32_t take_tot;
-        uint32_t pos = written + block_excl_sum(ntake, sm.warp_tot2, take_tot);
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-            if (take[u]) orow[pos++] = (int32_t)lj[e0 + u];
-        eq_seen += eq_tot;
-        written += take_tot;
-        __syncthreads();
+        return;
     }
+    block_topk_ordered(lk, lj, (int)cnt, p.topk, orow, sm);
+}
+
+// The merge of a chunked row: one CTA per (sequence, group) row stages the
+// chunks' lists (each ascending, chunks in order, so the whole is ascending in
+// j) in shared memory as (score bits, j) and takes their exact top K, ties to
+// the lower j.  The row's top K lies in the union of the chunks' top Ks.
+__global__ void __launch_bounds__(TK_THREADS) k2_chunk_merge_kernel(Problem p, int n_chunks, int64_t chunk_len,
+                                                                    const int32_t* __restrict__ cidx,
+                                                                    const float* __restrict__ cscore,
+                                                                    int32_t* __restrict__ idx) {
+    __shared__ TopkSmem sm;
+    __shared__ uint32_t chunk_cnt[32];
+    extern __shared__ __align__(16) uint32_t mg_dyn[];
+    const int K = p.topk;
+    uint32_t* lk = mg_dyn;                      // [n_chunks * K] score bits
+    uint32_t* lj = mg_dyn + n_chunks * K;       // [n_chunks * K] rows
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t row = blockIdx.x;             // b * H_kv + g
+    int32_t* orow = idx + row * p.nq * K;       // one query per sequence
+    // valid entries of each chunk (a prefix: -1 after)
+    if (warp < n_chunks) {
+        const int32_t* ir = cidx + (row * n_chunks + warp) * K;
+        int c = 0;
+        for (int u = lane; u < K; u += 32) c += ir[u] >= 0;
+        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+        if (lane == 0) chunk_cnt[warp] = c;
+    }
+    __syncthreads();
+    int total = 0;
+    for (int c = 0; c < n_chunks; ++c) total += chunk_cnt[c];
+    // stage the chunks' entries contiguously, in chunk order
+    int base = 0;
+    for (int c = 0; c < n_chunks; ++c) {
+        const int cc = chunk_cnt[c];
+        const int32_t* ir = cidx + (row * n_chunks + c) * K;
+        const float* sr = cscore + (row * n_chunks + c) * K;
+        for (int u = tid; u < cc; u += TK_THREADS) {
+            lk[base + u] = __float_as_uint(sr[u]);
+            lj[base + u] = (uint32_t)(ir[u] + c * chunk_len);
+        }
+        base += cc;
+    }
+    __syncthreads();
+    if (total <= K) {
+        for (int u = tid; u < K; u += TK_THREADS) orow[u] = u < total ? (int32_t)lj[u] : -1;
+        return;
+    }
+    block_topk_ordered(lk, lj, total, K, orow, sm);
 }
 
 template <int D, int G>
@@ -553,7 +668,64 @@ cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, 
     if (e != cudaSuccess) return e;
     dim3 grid(i_count, p.hkv, p.B);
     prof_begin(KID_TOPK, st);
-    k2_topk_kernel<<<grid, TK_THREADS, TK_DYN_SMEM, st>>>(p, scores, sstride, idx, i_begin, i_count);
+    k2_topk_kernel<<<grid, TK_THREADS, TK_DYN_SMEM, st>>>(p, scores, sstride, idx, i_begin, i_count, 0, nullptr,
+                                                          nullptr);
+    prof_end(st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+// Decode rows (one query per sequence) that are too few to fill the SMs: each row
+// is cut into key chunks (about two CTAs per SM in all), then merged per row.
+void topk_chunk_geometry(const Problem& p, int64_t n_cand_max, int64_t& chunk_len, int& n_chunks) {
+    const int64_t rows = (int64_t)p.B * p.hkv;
+    chunk_len = 0;
+    n_chunks = 1;
+    if (p.nq != 1 || rows > 74 || n_cand_max < 4 * TK_CAP) return;
+    int want = (int)(2 * 148 / rows);
+    if (want > 16) want = 16;
+    if (want < 2) return;
+    int64_t len = (n_cand_max + want - 1) / want;
+    if (len < TK_CAP) len = TK_CAP;
+    len = (len + 3) / 4 * 4;  // chunks start on 16-byte boundaries of the score rows
+    const int nc = (int)((n_cand_max + len - 1) / len);
+    if (nc < 2) return;
+    chunk_len = len;
+    n_chunks = nc;
+}
+
+size_t topk_chunk_bytes(const Problem& p, int64_t n_cand_max) {
+    int64_t len;
+    int nc;
+    topk_chunk_geometry(p, n_cand_max, len, nc);
+    if (nc < 2) return 0;
+    return (size_t)nc * p.B * p.hkv * p.topk * 8 + 256;
+}
+
+cudaError_t launch_topk_decode(const Problem& p, const float* scores, int64_t sstride, int64_t n_cand_max,
+                               int32_t* idx, void* chunk_scratch, cudaStream_t st) {
+    int64_t len;
+    int nc;
+    topk_chunk_geometry(p, n_cand_max, len, nc);
+    if (nc < 2 || chunk_scratch == nullptr) return launch_topk(p, scores, sstride, idx, 0, 1, st);
+    cudaError_t e = cudaFuncSetAttribute(k2_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, TK_DYN_SMEM);
+    if (e != cudaSuccess) return e;
+    const int64_t rows = (int64_t)p.B * p.hkv;
+    int32_t* cidx = reinterpret_cast<int32_t*>(chunk_scratch);
+    float* cscore = reinterpret_cast<float*>(cidx + (size_t)nc * rows * p.topk);
+    prof_begin(KID_TOPK, st);
+    k2_topk_kernel<<<dim3(nc, p.hkv, p.B), TK_THREADS, TK_DYN_SMEM, st>>>(p, scores, sstride, idx, 0, 1, len, cidx,
+                                                                         cscore);
+    prof_end(st);
+    count_launch();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    const int smem = nc * p.topk * 8;  // at most 16 x 2048 x 8 = 256 KB: nc * topk <= 16384 is required
+    if (smem > 200 * 1024) return cudaErrorInvalidValue;
+    if ((e = cudaFuncSetAttribute(k2_chunk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem)) !=
+        cudaSuccess)
+        return e;
+    prof_begin(KID_TOPK, st);
+    k2_chunk_merge_kernel<<<(unsigned)rows, TK_THREADS, smem, st>>>(p, nc, len, cidx, cscore, idx);
     prof_end(st);
     count_launch();
     return cudaGetLastError();
