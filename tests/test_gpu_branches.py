@@ -113,3 +113,30 @@ def test_prefill_32k_branches_sampled():
     res = _run(w, inp, swa, idx)
     errs = _check_rows(w, inp, swa, idx, res, 0, wl.stratified_rows(w, 8))
     print("32k branches", errs)
+
+
+def test_checked_build_reports_invalid_selection_in_the_selected_branch():
+    """The checked build validates the selected branch's idx rows like the union
+    layer's: an index inside the window is reported through the error word."""
+    w = wl.custom("bad_branch_idx", n_q=64, q_pos0=500, h_q=8, h_kv=1, head_dim=64, window=32, topk=16, seed=2)
+    inp = wl.make_inputs(w, "cuda")
+    swa = wl.make_swa_cache(w, "cuda")
+    nv.load(True)
+    _, _, idx = nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk, q_pos0=w.q_pos0,
+                                    checked=True)
+    shape = nv.shape_of(inp["q"], inp["k"], window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_SPARSE, checked=True)
+    q = inp["q_sparse"][0]
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    l1 = torch.empty(q.shape[:3], dtype=torch.float32, device="cuda")
+    l2 = torch.empty_like(l1)
+    nv.hs2_swa_branches(shape, q, swa["k_swa"], swa["v_swa"], inp["k"], inp["v"], idx, o1, l1, o2, l2, ws,
+                        checked=True)
+    rc, info = nv.hs2_get_device_status(ws, checked=True)
+    assert rc == nv.HS2_OK, (rc, info)
+    bad = idx.clone()
+    bad[0, 0, 7, 2] = w.q_pos0 + 7  # the query itself: inside the window
+    nv.hs2_swa_branches(shape, q, swa["k_swa"], swa["v_swa"], inp["k"], inp["v"], bad, o1, l1, o2, l2, ws,
+                        checked=True)
+    rc, info = nv.hs2_get_device_status(ws, checked=True)
+    assert rc == 5 and info[1] == 4, (rc, info)

@@ -104,3 +104,23 @@ def test_merge_handles_rows_with_fewer_candidates_than_the_budget():
         n = max(0, t - w.window + 1)
         want = np.concatenate([np.arange(n), -np.ones(w.topk - n)]).astype(np.int32)
         assert np.array_equal(idx[0, :, i], np.broadcast_to(want, idx[0, :, i].shape)), f"row t={t}"
+
+
+def test_slice_steps_report_timeouts_and_checks_through_their_workspace():
+    """A slice call's workspace carries the error word: a valid run leaves it clear."""
+    w = wl.WORKLOADS["tiny"]
+    inp = wl.make_inputs(w, "cuda")
+    offs, ks, vs = cp.split_cache(inp["k"], inp["v"], 2)
+    shape = nv.shape_of(inp["q"], ks[1], window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = torch.empty(nv.hs2_cp_workspace_size(shape, offs[1], nv.HS2_ENTRY_CP_ATTN), dtype=torch.uint8,
+                     device="cuda")
+    nv.hs2_workspace_init(ws)
+    out = torch.empty_like(inp["q"])
+    lse = torch.empty(inp["q"].shape[:3], dtype=torch.float32, device="cuda")
+    nv.hs2_cp_attn_partial(shape, offs[1], inp["q"], ks[1], vs[1], out, lse, ws)
+    rc, info = nv.hs2_get_device_status(ws)
+    assert rc == nv.HS2_OK, (rc, info)
+    # queries before the slice have no key there: output 0, LSE -inf
+    first = offs[1] - w.q_pos0
+    assert torch.all(torch.isneginf(lse[:, :, :first])) and torch.all(out[:, :, :first] == 0)
+    assert torch.all(torch.isfinite(lse[:, :, first:]))
