@@ -342,16 +342,20 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
         bool ok = true;
         float s[PP_BN];
         for (int j = 0; j < n_tiles && ok; ++j) {
-            ok = tc::mbar_wait(bar(PB_SFULL + x), j & 1, ab, p.err, KID_FULL, 8);
+            // (votes keep each warp's tcgen05 loads converged on an aborted wait)
+            ok = __all_sync(~0u, tc::mbar_wait(bar(PB_SFULL + x), j & 1, ab, p.err, KID_FULL, 8));
             if (!ok) break;
             tc::fence_after_sync();
             const int64_t j0 = (int64_t)(jt0 + j) * PP_BN;
             load_scores(s_addr, s, j0 + PP_BN - 1 > t, j0, t);
             const float mt = tile_max(s) * p.scale_log2;
-            if (mt > m + 8.f) {
-                // the running max grew by more than 2^8: rescale l and O.  The
-                // commit behind S_X,j covers O_X += P_X,j-1 V_j-1, so O is final.
-                const float alpha = ex2(m - mt);
+            const bool grow = mt > m + 8.f;
+            if (__any_sync(0xffffffffu, grow)) {
+                // the running max of a row grew by more than 2^8: rescale its l
+                // and O.  tcgen05.ld / st are warp-collective, so the whole warp
+                // runs the O pass and the rows that keep their max scale by 1.
+                // The commit behind S_X,j covers O_X += P_X,j-1 V_j-1: O is final.
+                const float alpha = grow ? ex2(m - mt) : 1.f;
                 if (j > 0) {
                     float o[32];
 #pragma unroll
@@ -363,8 +367,10 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                         tc::tmem_st32(o_addr + c * 32, o);
                     }
                 }
-                l *= alpha;
-                m = mt;
+                if (grow) {
+                    l *= alpha;
+                    m = mt;
+                }
             }
             // (m stays -inf only while every key so far is masked, which a split
             // can start with: those exponentials are 0)
@@ -378,7 +384,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
         }
         // epilogue: O / l -> out (bf16), lse; with a split, the part's O / l (fp32)
         // and base-2 log-sum-exp for the merge
-        if (ok && n_tiles > 0) ok = tc::mbar_wait(bar(PB_ODONE + x), 0, ab, p.err, KID_FULL, 9);
+        if (ok && n_tiles > 0) ok = __all_sync(~0u, tc::mbar_wait(bar(PB_ODONE + x), 0, ab, p.err, KID_FULL, 9));
         if (ok && n_split > 1) {
             tc::fence_after_sync();
             const int i = i0 + x * PP_BM + r;

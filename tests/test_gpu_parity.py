@@ -253,3 +253,24 @@ def test_decode_shapes_every_sequence(name, kw):
     for b in range(w.batch):
         P.compare_rows(w, inp, gpu, b, np.array([0]), ts=np.array([w.kv_len - 1]))
     _row_properties(gpu["idx"], w)
+
+
+@pytest.mark.parametrize("head_dim,h_q,h_kv", [(128, 8, 1), (64, 8, 2)])
+def test_full_attention_rescale_of_single_rows(head_dim, h_q, h_kv):
+    """Keys far above every earlier logit of a few rows, several key tiles after
+    the first: those rows rescale their running output at that tile, and each
+    other row of their warps does or does not, at random (the spike key is a
+    large random direction for them).  The rescale of the output in tensor
+    memory is a warp-collective pass; every row must still match the oracle."""
+    w = wl.custom(f"spike_d{head_dim}", n_q=256, q_pos0=512, kv_len=768, h_q=h_q, h_kv=h_kv, head_dim=head_dim,
+                  window=128, topk=64, n_sparse=0, seed=5)
+    inp = wl.make_inputs(w, "cuda", with_sparse=False)
+    q, k = inp["q"], inp["k"]
+    G = h_q // h_kv
+    for r in (3, 45, 130, 250):
+        j = w.q_pos0 + r - 2  # a later key tile than the rows' first one, still causal for row r
+        for g in range(h_kv):
+            u = q[0, g * G:(g + 1) * G, r].float().sum(0)
+            k[0, g, j] = (160.0 * u / u.norm()).to(torch.bfloat16)
+    gpu = P.run_gpu(w, inp)
+    P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
