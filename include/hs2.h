@@ -319,7 +319,7 @@ uint64_t hs2_launch_count(void);
  * threshold estimate, 9 filtered selection sweep, 10 selection retry,
  * 11 KV bridging, 12 block-selection score sweep, 13 block top-k,
  * 14 context-parallel combine, 15 context-parallel selection merge,
- * 16 context-parallel selection slicing. */
+ * 16 context-parallel selection slicing, 17 the bounded-wait self-test. */
 hs2_status hs2_profile_start(void);
 hs2_status hs2_profile_stop(uint32_t n_kinds, float* total_ms, uint64_t* launches);
 
@@ -395,6 +395,19 @@ hs2_status hs2_gather_probe(const void* rows, int64_t n_rows, const int32_t* ord
  * times the call.  Requires iters >= 1 and non-null pointers, else
  * HS2_ERR_INVALID_ARG.  Not part of the method (no counterpart in the paper). */
 hs2_status hs2_ex2_probe(int32_t iters, float* sink, hs2_stream_t stream, int64_t* ex2_count);
+
+/* Diagnostics: the timeout path of the bounded device-side waits.  One CTA of
+ * four warps waits, on `stream`, on an mbarrier that nothing completes, with
+ * the same wait the tcgen05 kernels use but bounded by limit_cycles SM clock
+ * cycles (those kernels use 2^32).  The wait gives up, the CTA's abort flag
+ * releases the other warps, HS2_ERR_TIMEOUT is written into the error word of
+ * `ws` (kernel id 17, a = 1, b = the reporting block) and the kernel returns:
+ * hs2_get_device_status then reads HS2_ERR_TIMEOUT, and the context stays
+ * usable.  ws: a workspace of ws_bytes >= 256 bytes, 256-byte aligned, owned
+ * by the caller (its header is the error word; hs2_workspace_init clears it).
+ * Requires 1 <= limit_cycles <= 2^32, else HS2_ERR_INVALID_ARG.  Not part of
+ * the method (no counterpart in the paper). */
+hs2_status hs2_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, hs2_stream_t stream);
 
 /* 1 when the library was built with device-side input checks (HS2_CHECKED). */
 int hs2_is_checked_build(void);

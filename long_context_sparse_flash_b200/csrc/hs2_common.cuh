@@ -39,6 +39,7 @@ enum KernelId : uint32_t {
     KID_CP_COMBINE = 14,
     KID_CP_MERGE = 15,
     KID_CP_IDX = 16,
+    KID_SELFTEST_WAIT = 17,
 };
 
 __device__ __forceinline__ void report_error(WsHeader* h, uint32_t code, uint32_t kid, uint32_t a,

@@ -1,7 +1,9 @@
 // hs2_selftest.cu -- diagnostics: evaluate the library's exp2 implementations
-// on caller-given points, so tests can bound their error on the device.
+// on caller-given points, so tests can bound their error on the device; the
+// probes behind the rooflines; and the timeout path of the bounded waits.
 #include "exp2_poly.cuh"
 #include "hs2_kernels.h"
+#include "tc05.cuh"
 
 namespace hs2 {
 namespace {
@@ -107,5 +109,38 @@ extern "C" hs2_status hs2_ex2_probe(int32_t iters, float* sink, hs2_stream_t str
     hs2::ex2_probe_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(iters, sink);
     hs2::count_launch();
     *ex2_count = (int64_t)blocks * 256 * 8 * iters;
+    return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
+}
+
+namespace hs2 {
+namespace {
+// Four warps wait on an mbarrier that nothing arrives on, with the wait every
+// tcgen05 kernel uses (bounded by `limit` cycles instead of 2^32): the first
+// thread to run out raises the CTA's abort flag and writes HS2_ERR_TIMEOUT
+// (kernel 17, wait site 1) into the error word; the others see the flag.
+__global__ void __launch_bounds__(128) selftest_wait_kernel(WsHeader* err, long long limit) {
+    __shared__ __align__(8) uint64_t bar_s;
+    __shared__ tc::Abort ab;
+    const uint32_t bar = smem_u32(&bar_s);
+    if (threadIdx.x == 0) {
+        tc::mbar_init(bar, 1);
+        ab.flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    const bool ok = tc::mbar_wait(bar, 0, &ab, err, KID_SELFTEST_WAIT, 1, limit);
+    // every thread leaves through the failed wait; none arrives on the barrier
+    if (ok) report_error(err, HS2_ERR_DEVICE_CHECK, KID_SELFTEST_WAIT, 2, threadIdx.x);
+}
+}  // namespace
+}  // namespace hs2
+
+extern "C" hs2_status hs2_selftest_wait(void* ws, size_t ws_bytes, int64_t limit_cycles, hs2_stream_t stream) {
+    if (ws == nullptr || ws_bytes < sizeof(hs2::WsHeader) || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0 ||
+        limit_cycles < 1 || limit_cycles > (int64_t(1) << 32))
+        return HS2_ERR_INVALID_ARG;
+    hs2::selftest_wait_kernel<<<1, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        reinterpret_cast<hs2::WsHeader*>(ws), (long long)limit_cycles);
+    hs2::count_launch();
     return cudaGetLastError() == cudaSuccess ? HS2_OK : HS2_ERR_CUDA;
 }

@@ -60,13 +60,13 @@ struct Abort {
 // the CTA's abort flag and the device error word) if it does not complete
 // within kWaitCycles, or if another role of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, Abort* ab, WsHeader* err, uint32_t kid,
-                                          uint32_t where) {
+                                          uint32_t where, long long limit = kWaitCycles) {
     if (mbar_try(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_sleep(bar, parity)) return true;
         if (ab->flag) return false;
-        if (clock64() - t0 > kWaitCycles) {
+        if (clock64() - t0 > limit) {
             ab->flag = 1;
             report_error(err, HS2_ERR_TIMEOUT, kid, where, blockIdx.x);
             return false;

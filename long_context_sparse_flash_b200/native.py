@@ -32,12 +32,12 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
            "hs2_swa_branches", "hs2_cp_workspace_size", "hs2_cp_attn_partial", "hs2_cp_select_local",
            "hs2_cp_sparse_partial", "hs2_cp_combine", "hs2_cp_select_merge",
-           "hs2_kv_bridge_workspace_size")
+           "hs2_kv_bridge_workspace_size", "hs2_selftest_wait")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
                 10: "select_retry", 11: "kv_bridge", 12: "block_sweep", 13: "block_topk",
-                14: "cp_combine", 15: "cp_select_merge", 16: "cp_idx_local"}
+                14: "cp_combine", 15: "cp_select_merge", 16: "cp_idx_local", 17: "selftest_wait"}
 
 
 class HS2Error(RuntimeError):
@@ -109,6 +109,7 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     lib.hs2_gather_probe.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int32, P, P]
     lib.hs2_ex2_probe.argtypes = [ctypes.c_int32, P, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.hs2_selftest_wait.argtypes = [P, S, ctypes.c_int64, P]
     lib.hs2_kv_bridge.argtypes = [ctypes.POINTER(hs2_bridge_shape), P, P, P, P, P, P, S, P]
     lib.hs2_kv_bridge_workspace_size.argtypes = [ctypes.POINTER(hs2_bridge_shape)]
     lib.hs2_kv_bridge_workspace_size.restype = S
@@ -297,6 +298,12 @@ def hs2_ex2_probe(iters: int, sink: torch.Tensor, stream=None) -> int:
     n = ctypes.c_int64(0)
     _check(load().hs2_ex2_probe(int(iters), _ptr(sink), _stream(stream), ctypes.byref(n)), "hs2_ex2_probe")
     return int(n.value)
+
+
+def hs2_selftest_wait(ws: torch.Tensor, limit_cycles: int, stream=None, checked=False) -> None:
+    """The bounded-wait self-test: its timeout lands in the error word of ws."""
+    _check(load(checked).hs2_selftest_wait(_ptr(ws), ws.numel() * ws.element_size(), int(limit_cycles),
+                                           _stream(stream)), "hs2_selftest_wait")
 
 
 def hs2_kv_bridge(shape: hs2_bridge_shape, seq_pos, hidden, w_kv, k_cache, v_cache, ws=None, stream=None,

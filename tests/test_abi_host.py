@@ -115,6 +115,20 @@ def test_pointer_and_workspace_checks():
     assert L.hs2_full_attn_select(ctypes.byref(s2), *args, need, None) == 1
 
 
+def test_selftest_wait_argument_checks():
+    """The bounded-wait self-test validates its workspace and bound on the host,
+    before any launch."""
+    L = nv.load()
+    before = nv.hs2_launch_count()
+    ws = ctypes.c_void_p(1 << 40)  # 256-byte aligned fake device address
+    assert L.hs2_selftest_wait(None, 256, 1 << 20, None) == 1
+    assert L.hs2_selftest_wait(ws, 255, 1 << 20, None) == 1
+    assert L.hs2_selftest_wait(ctypes.c_void_p((1 << 40) + 16), 256, 1 << 20, None) == 1
+    assert L.hs2_selftest_wait(ws, 256, 0, None) == 1
+    assert L.hs2_selftest_wait(ws, 256, (1 << 32) + 1, None) == 1
+    assert nv.hs2_launch_count() == before
+
+
 def test_empty_calls_are_noops():
     L = nv.load()
     before = nv.hs2_launch_count()
