@@ -274,3 +274,37 @@ def test_full_attention_rescale_of_single_rows(head_dim, h_q, h_kv):
             k[0, g, j] = (160.0 * u / u.norm()).to(torch.bfloat16)
     gpu = P.run_gpu(w, inp)
     P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+
+
+def _check_selection_and_scores(g_idx, g_score, ores, ts, w, what):
+    """g_idx, g_score [n_rows, H_kv, K] from the selection pass; the selected
+    sets against the oracle's (near-tie rule) and the score the pass returns for
+    each selected row against the oracle's score of that row."""
+    P.check_idx(g_idx, ores, ts, w.window, w.topk, what)
+    for r, t in enumerate(ts):
+        n_sel = min(w.topk, max(0, int(t) - w.window + 1))
+        for g in range(g_idx.shape[1]):
+            sel = g_idx[r, g, :n_sel]
+            want = ores["scores"][r, g, sel]
+            got = g_score[r, g, :n_sel].astype(np.float64)
+            assert np.all(np.abs(got - want) <= 1e-9 + 1e-4 * np.abs(want)), f"{what} row t={t} g={g}: scores"
+
+
+def test_selection_pass_fed_the_oracle_lse():
+    """The selection pass alone (the slice step of context parallelism over the
+    whole cache), fed the oracle's LSE instead of the full-attention kernel's:
+    isolates the selection kernel from the LSE the first kernel computes."""
+    from long_context_sparse_flash_b200 import cp
+    w = wl.custom("k2_oracle_lse", n_q=600, q_pos0=1400, h_q=16, h_kv=2, head_dim=128, window=128, topk=256,
+                  n_sparse=0, seed=9)
+    inp = wl.make_inputs(w, "cuda", with_sparse=False)
+    ts = w.q_pos0 + np.arange(w.n_q)
+    qb = np.ascontiguousarray(P.bits(inp["q"][0]).transpose(1, 0, 2))
+    ores = oracle.full_select(qb, ts, P.bits(inp["k"][0]), P.bits(inp["v"][0]), window=w.window, topk=w.topk,
+                              want_scores=True)
+    lse = torch.as_tensor(np.ascontiguousarray(ores["lse"].T[None]).astype(np.float32), device="cuda")
+    idx, score = cp.select_local(inp["q"], inp["k"], lse, kv_off=0, window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    torch.cuda.synchronize()
+    g_idx = np.ascontiguousarray(idx[0].cpu().numpy().transpose(1, 0, 2))
+    g_score = np.ascontiguousarray(score[0].cpu().numpy().transpose(1, 0, 2))
+    _check_selection_and_scores(g_idx, g_score, ores, ts, w, "selection on the oracle LSE")
