@@ -806,8 +806,11 @@ def run_ours(args):
                         "max": round(max(ms), 4)},
         }
         print(json.dumps(line), flush=True)
+    else:
+        line = None
     if ws > 1:
         torch.distributed.destroy_process_group()
+    return line
 
 
 def run_reference(args):
@@ -842,6 +845,39 @@ def run_reference(args):
         "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+    return line
+
+
+def git_sha() -> str:
+    """The commit the run measured (or "unknown" outside a git checkout)."""
+    import subprocess
+    try:
+        r = subprocess.run(["git", "-C", ROOT, "rev-parse", "--short=12", "HEAD"], capture_output=True, text=True,
+                           timeout=10)
+        return r.stdout.strip() or "unknown"
+    except Exception:
+        return "unknown"
+
+
+def run_key(args, sha: str) -> dict:
+    """What identifies one bench entry in a JSONL log (a rerun with the same key is skipped)."""
+    return {"impl": args.impl, "workload": args.workload, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "git_sha": sha}
+
+
+def logged_line(path: str, key: dict):
+    """The logged line with this key, or None (unreadable lines are ignored)."""
+    if not path or not os.path.exists(path):
+        return None
+    with open(path) as f:
+        for raw in f:
+            try:
+                d = json.loads(raw)
+            except ValueError:
+                continue
+            if d.get("log_key") == key:
+                return d
+    return None
 
 
 def main():
@@ -858,13 +894,26 @@ def main():
                          "context parallelism) that run after the timed steps")
     ap.add_argument("--cpu-rows", type=int, default=1536, help="query rows in the oracle baseline sample (about 10 s of host work)")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference-arm step")
+    ap.add_argument("--log", default="", help="append the JSON line, with the git commit and its key, to this "
+                                                 "JSONL file (rank 0)")
+    ap.add_argument("--skip-logged", action="store_true",
+                    help="with --log: if the log already holds this entry (impl, workload, GPUs, steps, warm-up, "
+                         "commit), print that line and run nothing, so a killed sweep resumes where it stopped")
     args = ap.parse_args()
+    sha = git_sha() if args.log else None
+    key = run_key(args, sha) if args.log else None
+    if args.log and args.skip_logged:
+        done = logged_line(args.log, key)
+        if done is not None:
+            if int(os.environ.get("RANK", "0")) == 0:
+                print(json.dumps({k: v for k, v in done.items() if k not in ("log_key", "logged_at")}), flush=True)
+            return
     if args.warmup < 3 and args.impl == "ours":
         print("note: fewer than 3 warm-up steps", file=sys.stderr)
-    if args.impl == "reference":
-        run_reference(args)
-    else:
-        run_ours(args)
+    line = run_reference(args) if args.impl == "reference" else run_ours(args)
+    if args.log and line is not None:
+        with open(args.log, "a") as f:
+            f.write(json.dumps({**line, "log_key": key, "logged_at": round(time.time(), 1)}) + "\n")
 
 
 if __name__ == "__main__":

@@ -66,3 +66,45 @@ def test_reference_arm_runs_on_rank_zero_only(monkeypatch, capsys):
     args = argparse.Namespace(workload="tiny", ref_rows=1, warmup=3, steps=2, gpus=2)
     assert bench.run_reference(args) is None
     assert capsys.readouterr().out == ""
+
+
+def _failing_rank_main(rank: int, ws: int, port: int, q):
+    """Rank 1 leaves between steps (an exception before the timing collective);
+    rank 0 learns of it when its next collective ends with an error within the
+    process group's short timeout, instead of waiting for good."""
+    import datetime
+    import time
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(ws))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=ws, timeout=datetime.timedelta(seconds=5))
+    import bench
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        q.close()
+        q.join_thread()  # the message is sent before the process vanishes
+        os._exit(3)  # no destroy, no further collective: the rank is gone
+    t0 = time.time()
+    try:
+        bench.max_over_ranks(10.0, ws)
+        q.put((rank, "no error", time.time() - t0))
+    except Exception as e:  # gloo reports the lost peer or the timeout
+        q.put((rank, type(e).__name__, time.time() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_a_rank_that_leaves_ends_the_others_collective_with_an_error():
+    ws, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_failing_rank_main, args=(r, ws, port, q)) for r in range(ws)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert [p.exitcode for p in procs] == [0, 3]
+    res = dict((r[0], r[1:]) for r in (q.get(timeout=5) for _ in range(ws)))
+    assert res[1][0] == "left"
+    assert res[0][0] != "no error", res
+    assert res[0][1] < 60.0, res  # ended by the short timeout or the lost connection, not a hang
