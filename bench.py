@@ -58,19 +58,32 @@ def peaks():
 # algorithmic work per kernel (per call of the entry point, all sequences)
 
 
-def kernel_work(w: wl.Workload):
-    """Algorithmic work of each kernel per call (all sequences of the call)."""
+def kernel_work(w: wl.Workload, unique_rows: Optional[float] = None):
+    """Algorithmic work of each kernel per call (all sequences of the call).
+
+    unique_rows: distinct K/V rows the sparse layer touches per call (summed over
+    sequences and KV heads: the union of every query's selected rows and window),
+    counted from the step's selection; it gives the sparse layer's compulsory
+    HBM bytes."""
     f = wl.flops_and_bytes(w)
     Hq = w.h_q
     n_rows = w.batch * w.n_q
     cand = f["cand"]  # sum over (sequence, query, KV head) of candidate counts
+    io = 2 * f["q_bytes"] + f["idx_bytes"]
+    sparse = dict(bound="l2" if f["kv_bytes"] <= L2_RESIDENT_BYTES else "hbm",
+                  bytes=f["sparse_bytes_per_layer"] + io)
+    if unique_rows is not None:
+        # two roofs: the logical gather (every attended row of every query) against the
+        # random-row L2 gather peak, and the compulsory bytes (each distinct row once)
+        # against HBM bandwidth; the one nearer its roof binds
+        sparse = dict(bound="gather", bytes=f["sparse_bytes_per_layer"] + io,
+                      hbm_bytes=unique_rows * w.head_dim * 2 * 2 + io)
     work = {
         # dense causal contraction: QK^T and PV over the causal pairs
         "full_attn": dict(bound="tensor", flops=f["full_flops"]),
         "decode_attn": dict(bound="hbm", bytes=f["kv_bytes"] + 2 * f["q_bytes"] + 4 * n_rows * Hq),
         # gathered K/V rows + q + out + idx, per layer
-        "sparse_attn": dict(bound="l2" if f["kv_bytes"] <= L2_RESIDENT_BYTES else "hbm",
-                            bytes=f["sparse_bytes_per_layer"] + 2 * f["q_bytes"] + f["idx_bytes"]),
+        "sparse_attn": sparse,
     }
     if w.decode:
         # decode: the attention pass stores each candidate's G scaled logits (fp32); the score
@@ -88,6 +101,24 @@ def kernel_work(w: wl.Workload):
         work["select_filter"] = dict(bound="alu", ex2=G * cand, flops=f["select_qk_flops"],
                                      stream_bytes=select_stream_bytes(w))
     return work
+
+
+def unique_kv_rows(w: wl.Workload, idx: torch.Tensor) -> float:
+    """Distinct K/V rows one sparse layer reads: per (sequence, KV head), the
+    union over the call's queries of the selected rows and the window."""
+    B, H, nq, K = idx.shape
+    total = 0
+    for b in range(B):
+        # padding (-1) goes to an extra column that is dropped
+        mask = torch.zeros(H, w.kv_len + 1, dtype=torch.bool, device=idx.device)
+        sel = idx[b].reshape(H, -1).long()
+        mask.scatter_(1, torch.where(sel >= 0, sel, w.kv_len), True)
+        mask = mask[:, :w.kv_len]
+        t_lo = (w.kv_len - 1) if w.decode else w.q_pos0
+        t_hi = (w.kv_len - 1) if w.decode else w.q_pos0 + nq - 1
+        mask[:, max(0, t_lo - w.window + 1):t_hi + 1] = True
+        total += int(mask.sum().item())
+    return float(total)
 
 
 def select_stream_bytes(w: wl.Workload) -> float:
@@ -668,8 +699,8 @@ def cpu_baseline(w: wl.Workload, inp: dict, n_rows: int, seed: int = 2024) -> di
             "_rows": n, "_seconds": dt}
 
 
-def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
-    work = kernel_work(w)
+def roofline(w: wl.Workload, prof: dict, K: int, pk: dict, unique_rows: Optional[float] = None):
+    work = kernel_work(w, unique_rows)
     per = {}
     for name, (ms, launches) in prof.items():
         if name not in work or ms <= 0:
@@ -686,6 +717,20 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
         elif wk["bound"] == "alu":
             achieved = wk["ex2"] * calls / (ms / 1e3) / 1e9
             peak, unit = round(pk["ex2"] / 1e9, 1), "Gex2/s"
+        elif wk["bound"] == "gather":
+            l2 = wk["bytes"] * calls / (ms / 1e3) / 1e9
+            hbm = wk["hbm_bytes"] * calls / (ms / 1e3) / 1e9
+            l2_frac, hbm_frac = l2 / pk["l2_gather"], hbm / pk["hbm"]
+            entry = dict(ms=ms / K, launches=launches // K if K else launches,
+                         l2=dict(achieved=round(l2, 2), peak=round(pk["l2_gather"], 1), unit="GB/s",
+                                 frac=round(l2_frac, 4), bytes="every attended row of every query"),
+                         hbm=dict(achieved=round(hbm, 2), peak=pk["hbm"], unit="GB/s", frac=round(hbm_frac, 4),
+                                  bytes="each distinct row once (compulsory)"))
+            b = "l2" if l2_frac >= hbm_frac else "hbm"
+            entry.update(bound=b, achieved=entry[b]["achieved"], peak=entry[b]["peak"], unit="GB/s",
+                         frac=entry[b]["frac"])
+            per[name] = entry
+            continue
         else:
             achieved = wk["bytes"] * calls / (ms / 1e3) / 1e9
             peak, unit = pk["hbm"], "GB/s"
@@ -701,6 +746,11 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
     p = per[top]
     launches_total = prof[top][1]
     traffic = dram_traffic(top, w.name)
+    for name, e in per.items():  # measured DRAM bytes of the kernel (ncu), where current
+        tb = dram_traffic(name, w.name)
+        if tb is not None and e.get("ms"):
+            e["dram_bytes_per_launch"] = tb
+            e["dram_frac"] = round(tb / (e["ms"] / max(1, e["launches"]) / 1e3) / 1e9 / pk["hbm"], 4)
     src = {"tensor": pk["src"] + " (sustained bf16)", "hbm": pk["src"] + " (copy GB/s)",
            "l2": "measured here (random 256-byte-row gather from a 64 MiB L2-resident buffer, hs2_gather_probe)",
            "alu": "measured here (special-function-unit ex2 rate, hs2_ex2_probe)"}
@@ -712,18 +762,25 @@ def roofline(w: wl.Workload, prof: dict, K: int, pk: dict):
     return rf, per
 
 
-def run_ours(args):
-    ws, rank, local = dist_setup(args.gpus)
-    dev = torch.device("cuda", torch.cuda.current_device())
-    w = wl.WORKLOADS[args.workload]
-    nv.load()
-    # the L2 gather peak is taken first, on an idle GPU (a burst figure, like
-    # the other measured peaks), before the workload's tensors exist
-    l2_gather = measure_l2_gather(dev) if any(wk["bound"] == "l2" for wk in kernel_work(w).values()) else None
-    ex2_rate = measure_ex2(dev) if any(wk["bound"] == "alu" for wk in kernel_work(w).values()) else None
+# the 1M-context configuration is one 4096-token prefill chunk and one batch-8
+# decode step over independent 1M contexts: the chunk is the line's `value`,
+# the decode step is measured in the same run and reported beside it
+COMPANION = {"chunk_1m": "decode_1m"}
+
+
+def default_cpu_rows(w: wl.Workload) -> int:
+    """Oracle rows of the CPU baseline: about 12 s of host work on 16 cores
+    (1536 rows at a 16K mean context), scaled by the workload's mean context."""
+    return max(8, int(1536 * 16384 / wl.mean_context(w)))
+
+
+def measure(w: wl.Workload, args, ws: int, rank: int, local: int, dev, pk: dict, flush: torch.Tensor,
+            extras: bool) -> dict:
+    """Time `args.steps` steps of workload w (after `args.warmup` untimed ones),
+    L2 flushed before each; per-kernel times from the library's event pairs;
+    with `extras`, also the warm-L2 figure, e2e, next rows and the CPU baseline."""
     inp = wl.make_inputs(w, dev, seed=replica_seed(w, rank))  # independent replica per rank
     step = Step(w, inp, dev)
-    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     for _ in range(args.warmup):
         flush.zero_()
         step()
@@ -741,51 +798,79 @@ def run_ours(args):
     launches = nv.hs2_launch_count() - l0
     clk = clocks.stop()
     total_ms = max_over_ranks(float(sum(ms)), ws)
-    ms_per_step = total_ms / args.steps
-    tokens = w.query_tokens * ws * args.steps
     value = job_value(w.query_tokens, ws, args.steps, total_ms)
+    rf, per_kernel = roofline(w, prof, args.steps, pk, unique_kv_rows(w, step.idx) if w.topk else None)
+    if rf is not None:
+        rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
+    res = {"workload": w.name, "value": round(value, 2), "ms_per_step": round(total_ms / args.steps, 4),
+           "per_kernel": per_kernel, "roofline": rf, "gpu_launches": launches, "clocks": clk,
+           "step_ms": {"median": round(statistics.median(ms), 4), "min": round(min(ms), 4),
+                       "max": round(max(ms), 4)},
+           "inputs_sha256_64MiB": input_digests(inp)}
+    if not extras:
+        del step, inp
+        return res
 
     # the same steps with L2 left warm between them (a second figure, not `value`)
     warm_ms = max_over_ranks(float(sum(time_steps(step, args.steps, None, ws))), ws)
-    warm = {"ms_per_step": round(warm_ms / args.steps, 4),
-            "value": round(job_value(w.query_tokens, ws, args.steps, warm_ms), 2)}
-
-    e2e = None
+    res["warm_l2"] = {"ms_per_step": round(warm_ms / args.steps, 4),
+                      "value": round(job_value(w.query_tokens, ws, args.steps, warm_ms), 2)}
+    res["e2e"] = None
     if not args.no_e2e:
+        tokens = w.query_tokens * ws * args.steps
         e_ms, bi, bo = time_e2e(step, args.steps, ws, inp, dev)
         e_total = max_over_ranks(float(e_ms), ws)
-        e2e = {"value": round(tokens / (e_total / 1e3), 2), "unit": UNIT, "h2d_bytes_per_step": bi,
-               "d2h_bytes_per_step": bo, "ms_per_step": round(e_total / args.steps, 3)}
-
-    pk = peaks()
-    pk["l2_gather"] = l2_gather
-    pk["ex2"] = ex2_rate
-    rf, per_kernel = roofline(w, prof, args.steps, pk)
-    next_rows = None
+        res["e2e"] = {"value": round(tokens / (e_total / 1e3), 2), "unit": UNIT, "h2d_bytes_per_step": bi,
+                      "d2h_bytes_per_step": bo, "ms_per_step": round(e_total / args.steps, 3)}
+    res["next_rows"] = None
     if not args.no_next_rows:
-        next_rows = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
+        nr = {"kv_bridge": bench_bridge(w, dev, args.steps, args.warmup, pk)}
         sel_kernels = ("select_score", "select_thresh", "select_filter", "select_retry", "select_topk")
         token_sel_ms = sum(per_kernel[n]["ms"] for n in sel_kernels if n in per_kernel)
         blk = bench_block_select(w, inp, dev, args.steps, args.warmup, pk, flush, token_sel_ms)
         if blk is not None:
-            next_rows["block_select"] = blk
-        next_rows["swa_comparator"] = bench_swa_comparator(w, inp, dev, args.steps, args.warmup, flush, step.idx)
+            nr["block_select"] = blk
+        nr["swa_comparator"] = bench_swa_comparator(w, inp, dev, args.steps, args.warmup, flush, step.idx)
         cpr = bench_context_parallel(w, inp, dev, args.steps, args.warmup, flush)
         if cpr is not None:
-            next_rows["context_parallel"] = cpr
-    if rf is not None:
-        rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
-
-    cpu = None
+            nr["context_parallel"] = cpr
+        res["next_rows"] = nr
+    res["cpu_baseline"] = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp, args.cpu_rows)
+        rows = args.cpu_rows if args.cpu_rows else default_cpu_rows(w)
+        cpu = cpu_baseline(w, inp, rows)
         cpu.pop("_rows"), cpu.pop("_seconds")
         cpu["value"] = round(cpu["value"], 4)
+        res["cpu_baseline"] = cpu
+    del step, inp
+    return res
+
+
+def run_ours(args):
+    ws, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = wl.WORKLOADS[args.workload]
+    comp = None if args.no_companion else COMPANION.get(w.name)
+    nv.load()
+    kinds = {wk["bound"] for x in [w] + ([wl.WORKLOADS[comp]] if comp else []) for wk in kernel_work(x, 0.0).values()}
+    # the L2 gather and ex2 peaks are taken first, on an idle GPU (burst figures,
+    # like the other measured peaks), before the workload's tensors exist
+    pk = peaks()
+    pk["l2_gather"] = measure_l2_gather(dev) if kinds & {"l2", "gather"} else None
+    pk["ex2"] = measure_ex2(dev) if "alu" in kinds else None
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    main_res = measure(w, args, ws, rank, local, dev, pk, flush, extras=True)
+    comp_res = None
+    if comp:
+        torch.cuda.empty_cache()
+        comp_res = measure(wl.WORKLOADS[comp], args, ws, rank, local, dev, pk, flush, extras=False)
+        comp_res["note"] = ("the other half of the 1M-context configuration, measured in the same run with the "
+                            "same steps, warm-up and L2 flush; not part of `value`")
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4), "higher_is_better": True,
+            "metric": METRIC, "value": main_res["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"], "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded, shapes and value distributions of the workload; no dataset)",
             "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "q_pos0": w.q_pos0,
@@ -793,18 +878,19 @@ def run_ours(args):
                        "window": w.window, "topk": w.topk, "sparse_layers": w.n_sparse,
                        "parallelism": f"replicas x{ws} (independent sequences per GPU)",
                        "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write, outside the events)"},
-            "per_kernel": per_kernel,
-            "roofline": rf,
-            "warm_l2": warm,
-            "inputs_sha256_64MiB": input_digests(inp),
-            "next_rows": next_rows,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches,
-            "clocks": clk,
-            "step_ms": {"median": round(statistics.median(ms), 4), "min": round(min(ms), 4),
-                        "max": round(max(ms), 4)},
+            "per_kernel": main_res["per_kernel"],
+            "roofline": main_res["roofline"],
+            "warm_l2": main_res["warm_l2"],
+            "inputs_sha256_64MiB": main_res["inputs_sha256_64MiB"],
+            "next_rows": main_res["next_rows"],
+            "cpu_baseline": main_res["cpu_baseline"],
+            "e2e": main_res["e2e"],
+            "gpu_launches": main_res["gpu_launches"],
+            "clocks": main_res["clocks"],
+            "step_ms": main_res["step_ms"],
         }
+        if comp_res is not None:
+            line[comp] = comp_res
         print(json.dumps(line), flush=True)
     else:
         line = None
@@ -886,13 +972,17 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="prefill_32k", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--workload", default="chunk_1m", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--no-companion", action="store_true",
+                    help="chunk_1m only: skip the batch-8 1M decode step measured beside the chunk")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="skip the next-row measurements (KV bridging, block selection, SWA comparator, "
                          "context parallelism) that run after the timed steps")
-    ap.add_argument("--cpu-rows", type=int, default=1536, help="query rows in the oracle baseline sample (about 10 s of host work)")
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="query rows in the oracle baseline sample (default: about 12 s of host work, "
+                         "1536 rows at a 16K mean context, scaled by the workload's mean context)")
     ap.add_argument("--ref-rows", type=int, default=8, help="query rows per reference-arm step")
     ap.add_argument("--log", default="", help="append the JSON line, with the git commit and its key, to this "
                                                  "JSONL file (rank 0)")

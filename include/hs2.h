@@ -35,7 +35,9 @@
  *
  * Ownership: the caller allocates and owns every buffer, including the
  * workspace; the library allocates no device memory and keeps no per-call
- * state.  Execution: every entry point validates its arguments on the host,
+ * state, with one exception: the static device array behind
+ * hs2_full_attn_select_static (HS2_STATIC_SCRATCH_BYTES, held on every GPU
+ * that loads the library until the process exits).  Execution: every entry point validates its arguments on the host,
  * returns an error status without launching anything if a check fails, and
  * otherwise enqueues its kernels on `stream` and returns at once (no host
  * synchronisation), except hs2_get_device_status which synchronises `stream`.
@@ -282,13 +284,16 @@ hs2_status hs2_decode_sparse(const hs2_shape* shape, const int64_t* kv_len_per_s
  * status hs2_full_attn_select would give.
  *
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress, with that device current); make that first call
- * before any stream capture.  Every call clears the error-word header of the
- * array on `stream` (the array keeps the previous call's contents), so a
- * device-side check failure of this entry point cannot be read back.  All
- * calls on a device share the one array: calls that overlap on the GPU (other
- * streams, or other host threads without ordering) race on it and corrupt
- * each other's selections; order them on one stream or serialise them. */
+ * (cudaGetSymbolAddress, with that device current) and keeps it for the life
+ * of the process; make that first call before any stream capture, and do not
+ * use this entry point across a cudaDeviceReset (or any teardown of the
+ * device's primary context): the kept address would then be stale.  Every
+ * call first clears the error-word header of the array on `stream` (the array
+ * keeps the previous call's contents); hs2_static_scratch_status reads what
+ * the last call reported.  All calls on a device share the one array: calls
+ * that overlap on the GPU (other streams, or other host threads without
+ * ordering) race on it and corrupt each other's selections; order them on one
+ * stream or serialise them. */
 hs2_status hs2_full_attn_select_static(const hs2_shape* shape, const void* q, const void* k,
                                        const void* v, void* out, float* lse, int32_t* idx,
                                        hs2_stream_t stream);
@@ -296,11 +301,32 @@ hs2_status hs2_full_attn_select_static(const hs2_shape* shape, const void* q, co
 /* HS2_STATIC_SCRATCH_BYTES, for callers that load the library dynamically. */
 size_t hs2_static_scratch_bytes(void);
 
+/* The device error word of the static array, as hs2_get_device_status reads a
+ * workspace's: synchronises `stream`, returns HS2_OK, HS2_ERR_DEVICE_CHECK or
+ * HS2_ERR_TIMEOUT for the last hs2_full_attn_select_static call on the
+ * current device (HS2_ERR_CUDA if a runtime call fails), fills info[0..4) if
+ * non-NULL, and clears the word.  Copies through host stack memory; allocates
+ * nothing.  Read it before the next static call, which clears the word. */
+hs2_status hs2_static_scratch_status(hs2_stream_t stream, uint32_t* info);
+
 /* Synchronise `stream`, read and clear the workspace error word.  Returns
  * HS2_OK, HS2_ERR_DEVICE_CHECK or HS2_ERR_TIMEOUT (or HS2_ERR_CUDA).  If
  * `info` is non-NULL it receives 4 words: code, kernel id, and two values
  * describing the first failure. */
 hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info);
+
+/* Diagnostics: how many selection rows of the last query chunk of the last
+ * hs2_full_attn_select / hs2_prefill_chunk call on this workspace ran the
+ * selection's retry pass.  The selection first estimates, per (query, KV head)
+ * row, a score bound that at least min(topk, candidates) candidates exceed,
+ * from a fixed-stride sample of the keys; a row where fewer candidates pass is
+ * marked and swept again with bound 0, which keeps the selection exact.  This
+ * reads those marks: synchronises `stream`, copies them from `ws` (the call's
+ * workspace, same shape) to host memory and writes their count to *n_rows (0
+ * for shapes whose selection takes no sample: few candidates, n_q < 16 or
+ * topk == 0).  Not part of the method (no counterpart in the paper). */
+hs2_status hs2_select_retry_rows(const hs2_shape* shape, const void* ws, size_t ws_bytes, hs2_stream_t stream,
+                                 int64_t* n_rows);
 
 /* Static description of a status code. */
 const char* hs2_status_string(hs2_status status);

@@ -603,6 +603,31 @@ hs2_status hs2_get_device_status(void* ws, hs2_stream_t stream, uint32_t* info) 
     return h[0] == 0 ? HS2_OK : HS2_ERR_DEVICE_CHECK;
 }
 
+hs2_status hs2_select_retry_rows(const hs2_shape* shape, const void* ws, size_t ws_bytes, hs2_stream_t stream,
+                                 int64_t* n_rows) {
+    Problem p;
+    hs2_status s = check_shape(shape, &p);
+    if (s != HS2_OK) return s;
+    if (n_rows == nullptr || ws == nullptr || !aligned(ws, 256)) return HS2_ERR_INVALID_ARG;
+    *n_rows = 0;
+    const ScorePlan sp = score_plan(p, false);
+    if (!sp.tc || p.topk == 0 || p.B == 0 || p.nq == 0) return HS2_OK;  // no sampled selection pass ran
+    if (ws_bytes < kHeader + prefill_body_bytes(p, sp)) return HS2_ERR_WORKSPACE;
+    const int i_last = (p.nq - 1) / sp.chunk * sp.chunk;  // first query of the last chunk
+    const int cnt = p.nq - i_last;
+    const size_t rows = (size_t)p.B * p.hkv * cnt;
+    const size_t off = kHeader + select_tc_status_offset(p, cnt, sp.n_cand_max);
+    std::vector<int32_t> mark(rows);
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return HS2_ERR_CUDA;
+    if (cudaMemcpy(mark.data(), reinterpret_cast<const uint8_t*>(ws) + off, rows * sizeof(int32_t),
+                   cudaMemcpyDeviceToHost) != cudaSuccess)
+        return HS2_ERR_CUDA;
+    int64_t n = 0;
+    for (int32_t m : mark) n += m != 0;
+    *n_rows = n;
+    return HS2_OK;
+}
+
 const char* hs2_status_string(hs2_status status) {
     switch (status) {
         case HS2_OK: return "ok";

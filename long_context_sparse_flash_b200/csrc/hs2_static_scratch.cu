@@ -63,3 +63,14 @@ extern "C" hs2_status hs2_full_attn_select_static(const hs2_shape* shape, const 
 }
 
 extern "C" size_t hs2_static_scratch_bytes(void) { return hs2::kStaticScratchBytes; }
+
+// The error word of the static array: what the last hs2_full_attn_select_static
+// call on this device reported (the next call clears it first).  Synchronises
+// the stream; copies the word to host memory on the stack and clears it;
+// allocates nothing.
+extern "C" hs2_status hs2_static_scratch_status(hs2_stream_t stream, uint32_t* info) {
+    void* scratch = nullptr;
+    const hs2_status s = hs2::scratch_address(&scratch);
+    if (s != HS2_OK) return s;
+    return hs2_get_device_status(scratch, stream, info);
+}

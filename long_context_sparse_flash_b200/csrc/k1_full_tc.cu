@@ -3,7 +3,7 @@
 // (xiawanshe.com report, section "两级KV共享": this layer's cache and its token
 // selection are reused by the following sparse layers).
 //
-// One CTA = two 128-row query tiles (A, B) of one head, 10 warps:
+// One CTA = two 128-row query tiles (A, B) of one head, 12 warps (384 threads):
 //   warps 0-3  softmax of tile A, warps 4-7 softmax of tile B: thread r of a
 //              warpgroup owns query row r of its tile = TMEM lane r
 //   warp 8     TMA producer: both Q tiles once, then K and V tiles of 128 keys

@@ -809,6 +809,13 @@ size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max
     return (size_t)n_slots * SL_QT * cmax * sizeof(uint2) + (size_t)rows * per_row;
 }
 
+size_t select_tc_status_offset(const Problem& p, int i_count, int64_t n_cand_max) {
+    int cmax, n_slots, by_block;
+    select_tc_geometry(p, i_count, n_cand_max, cmax, n_slots, by_block);
+    const int64_t rows = (int64_t)p.B * p.hkv * i_count;
+    return (size_t)n_slots * SL_QT * cmax * sizeof(uint2) + (size_t)rows * (SL_SPR * 4 + 2 * 4);
+}
+
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
                              void* scratch, int i_begin, int i_count, int64_t n_cand_max, cudaStream_t st,
                              float* sel_score) {

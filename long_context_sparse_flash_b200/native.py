@@ -32,7 +32,8 @@ EXPORTS = ("hs2_workspace_size", "hs2_workspace_init", "hs2_full_attn_select", "
            "hs2_gather_probe", "hs2_ex2_probe", "hs2_kv_bridge", "hs2_full_attn_block_select",
            "hs2_swa_branches", "hs2_cp_workspace_size", "hs2_cp_attn_partial", "hs2_cp_select_local",
            "hs2_cp_sparse_partial", "hs2_cp_combine", "hs2_cp_select_merge",
-           "hs2_kv_bridge_workspace_size", "hs2_selftest_wait")
+           "hs2_kv_bridge_workspace_size", "hs2_selftest_wait", "hs2_static_scratch_status",
+           "hs2_select_retry_rows")
 
 KERNEL_NAMES = {1: "full_attn", 2: "select_score", 3: "select_topk", 4: "sparse_attn", 5: "decode_attn",
                 6: "decode_combine", 7: "fused_attn_select", 8: "select_thresh", 9: "select_filter",
@@ -106,6 +107,10 @@ def load(checked: bool = False) -> ctypes.CDLL:
     lib.hs2_full_attn_select_static.argtypes = [sh, P, P, P, P, P, P, P]
     lib.hs2_static_scratch_bytes.argtypes = []
     lib.hs2_static_scratch_bytes.restype = S
+    lib.hs2_static_scratch_status.argtypes = [P, ctypes.POINTER(ctypes.c_uint32)]
+    lib.hs2_static_scratch_status.restype = ctypes.c_int
+    lib.hs2_select_retry_rows.argtypes = [sh, P, S, P, ctypes.POINTER(ctypes.c_int64)]
+    lib.hs2_select_retry_rows.restype = ctypes.c_int
     lib.hs2_selftest_exp2.argtypes = [P, P, ctypes.c_int, P]
     lib.hs2_gather_probe.argtypes = [P, ctypes.c_int64, P, ctypes.c_int64, ctypes.c_int32, P, P]
     lib.hs2_ex2_probe.argtypes = [ctypes.c_int32, P, P, ctypes.POINTER(ctypes.c_int64)]
@@ -275,6 +280,13 @@ def hs2_full_attn_select_static(shape, q, k, v, out, lse, idx, stream=None, chec
            "hs2_full_attn_select_static")
 
 
+def hs2_static_scratch_status(stream=None, checked=False):
+    """Returns (status, [code, kernel, a, b]) of the static array's error word; synchronises."""
+    info = (ctypes.c_uint32 * 4)()
+    rc = load(checked).hs2_static_scratch_status(_stream(stream), info)
+    return int(rc), list(info)
+
+
 def hs2_selftest_exp2(x: torch.Tensor, stream=None):
     """(hardware ex2, degree-3, degree-5, packed degree-5 at x, packed degree-5
     at x/2) evaluations of 2^x on the device."""
@@ -345,6 +357,15 @@ def hs2_get_device_status(ws: torch.Tensor, stream=None, checked=False):
     info = (ctypes.c_uint32 * 4)()
     rc = load(checked).hs2_get_device_status(_ptr(ws), _stream(stream), info)
     return int(rc), list(info)
+
+
+def hs2_select_retry_rows(shape, ws, stream=None, checked=False) -> int:
+    """Rows of the last query chunk of the last selection on `ws` that ran the retry pass."""
+    n = ctypes.c_int64(0)
+    wp, wn = _ws(ws)
+    _check(load(checked).hs2_select_retry_rows(ctypes.byref(shape), wp, wn, _stream(stream), ctypes.byref(n)),
+           "hs2_select_retry_rows")
+    return int(n.value)
 
 
 def hs2_status_string(status: int, checked=False) -> str:

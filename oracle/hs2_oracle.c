@@ -464,7 +464,10 @@ int hs2o_kv_bridge(int64_t n_rows, int d_model, int h_kv, int d, const uint16_t*
                    double* out_k, double* out_v, int n_threads) {
     if (n_rows < 0 || d_model <= 0 || h_kv <= 0 || d <= 0) return HS2O_EINVAL;
     const int64_t hd = (int64_t)h_kv * d;
-#pragma omp parallel for schedule(dynamic, 4) num_threads(n_threads > 0 ? n_threads : omp_get_max_threads())
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 4)
+#endif
     for (int64_t r = 0; r < n_rows; ++r) {
         const uint16_t* x = hidden + r * (int64_t)d_model;
         for (int64_t f = 0; f < 2 * hd; ++f) {

@@ -70,3 +70,39 @@ def test_roofline_assembly():
 def test_job_value_is_whole_job_tokens_over_the_slowest_rank():
     assert bench.job_value(1000, 4, 10, 2000.0) == pytest.approx(1000 * 4 * 10 / 2.0)
     assert math.isclose(bench.job_value(32768, 1, 10, 350.0), 32768 * 10 / 0.35)
+
+
+def test_sparse_layer_two_roofs():
+    """With the distinct rows known, the sparse layer carries two roofs: every
+    attended row against the L2 gather peak, each distinct row once against HBM;
+    the one nearer its roof is the reported bound."""
+    w = wl.WORKLOADS["chunk_1m"]
+    unique = 4 * 900_000.0
+    work = bench.kernel_work(w, unique)
+    f = wl.flops_and_bytes(w)
+    io = 2 * f["q_bytes"] + f["idx_bytes"]
+    assert work["sparse_attn"]["hbm_bytes"] == unique * 128 * 2 * 2 + io
+    assert work["sparse_attn"]["bytes"] == f["sparse_bytes_per_layer"] + io
+    K = 2
+    pk = dict(hbm=6552.0, tc=1590.0, tc_sustained=1403.2, src="measured", l2_gather=19000.0, ex2=4.6e12)
+    ms = 6.0  # 8 launches
+    rf, per = bench.roofline(w, {"sparse_attn": (ms, 8)}, K, pk, unique)
+    e = per["sparse_attn"]
+    l2 = work["sparse_attn"]["bytes"] * 8 / (ms / 1e3) / 1e9
+    hbm = work["sparse_attn"]["hbm_bytes"] * 8 / (ms / 1e3) / 1e9
+    assert e["l2"]["achieved"] == pytest.approx(l2, rel=1e-4)
+    assert e["hbm"]["achieved"] == pytest.approx(hbm, rel=1e-4)
+    want = "l2" if l2 / 19000.0 >= hbm / 6552.0 else "hbm"
+    assert e["bound"] == want and rf["bound"] == want
+    assert rf["frac"] == e[want]["frac"]
+
+
+def test_unique_rows_counts_the_union_of_selections_and_windows():
+    import torch
+    w = wl.custom("u", n_q=3, q_pos0=20, kv_len=23, h_q=2, h_kv=2, head_dim=64, window=4, topk=3)
+    idx = torch.full((1, 2, 3, 3), -1, dtype=torch.int32)
+    idx[0, 0, 0] = torch.tensor([0, 5, 9])
+    idx[0, 0, 1] = torch.tensor([5, 9, 16])   # 16 lies just below the windows' union [17, 22]
+    idx[0, 1, 2] = torch.tensor([1, -1, -1])
+    # windows: t in [20, 22] -> rows [17, 22] (6 rows) per head
+    assert bench.unique_kv_rows(w, idx) == (6 + 4) + (6 + 1)

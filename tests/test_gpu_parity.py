@@ -122,12 +122,12 @@ def test_chunk_256k_sampled():
     _row_properties(gpu["idx"], w)
 
 
-def test_decode_128k_sampled():
+def test_decode_128k_every_sequence():
     w = wl.WORKLOADS["decode_128k"]
     inp = wl.make_inputs(w, "cuda")
     gpu = P.run_gpu(w, inp)
     t = np.array([w.kv_len - 1])
-    for b in (0, 1, 17, 40, 63):
+    for b in range(w.batch):
         P.compare_rows(w, inp, gpu, b, np.array([0]), ts=t)
     _row_properties(gpu["idx"], w)
 
@@ -147,7 +147,7 @@ def test_chunk_1m_sampled():
     w = wl.WORKLOADS["chunk_1m"]
     inp = wl.make_inputs(w, "cuda")
     gpu = P.run_gpu(w, inp)
-    rows = wl.stratified_rows(w, 4)
+    rows = wl.stratified_rows(w, 32)
     res = P.compare_rows(w, inp, gpu, 0, rows)
     print("1m chunk", res["idx"], res["out_err"], res["sparse_err"])
     _row_properties(gpu["idx"], w)
@@ -308,3 +308,50 @@ def test_selection_pass_fed_the_oracle_lse():
     g_idx = np.ascontiguousarray(idx[0].cpu().numpy().transpose(1, 0, 2))
     g_score = np.ascontiguousarray(score[0].cpu().numpy().transpose(1, 0, 2))
     _check_selection_and_scores(g_idx, g_score, ores, ts, w, "selection on the oracle LSE")
+
+
+def test_overshooting_threshold_forces_the_retry_pass():
+    """The selection's retry pass, forced.  Every query carries a shared
+    per-group direction u_g, and the keys at the sampling stride (j = m S,
+    S = kv_len // 1024, the keys the threshold estimate is drawn from) are
+    strong plants along u_g.  The estimate is then the r-th best plant, far
+    above the K-th best candidate of every row: fewer than K candidates pass
+    the filtered sweep, every row is marked, and the retry pass re-sweeps it
+    with bound 0.  Every row must still match the oracle."""
+    w = wl.custom("retry", n_q=96, q_pos0=20000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=1, seed=12)
+    inp = wl.make_inputs(w, "cuda")
+    q, k = inp["q"], inp["k"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(77)
+    u = torch.randn(w.h_kv, w.head_dim, generator=gen, device="cuda")
+    u = u / u.norm(dim=-1, keepdim=True)
+    G = w.group
+    q_f = q.float().view(1, w.h_kv, G, w.n_q, w.head_dim) + 2.0 * u.view(1, w.h_kv, 1, 1, w.head_dim)
+    q.copy_(q_f.view_as(q).to(torch.bfloat16))
+    S = w.kv_len // 1024
+    pos = torch.arange(0, w.kv_len, S, device="cuda")
+    noise = torch.randn(w.h_kv, pos.numel(), w.head_dim, generator=gen, device="cuda")
+    k[0][:, pos, :] = (8.0 * u[:, None, :] + 0.1 * noise).to(torch.bfloat16)
+    shape = nv.shape_of(q, k, window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_FULL_SELECT)
+    out, lse, idx = nv.full_attn_select(q, k, inp["v"], window=w.window, topk=w.topk, q_pos0=w.q_pos0, ws=ws)
+    retried = nv.hs2_select_retry_rows(shape, ws)
+    assert retried == w.batch * w.h_kv * w.n_q, retried  # every row took the retry pass
+    sp = [nv.sparse_attn(qs, k, inp["v"], idx, window=w.window, q_pos0=w.q_pos0) for qs in inp["q_sparse"]]
+    torch.cuda.synchronize()
+    gpu = dict(out=out, lse=lse, idx=idx, sparse=sp)
+    P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+    _row_properties(idx, w)
+
+
+def test_ordinary_inputs_take_no_retry():
+    """The counterpart: on the needle workload's inputs the estimate holds and
+    no row is retried (the retry pass exists for inputs like the test above)."""
+    w = wl.custom("no_retry", n_q=96, q_pos0=20000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=0, needles=16, seed=12)
+    inp = wl.make_inputs(w, "cuda", with_sparse=False)
+    shape = nv.shape_of(inp["q"], inp["k"], window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_FULL_SELECT)
+    nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk, q_pos0=w.q_pos0, ws=ws)
+    assert nv.hs2_select_retry_rows(shape, ws) == 0

@@ -5,11 +5,14 @@ layer (a pre-sized memory pool they may not grow, a host runtime that hands
 them only input and output buffers, a step that must not synchronise the
 device).  Its scratch is a fixed static array inside the library; these tests
 check that, called through the C ABI, it gives the same outputs as
-hs2_full_attn_select with a caller-allocated workspace, on two calls in a row
-with different inputs, and that it refuses shapes whose scratch would not fit.
+hs2_full_attn_select with a caller-allocated workspace on two calls in a row
+with different inputs, that those outputs also match the fp64 oracle, that
+its error word reads clean afterwards, that a warm call leaves the device's
+free memory unchanged, and that it refuses shapes whose scratch would not fit.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
@@ -42,11 +45,23 @@ def test_static_scratch_entry_matches_allocating_entry():
         out = torch.full_like(q, float("nan"))
         lse = torch.full_like(ref_lse, float("nan"))
         idx = torch.full_like(ref_idx, -7)
+        torch.cuda.synchronize()
+        free_before = torch.cuda.mem_get_info()[0]
         assert _static_call(shape, q, k, v, out, lse, idx) == nv.HS2_OK
         torch.cuda.synchronize()
+        free_after = torch.cuda.mem_get_info()[0]
+        if call == 1:
+            # the first call may load the library's kernels (and its static
+            # array) onto the device; a warm call takes no device memory
+            assert free_after == free_before, (free_before, free_after)
+        rc, info = nv.hs2_static_scratch_status()
+        assert rc == nv.HS2_OK, (rc, info)
         P.assert_close(P.to_f64(out), P.to_f64(ref_out), f"call {call} out")
         P.assert_close(P.to_f64(lse), P.to_f64(ref_lse), f"call {call} lse", atol=P.LSE_ATOL, rtol=0.0)
         assert torch.equal(idx, ref_idx), f"call {call}: selection differs"
+        # and against the oracle itself, on rows around the window and top-k boundaries
+        gpu = dict(out=out, lse=lse, idx=idx, sparse=[])
+        P.compare_rows(w, inp, gpu, 0, np.array([0, 1, 127, 128, 300, 383, 384, 385, 600, 699]))
 
 
 def test_static_scratch_entry_rejects_oversized_shapes():
