@@ -12,11 +12,14 @@ query), over one batch of seeded synthetic input already resident in HBM.
 Prints ONE JSON line on rank 0.  Metric: query tokens/s through the whole
 step.  With N > 1 (torchrun), every rank runs an independent replica of the
 workload (its own sequences: weak scaling, no data-path collective); value =
-all ranks' query tokens / the slowest rank's time.
+all ranks' query tokens / the slowest rank's time.  With --split heads the
+ranks instead share one workload by KV-head group (strong scaling, still no
+exchange); value = its query tokens / the slowest rank's time.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -584,6 +587,24 @@ def job_value(query_tokens: int, ws: int, steps: int, total_ms: float) -> float:
     return query_tokens * ws * steps / (total_ms / 1e3)
 
 
+def head_shard(w: wl.Workload, inp: dict, rank: int, ws: int):
+    """Rank `rank`'s share of one workload split by KV-head group: KV heads
+    [rank H_kv / ws, (rank + 1) H_kv / ws) with the G query heads of each
+    (head h belongs to group h // G), copied into contiguous tensors, and the
+    workload of that share.  Every (query, group) is computed from its own
+    heads' q, K and V alone (full attention, selection and every sparse layer),
+    so the shares need no exchange."""
+    if w.h_kv % ws:
+        raise ValueError(f"{w.h_kv} KV heads do not split over {ws} ranks")
+    per, G = w.h_kv // ws, w.group
+    g0, g1 = rank * per, (rank + 1) * per
+    cut = lambda t, a, b: t[:, a:b].contiguous()
+    share = dict(q=cut(inp["q"], g0 * G, g1 * G), k=cut(inp["k"], g0, g1), v=cut(inp["v"], g0, g1),
+                 q_sparse=[cut(x, g0 * G, g1 * G) for x in inp["q_sparse"]],
+                 probes=inp.get("probes"), needles=inp.get("needles"))
+    return dataclasses.replace(w, h_q=per * G, h_kv=per), share
+
+
 def input_digests(inp: dict) -> dict:
     """SHA-256 (first 16 hex digits) of the first 64 MiB of each input tensor, for reproducibility."""
     def dig(t):
@@ -779,7 +800,16 @@ def measure(w: wl.Workload, args, ws: int, rank: int, local: int, dev, pk: dict,
     """Time `args.steps` steps of workload w (after `args.warmup` untimed ones),
     L2 flushed before each; per-kernel times from the library's event pairs;
     with `extras`, also the warm-L2 figure, e2e, next rows and the CPU baseline."""
-    inp = wl.make_inputs(w, dev, seed=replica_seed(w, rank))  # independent replica per rank
+    if args.split == "heads":
+        # one sequence (the same seed on every rank), its KV-head groups split over the ranks
+        full = wl.make_inputs(w, dev, seed=w.seed)
+        w_full, (w, inp) = w, head_shard(w, full, rank, ws)
+        del full
+        torch.cuda.empty_cache()
+        tokens_per_rank = 0  # every rank serves the same query tokens
+    else:
+        inp = wl.make_inputs(w, dev, seed=replica_seed(w, rank))  # independent replica per rank
+        w_full, tokens_per_rank = w, w.query_tokens
     step = Step(w, inp, dev)
     for _ in range(args.warmup):
         flush.zero_()
@@ -798,11 +828,13 @@ def measure(w: wl.Workload, args, ws: int, rank: int, local: int, dev, pk: dict,
     launches = nv.hs2_launch_count() - l0
     clk = clocks.stop()
     total_ms = max_over_ranks(float(sum(ms)), ws)
-    value = job_value(w.query_tokens, ws, args.steps, total_ms)
+    # replicas: all ranks' query tokens; head split: the one sequence's query tokens
+    job_tokens, job_ranks = (w.query_tokens, ws) if tokens_per_rank else (w_full.query_tokens, 1)
+    value = job_value(job_tokens, job_ranks, args.steps, total_ms)
     rf, per_kernel = roofline(w, prof, args.steps, pk, unique_kv_rows(w, step.idx) if w.topk else None)
     if rf is not None:
         rf["share_of_step"] = round(per_kernel[rf["kernel"]]["ms"] / (sum(ms) / args.steps), 4)
-    res = {"workload": w.name, "value": round(value, 2), "ms_per_step": round(total_ms / args.steps, 4),
+    res = {"workload": w_full.name, "value": round(value, 2), "ms_per_step": round(total_ms / args.steps, 4),
            "per_kernel": per_kernel, "roofline": rf, "gpu_launches": launches, "clocks": clk,
            "step_ms": {"median": round(statistics.median(ms), 4), "min": round(min(ms), 4),
                        "max": round(max(ms), 4)},
@@ -814,10 +846,10 @@ def measure(w: wl.Workload, args, ws: int, rank: int, local: int, dev, pk: dict,
     # the same steps with L2 left warm between them (a second figure, not `value`)
     warm_ms = max_over_ranks(float(sum(time_steps(step, args.steps, None, ws))), ws)
     res["warm_l2"] = {"ms_per_step": round(warm_ms / args.steps, 4),
-                      "value": round(job_value(w.query_tokens, ws, args.steps, warm_ms), 2)}
+                      "value": round(job_value(job_tokens, job_ranks, args.steps, warm_ms), 2)}
     res["e2e"] = None
     if not args.no_e2e:
-        tokens = w.query_tokens * ws * args.steps
+        tokens = job_tokens * job_ranks * args.steps
         e_ms, bi, bo = time_e2e(step, args.steps, ws, inp, dev)
         e_total = max_over_ranks(float(e_ms), ws)
         res["e2e"] = {"value": round(tokens / (e_total / 1e3), 2), "unit": UNIT, "h2d_bytes_per_step": bi,
@@ -851,6 +883,10 @@ def run_ours(args):
     dev = torch.device("cuda", torch.cuda.current_device())
     w = wl.WORKLOADS[args.workload]
     comp = None if args.no_companion else COMPANION.get(w.name)
+    if args.split == "heads":
+        for x in [w] + ([wl.WORKLOADS[comp]] if comp else []):
+            if x.h_kv % ws:
+                raise SystemExit(f"--split heads: {x.name} has {x.h_kv} KV heads, not divisible by {ws} ranks")
     nv.load()
     kinds = {wk["bound"] for x in [w] + ([wl.WORKLOADS[comp]] if comp else []) for wk in kernel_work(x, 0.0).values()}
     # the L2 gather and ex2 peaks are taken first, on an idle GPU (burst figures,
@@ -871,12 +907,14 @@ def run_ours(args):
         line = {
             "metric": METRIC, "value": main_res["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"], "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "strong" if args.split == "heads" else "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded, shapes and value distributions of the workload; no dataset)",
             "config": {"workload": w.name, "batch": w.batch, "n_q": w.n_q, "q_pos0": w.q_pos0,
                        "kv_len": w.kv_len, "h_q": w.h_q, "h_kv": w.h_kv, "head_dim": w.head_dim,
                        "window": w.window, "topk": w.topk, "sparse_layers": w.n_sparse,
-                       "parallelism": f"replicas x{ws} (independent sequences per GPU)",
+                       "parallelism": (f"heads x{ws} (the KV-head groups of one workload split over the GPUs, "
+                                       f"no exchange)" if args.split == "heads"
+                                       else f"replicas x{ws} (independent sequences per GPU)"),
                        "l2": f"flushed before every timed step ({FLUSH_BYTES >> 20} MiB write, outside the events)"},
             "per_kernel": main_res["per_kernel"],
             "roofline": main_res["roofline"],
@@ -948,7 +986,7 @@ def git_sha() -> str:
 def run_key(args, sha: str) -> dict:
     """What identifies one bench entry in a JSONL log (a rerun with the same key is skipped)."""
     return {"impl": args.impl, "workload": args.workload, "n_gpus": args.gpus, "steps": args.steps,
-            "warmup": args.warmup, "git_sha": sha}
+            "warmup": args.warmup, "split": getattr(args, "split", "replicas"), "git_sha": sha}
 
 
 def logged_line(path: str, key: dict):
@@ -973,6 +1011,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="chunk_1m", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--split", choices=["replicas", "heads"], default="replicas",
+                    help="with N > 1: independent replicas per GPU (weak scaling), or the KV-head groups of one "
+                         "workload split over the GPUs (strong scaling; N must divide H_kv)")
     ap.add_argument("--no-companion", action="store_true",
                     help="chunk_1m only: skip the batch-8 1M decode step measured beside the chunk")
     ap.add_argument("--no-e2e", action="store_true")

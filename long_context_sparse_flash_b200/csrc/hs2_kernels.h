@@ -63,7 +63,8 @@ cudaError_t launch_topk(const Problem& p, const float* scores, int64_t sstride, 
 // with on-chip survivor lists, exact final top-k, retry of underestimated rows.
 size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
 // Byte offset, inside that scratch, of the per-row retry marks (int32, one per
-// (sequence, KV head, query) row of the chunk; 1 = the row ran the retry pass).
+// (sequence, KV head, query) row of the chunk; non-zero after the call = the
+// row ran the retry pass).
 size_t select_tc_status_offset(const Problem& p, int i_count, int64_t n_cand_max);
 // Decode selection over few, long rows: each row cut into key chunks (each
 // chunk's exact top-K with scores on its own CTA, then a per-row merge);

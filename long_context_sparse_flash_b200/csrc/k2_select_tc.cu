@@ -100,7 +100,7 @@ struct SelArgs {
     float* samples;         // [rows][SL_SPR]
     int32_t* s_valid;       // [rows] valid samples per row
     float* tau;             // [rows] threshold estimate
-    int32_t* status;        // [rows] 1 = needs the retry pass
+    int32_t* status;        // [rows] 1 = needs the retry pass, 2 = selected by it
     uint2* slots;           // [n_slots][32][cmax] (score bits, j)
     int i_begin, i_count;   // query chunk of this call
     int cmax;               // survivor list capacity per row
@@ -586,7 +586,9 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     orow[u] = -1;
                     if (srow) srow[u] = -1.f;
                 }
-                if (lane == 0) a.status[row0 + q] = 0;
+                // 0: selected by the filtered sweep; 2: selected by the retry pass (a
+                // later call's filtered sweep overwrites every row's mark)
+                if (lane == 0) a.status[row0 + q] = MODE == MODE_RETRY ? 2 : 0;
             }
         }
     }

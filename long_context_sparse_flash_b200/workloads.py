@@ -68,6 +68,9 @@ WORKLOADS: Dict[str, Workload] = {
                  decode=True),
         # profiling case: the last 4096 queries of the 32K prefill (same per-row work, 1/8 of the rows)
         Workload("prefill_32k_tail", 1, 4096, 28672, 32768, 32, 4, 128, 128, 1024, 4, "gaussian", 16, 1),
+        # profiling case: 512 queries over the 1M cache (the sweep's per-CTA work of the 1M
+        # chunk: about 8200 key tiles per CTA, on 64 CTAs; 2.15 GB of K+V)
+        Workload("chunk_1m_prof", 1, 512, 1048576, 1049088, 32, 4, 128, 128, 1024, 4, "segments", 64, 4),
         # profiling case: 4 of the 128K decode sequences (1.07 GB of K+V, > L2)
         Workload("decode_128k_b4", 4, 1, 131071, 131072, 32, 4, 128, 128, 1024, 4, "gaussian", 32, 3,
                  decode=True),

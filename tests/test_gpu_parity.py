@@ -355,3 +355,25 @@ def test_ordinary_inputs_take_no_retry():
     ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_FULL_SELECT)
     nv.full_attn_select(inp["q"], inp["k"], inp["v"], window=w.window, topk=w.topk, q_pos0=w.q_pos0, ws=ws)
     assert nv.hs2_select_retry_rows(shape, ws) == 0
+
+
+def test_kv_head_halves_match_the_whole_call():
+    """One workload's KV-head groups split in two, each half run as its own set
+    of calls (what each GPU of a head-split run computes): every output of a
+    half is bit-identical to the whole call's output for those heads, and the
+    halves match the oracle."""
+    import bench
+    w = wl.custom("head_split", n_q=512, q_pos0=6000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=1, seed=14)
+    inp = wl.make_inputs(w, "cuda")
+    whole = P.run_gpu(w, inp)
+    for r in range(2):
+        w_r, share = bench.head_shard(w, inp, r, 2)
+        half = P.run_gpu(w_r, share)
+        h0, h1 = r * w_r.h_q, (r + 1) * w_r.h_q
+        g0, g1 = r * w_r.h_kv, (r + 1) * w_r.h_kv
+        assert torch.equal(half["idx"], whole["idx"][:, g0:g1])
+        assert torch.equal(half["out"], whole["out"][:, h0:h1])
+        assert torch.equal(half["lse"], whole["lse"][:, h0:h1])
+        assert torch.equal(half["sparse"][0], whole["sparse"][0][:, h0:h1])
+        P.compare_rows(w_r, share, half, 0, np.array([0, 1, 255, 511]))
