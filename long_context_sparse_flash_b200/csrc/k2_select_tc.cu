@@ -6,12 +6,12 @@
 //
 //   score_{g,j}(t) = sum_{h in g} 2^(s2_{h,j} - lse2_h),  s2 = scale*log2(e)*<q_h, k_j>
 //
-// One CTA = one KV group x 32 consecutive queries (N = 32*G columns ordered
+// One CTA = one KV group x QT consecutive queries (N = QT*G columns ordered
 // (query, head)); it sweeps the candidate keys in 128-key tiles:
 //   S^T (TMEM, 128 keys x N, double buffered) = K_tile Q^T    tcgen05.mma
 // and the epilogue thread that owns TMEM lane r (= key j) forms the group sum
-// for each of the 32 queries inside one thread.  Three passes keep the work
-// on chip and exact:
+// for each of its queries inside one thread.  Three passes keep the work on
+// chip and exact:
 //   SAMPLE  1024 keys at a fixed stride S = kv_len / 1024 over the whole cache
 //           (a strided tensor-map view, 8 tiles of 128): sample scores spread
 //           over every segment of the context, not a few contiguous runs
@@ -19,19 +19,36 @@
 //           exceed with high probability: the r-th largest sample, r = L +
 //           4.5 sqrt(L) + 2, where L = K s/n is the expected number of samples
 //           above the K-th best candidate
-//   FILTER  every tile; candidates at or above the row's bound are appended,
-//           in ascending j, to the row's survivor list in this SM's slot of
-//           the workspace (L2-resident).  A list about to overflow is
-//           compacted in place to its exact top K and the bound is raised to
-//           its K-th entry.  At the end each row's exact top-min(K, n) is
-//           taken from the list (radix select on the fp32 bits, ties to the
-//           lower j, output ascending) -- or, if fewer than min(K, n)
-//           candidates passed (tau overestimated), the row is marked,
+//   FILTER  every tile; candidates at or above the row's bound are appended
+//           to the row's survivor list in this SM's slot of the workspace
+//           (L2-resident).  A list about to overflow is compacted in place to
+//           its exact top K and the bound is raised to its K-th entry.  At the
+//           end each row's exact top-min(K, n) is taken from the list (radix
+//           select on the fp32 bits, ties to the lower j, output ascending) --
+//           or, if fewer than min(K, n) candidates passed (tau overestimated),
+//           the row is marked,
 //   RETRY   re-runs only the tiles with a marked row, with bound 0.
-// Ordering of equal scores: the survivor lists are ascending in j, and every
-// selection step keeps the first (lowest-j) entries among equal keys.  The
-// exact select can also write each selected key's score (used to merge the
-// selections of several slices of one context).
+// Ties: every exact select keeps, among the entries equal to the K-th score,
+// those with the lowest j (a second radix pass on j when the tie straddles
+// the cut).  The exact select can also write each selected key's score (used
+// to merge the selections of several slices of one context).
+//
+// Two layouts of the epilogue share everything else (the MMA, TMA, score
+// math and exact selects):
+//   ORDERED  32 queries per CTA on 4 warpgroups of 8 queries.  Each tile, the
+//            four warps of a warpgroup exchange their per-row counts, so the
+//            survivors are appended in ascending j and the final select
+//            writes them out in list order.
+//   COUNTER  28 queries per CTA on 7 warpgroups of 4 queries.  A survivor
+//            takes its position from the row's shared counter (one shared
+//            atomic per key that passes): a tile's entries land in any order,
+//            tiles stay in order, and the final select ranks each kept entry
+//            inside its tile's run.
+// ORDERED serves short candidate ranges, whose rows keep many survivors
+// (about 12% of the candidates at a 32K context); COUNTER serves long ones
+// (under 1% at 1M), where its 28 warps hide more latency and 28-query CTAs
+// fill the last wave of a 4096-query chunk (588 CTAs = 3.97 waves of 148 SMs
+// against 512 = 3.46).
 //
 // The same sweep in MODE_BLOCK serves block-level selection (the design
 // token-level selection replaces, same report and section): the epilogue sums
@@ -53,42 +70,63 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn();                                  
 
 namespace {
 
-constexpr int SL_QT = 32;          // queries per CTA
 constexpr int SL_BN = 128;         // keys per tile (MMA M)
 constexpr int SL_NS = 3;           // K pipeline stages
-constexpr int SL_EPI_WARPS = 16;   // four warpgroups, each a quarter of the query columns
-constexpr int SL_NWG = SL_EPI_WARPS / 4;
-constexpr int SL_TMA_WARP = SL_EPI_WARPS;
-constexpr int SL_MMA_WARP = SL_EPI_WARPS + 1;
-constexpr int SL_THREADS = 32 * (SL_EPI_WARPS + 2);
 constexpr int SL_SAMPLE_TILES = 8; // sample tiles per CTA
 constexpr int SL_SPR = SL_SAMPLE_TILES * SL_BN;  // sample slots per row
 constexpr int SL_CMAX = 4096;      // survivor list capacity per row
 constexpr int SL_SLOTS = 256;      // per-SM survivor slots (indexed by %smid)
 constexpr int SL_MIN_SMEM = 120 * 1024;  // keeps one CTA per SM (slots are per SM)
+constexpr int SL_STAGE = 1024;     // COUNTER final select: one row's kept keys per warp in shared memory
+constexpr int64_t SL_COUNTER_MIN_CAND = int64_t(1) << 18;  // calls whose longest row has this many
+                                                           // candidates use the COUNTER layout
 
 enum { MODE_SAMPLE = 0, MODE_FILTER = 1, MODE_RETRY = 2, MODE_BLOCK = 3 };
+enum { ORDERED = 0, COUNTER = 1 };
 
-template <int D, int G>
+template <int L>
+struct Lay;
+template <>
+struct Lay<ORDERED> {
+    static constexpr int QT = 32, EPI_WARPS = 16;
+};
+template <>
+struct Lay<COUNTER> {
+    static constexpr int QT = 28, EPI_WARPS = 28;
+};
+
+template <int D, int G, int L>
 struct SlCfg {
-    static constexpr int N = SL_QT * G;            // MMA N: (query, head) columns
+    static constexpr int QT = Lay<L>::QT;               // queries per CTA
+    static constexpr int EPI_WARPS = Lay<L>::EPI_WARPS;  // epilogue warps
+    static constexpr int NWG = EPI_WARPS / 4;           // warpgroups, each 1/NWG of the query columns
+    static constexpr int QH = QT / NWG;                 // queries of one warpgroup
+    static constexpr int TMA_WARP = EPI_WARPS, MMA_WARP = EPI_WARPS + 1;
+    static constexpr int THREADS = 32 * (EPI_WARPS + 2);
+    static constexpr int N = QT * G;               // MMA N: (query, head) columns
     static constexpr int KB = D / 64;
     static constexpr int QBLK = N * 128;           // one 64-wide column block of Q (N rows x 128 B)
     static constexpr int KBLK = SL_BN * 128;       // one 64-wide column block of a K tile
     static constexpr int Q_OFF = 0;
     static constexpr int K_OFF = Q_OFF + KB * QBLK;
-    static constexpr int MISC_OFF = K_OFF + SL_NS * KB * KBLK;
+    static constexpr int K_END = K_OFF + SL_NS * KB * KBLK;
+    // COUNTER: after the sweep, the final select stages each row's kept keys over
+    // the dead Q tile and K ring, SL_STAGE int32 per epilogue warp
+    static constexpr int STAGE_BYTES = L == COUNTER ? EPI_WARPS * SL_STAGE * 4 : 0;
+    static constexpr int MISC_OFF = K_END > STAGE_BYTES ? K_END : STAGE_BYTES;
     // misc: barriers, l2[N], row state, per-warp histograms and counts
     static constexpr int BAR_BYTES = 256;
     static constexpr int L2_OFF = MISC_OFF + BAR_BYTES;
     static constexpr int ROW_OFF = L2_OFF + N * 4;
-    static constexpr int ROW_BYTES = SL_QT * 5 * 4;       // cnt[2], lo, tlim, act
-    static constexpr int WCNT_OFF = ROW_OFF + ROW_BYTES;  // [4 warps][32 rows]
-    static constexpr int HIST_OFF = WCNT_OFF + 4 * SL_QT * 4;
-    static constexpr int END = HIST_OFF + SL_EPI_WARPS * 256 * 4;
+    static constexpr int ROW_BYTES = QT * 5 * 4 + 32;    // cnt[2], lo, tlim, act; per-warpgroup ovf
+    static constexpr int WCNT_OFF = ROW_OFF + ROW_BYTES;  // ORDERED: [4 warps][QT rows]
+    static constexpr int HIST_OFF = WCNT_OFF + 4 * QT * 4;
+    static constexpr int END = HIST_OFF + EPI_WARPS * 256 * 4;
     static constexpr int SMEM_NEED = END + 1024;
     static constexpr int SMEM = SMEM_NEED > SL_MIN_SMEM ? SMEM_NEED : SL_MIN_SMEM;
     static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
+    static_assert(NWG <= 8, "named barriers 1..NWG");
+    static_assert(QT % NWG == 0, "whole queries per warpgroup");
 };
 
 enum : int { SB_Q = 0, SB_KFULL = 1, SB_KEMPTY = SB_KFULL + SL_NS, SB_SFULL = SB_KEMPTY + SL_NS,
@@ -101,7 +139,7 @@ struct SelArgs {
     int32_t* s_valid;       // [rows] valid samples per row
     float* tau;             // [rows] threshold estimate
     int32_t* status;        // [rows] 1 = needs the retry pass, 2 = selected by it
-    uint2* slots;           // [n_slots][32][cmax] (score bits, j)
+    uint2* slots;           // [n_slots][QT][cmax] (score bits, j)
     int i_begin, i_count;   // query chunk of this call
     int cmax;               // survivor list capacity per row
     int slot_by_block;      // 1: slot = block id (small grids); 0: slot = %smid (one CTA per SM)
@@ -129,20 +167,23 @@ __device__ __forceinline__ void named_sync(int id, int n) { asm volatile("bar.sy
 // ---------------------------------------------------------------------------
 // warp-level exact selection on (score bits, j) lists
 
-// The K-th largest key among the first n entries of `buf` (key = fp32 bits of a
-// non-negative score) and how many entries equal to it belong to the top K.
-__device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uint32_t* hist, uint32_t& kth,
-                         uint32_t& need_eq) {
+// The K-th largest key among the keys key(i) of the entries i < n that key()
+// accepts (8-bit radix, four passes, one warp): kth, how many entries equal to
+// kth belong to the top K (need_eq), and how many equal kth in all (eq_total).
+// K must not exceed the number of accepted entries.
+template <class KeyFn>
+__device__ void warp_radix_kth(int n, uint32_t K, uint32_t* hist, KeyFn key, uint32_t& kth, uint32_t& need_eq,
+                               uint32_t& eq_total) {
     const int lane = threadIdx.x & 31;
-    uint32_t prefix = 0, pmask = 0, k_rem = K;
+    uint32_t prefix = 0, pmask = 0, k_rem = K, in_bin = 0;
 #pragma unroll 1
     for (int pass = 0; pass < 4; ++pass) {
         const int shift = 24 - 8 * pass;
         for (int u = lane; u < 256; u += 32) hist[u] = 0;
         __syncwarp();
         for (int i = lane; i < n; i += 32) {
-            const uint32_t x = key[(int64_t)i * stride];
-            if ((x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
+            uint32_t x;
+            if (key(i, x) && (x & pmask) == prefix) atomicAdd(&hist[(x >> shift) & 255u], 1u);
         }
         __syncwarp();
         uint32_t bins[8], s = 0;
@@ -158,7 +199,7 @@ __device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uin
             if (lane >= o) incl += y;
         }
         const uint32_t excl = incl - s;
-        uint32_t digit = 0, krem_new = 0;
+        uint32_t digit = 0, krem_new = 0, cnt = 0;
         const bool mine = excl < k_rem && k_rem <= incl;
         if (mine) {
             uint32_t above = excl;
@@ -167,6 +208,7 @@ __device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uin
                 if (above + bins[u] >= k_rem) {
                     digit = 8 * (31 - lane) + u;
                     krem_new = k_rem - above;
+                    cnt = bins[u];
                     break;
                 }
                 above += bins[u];
@@ -176,6 +218,7 @@ __device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uin
         const int src = who ? __ffs(who) - 1 : 0;
         digit = __shfl_sync(0xffffffffu, digit, src);
         krem_new = __shfl_sync(0xffffffffu, krem_new, src);
+        in_bin = __shfl_sync(0xffffffffu, cnt, src);
         prefix |= digit << shift;
         pmask |= 255u << shift;
         k_rem = krem_new;
@@ -183,54 +226,139 @@ __device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uin
     }
     kth = prefix;
     need_eq = k_rem;
+    eq_total = in_bin;
 }
 
-// Keep, in list order, the entries with key > kth plus the first need_eq with
-// key == kth.  compact: write kept entries to the front of `list`; otherwise
-// write their j to `out` (and their scores to `sout` unless it is null).
-// Returns the number kept.
-__device__ int warp_keep(uint2* list, int n, uint32_t kth, uint32_t need_eq, int32_t* out, bool compact,
-                         float* sout = nullptr) {
+// The K-th largest of the first n keys of `key` (element stride `stride`).
+__device__ void warp_kth(const uint32_t* key, int stride, int n, uint32_t K, uint32_t* hist, uint32_t& kth,
+                         uint32_t& need_eq) {
+    uint32_t eq_total;
+    warp_radix_kth(
+        n, K, hist,
+        [&](int i, uint32_t& x) {
+            x = key[(int64_t)i * stride];
+            return true;
+        },
+        kth, need_eq, eq_total);
+}
+
+// The exact top K of a survivor list under the order (score desc, j asc): the
+// K-th score kth, and jth, the largest j kept among the entries whose score
+// equals kth (the need_eq smallest such j; all of them when none is left out).
+// The list's j are distinct.  Keeping the entries with score > kth, or score
+// == kth and j <= jth, keeps exactly K.
+__device__ void list_topk_bound(const uint2* list, int n, uint32_t K, uint32_t* hist, uint32_t& kth, uint32_t& jth) {
+    uint32_t need_eq, eq_total;
+    warp_radix_kth(
+        n, K, hist,
+        [&](int i, uint32_t& x) {
+            x = list[i].x;
+            return true;
+        },
+        kth, need_eq, eq_total);
+    jth = 0xffffffffu;
+    if (eq_total > need_eq) {  // ties at the K-th score straddle the cut: keep the lowest j
+        const uint32_t k_ = kth;
+        uint32_t njth, ne2, eq2;
+        warp_radix_kth(
+            n, need_eq, hist,
+            [&](int i, uint32_t& x) {
+                const uint2 e = list[i];
+                x = ~e.y;
+                return e.x == k_;
+            },
+            njth, ne2, eq2);
+        jth = ~njth;
+    }
+}
+
+__device__ __forceinline__ bool kept(uint2 e, uint32_t kth, uint32_t jth) {
+    return e.x > kth || (e.x == kth && e.y <= jth);
+}
+
+// Keep, in list order, the entries that list_topk_bound's (kth, jth) keeps,
+// compacted in place to the front of `list`; with `stage`, their j are also
+// written to stage[0..kept).  Returns the number kept.
+__device__ int warp_compact(uint2* list, int n, uint32_t kth, uint32_t jth, int32_t* stage = nullptr) {
     const int lane = threadIdx.x & 31;
     const uint32_t lt = (1u << lane) - 1u;
-    uint32_t eq_seen = 0, written = 0;
+    uint32_t written = 0;
     for (int base = 0; base < n; base += 32) {
         const int i = base + lane;
         uint2 e = make_uint2(0u, 0u);
         if (i < n) e = list[i];
-        const bool gt = i < n && e.x > kth;
-        const bool eq = i < n && e.x == kth;
-        const uint32_t eqb = __ballot_sync(0xffffffffu, eq);
-        const bool take = gt || (eq && eq_seen + __popc(eqb & lt) < need_eq);
+        const bool take = i < n && kept(e, kth, jth);
         const uint32_t tb = __ballot_sync(0xffffffffu, take);
         const uint32_t pos = written + __popc(tb & lt);
         __syncwarp();
         if (take) {
-            if (compact) {
-                list[pos] = e;
-            } else {
-                out[pos] = (int32_t)e.y;
-                if (sout) sout[pos] = __uint_as_float(e.x);
-            }
+            list[pos] = e;
+            if (stage) stage[pos] = (int32_t)e.y;
         }
-        eq_seen += __popc(eqb);
         written += __popc(tb);
     }
     __syncwarp();
     return (int)written;
 }
 
+// The kept entries' j (and, if sout is not null, their scores) written to out
+// in list order.  Returns the number written.
+__device__ int warp_take(const uint2* list, int n, uint32_t kth, uint32_t jth, int32_t* out, float* sout) {
+    const int lane = threadIdx.x & 31;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint32_t written = 0;
+    for (int base = 0; base < n; base += 32) {
+        const int i = base + lane;
+        uint2 e = make_uint2(0u, 0u);
+        if (i < n) e = list[i];
+        const bool take = i < n && kept(e, kth, jth);
+        const uint32_t tb = __ballot_sync(0xffffffffu, take);
+        if (take) {
+            const uint32_t pos = written + __popc(tb & lt);
+            out[pos] = (int32_t)e.y;
+            if (sout) sout[pos] = __uint_as_float(e.x);
+        }
+        written += __popc(tb);
+    }
+    __syncwarp();
+    return (int)written;
+}
+
+// The selection of one row, ascending by j, from its kept entries list[0..n),
+// ordered by key tile (j / SL_BN) but in any order inside a tile; their j are
+// read through jat(i) (a staged copy in shared memory, or the list itself).
+// An entry's output position is the number of kept entries in earlier tiles
+// -- the start of its tile's run -- plus its rank by j inside the run.
+// Writes out[0..n) and, if sout is not null, the scores beside them.
+template <class JFn>
+__device__ void warp_emit_sorted(const uint2* list, int n, JFn jat, int32_t* out, float* sout) {
+    const int lane = threadIdx.x & 31;
+    for (int i = lane; i < n; i += 32) {
+        const int32_t j = jat(i);
+        const int32_t tile = j / SL_BN;
+        int lo = i, hi = i + 1;
+        while (lo > 0 && jat(lo - 1) / SL_BN == tile) --lo;
+        while (hi < n && jat(hi) / SL_BN == tile) ++hi;
+        int rank = 0;
+        for (int u = lo; u < hi; ++u) rank += jat(u) < j;
+        out[lo + rank] = j;
+        if (sout) sout[lo + rank] = __uint_as_float(list[i].x);
+    }
+}
+
 // ---------------------------------------------------------------------------
 
-template <int D, int G, int MODE>
-__global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
-                                                                    const __grid_constant__ CUtensorMap tm_k,
-                                                                    Problem p, SelArgs a) {
-    using C = SlCfg<D, G>;
+template <int D, int G, int MODE, int L>
+__global__ void __launch_bounds__(SlCfg<D, G, L>::THREADS, 1)
+    k2_select_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Problem p,
+                        SelArgs a) {
+    using C = SlCfg<D, G, L>;
     constexpr int N = C::N;
-    constexpr int NH = N / SL_NWG;           // columns of one epilogue warpgroup
+    constexpr int QT = C::QT;
+    constexpr int NH = N / C::NWG;           // columns of one epilogue warpgroup
     constexpr int CW = NH < 32 ? NH : 32;    // columns per TMEM load
-    constexpr int QH = SL_QT / SL_NWG;       // queries of one epilogue warpgroup
+    constexpr int QH = C::QH;                // queries of one epilogue warpgroup
+    static_assert(NH % CW == 0 && CW % G == 0, "whole queries per TMEM load");
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -241,17 +369,21 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
     tc::Abort* ab = reinterpret_cast<tc::Abort*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 8);
     volatile int* okv = reinterpret_cast<volatile int*>(sgen + C::MISC_OFF + 8 * SB_COUNT + 16);  // [wg][2]
     float* l2s = reinterpret_cast<float*>(sgen + C::L2_OFF);
-    int32_t* r_cnt = reinterpret_cast<int32_t*>(sgen + C::ROW_OFF);  // [tile parity][32]
-    float* r_lo = reinterpret_cast<float*>(r_cnt + 2 * SL_QT);  // keep scores >= r_lo
-    int32_t* r_tlim = reinterpret_cast<int32_t*>(r_lo + SL_QT);  // last candidate key of the row
-    int32_t* r_act = r_tlim + SL_QT;                             // row takes part in this pass
-    int32_t* wcnt = reinterpret_cast<int32_t*>(sgen + C::WCNT_OFF);  // [4 key quarters][32 rows]
-    uint32_t* hist = reinterpret_cast<uint32_t*>(sgen + C::HIST_OFF);  // [8 warps][256]
+    // ORDERED: r_cnt[tile parity][QT] list lengths; COUNTER: r_cnt[QT], the rows' counters
+    int32_t* r_cnt = reinterpret_cast<int32_t*>(sgen + C::ROW_OFF);
+    float* r_lo = reinterpret_cast<float*>(r_cnt + 2 * QT);   // keep scores >= r_lo
+    int32_t* r_tlim = reinterpret_cast<int32_t*>(r_lo + QT);  // last candidate key of the row
+    int32_t* r_act = r_tlim + QT;                             // row takes part in this pass
+    // COUNTER, per warpgroup: the last tile after which one of its rows passed the
+    // compaction threshold (written by the appending lanes)
+    volatile int32_t* r_ovf = r_act + QT;
+    int32_t* wcnt = reinterpret_cast<int32_t*>(sgen + C::WCNT_OFF);    // ORDERED: [4 key quarters][QT rows]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sgen + C::HIST_OFF);  // [epilogue warps][256]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = blockIdx.y, b = blockIdx.z;
-    const int q0 = blockIdx.x * SL_QT;  // first query of the CTA within the chunk
-    const int nq_here = min(SL_QT, a.i_count - q0);
+    const int q0 = blockIdx.x * QT;  // first query of the CTA within the chunk
+    const int nq_here = min(QT, a.i_count - q0);
     const int64_t pos0 = seq_pos0(p, b, KID_SCORE) + a.i_begin;
     const int64_t t_max = pos0 + q0 + nq_here - 1;
     const int64_t cand_end = last_cand(p, t_max) + 1;  // candidate keys are j < cand_end
@@ -271,14 +403,18 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         return;
     }
     const int cmax = a.cmax;
-    uint2* lists = a.slots + (int64_t)slot * SL_QT * cmax;
+    // a row whose list grew past thr is compacted to its exact top K before the
+    // next tile (which adds at most SL_BN entries); cmax >= topk + SL_BN unless
+    // cmax holds every candidate of the call
+    const int thr = max(cmax - SL_BN, p.topk);
+    uint2* lists = a.slots + (int64_t)slot * QT * cmax;
     // sampling pass: tile it holds keys S (128 it + u), u < 128, of the strided view
     const int64_t S = a.sample_stride;
     const int64_t n_sb = cand_end > 0 ? (cand_end + S - 1) / S : 0;  // sampled keys below the candidate limit
     const int n_tiles = MODE == MODE_SAMPLE ? (int)min((int64_t)SL_SAMPLE_TILES, (n_sb + SL_BN - 1) / SL_BN) : n_ct;
 
     // row state
-    if (tid < SL_QT) {
+    if (tid < QT) {
         const int q = tid;
         const bool live = q < nq_here;
         const int64_t t = pos0 + q0 + q;
@@ -288,29 +424,30 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         if (MODE == MODE_FILTER && act) bs = a.tau[row0 + q];
         if (MODE == MODE_RETRY) act = live && a.status[row0 + q] != 0;
         r_cnt[q] = 0;
-        r_cnt[SL_QT + q] = 0;
+        r_cnt[QT + q] = 0;
+        if (q < C::NWG) r_ovf[q] = -1;
         r_lo[q] = act ? bs : INFINITY;
         r_tlim[q] = (int32_t)max(last_cand(p, t), (int64_t)-1);
         r_act[q] = act;
     }
-    for (int c = tid; c < N; c += SL_THREADS) {
+    for (int c = tid; c < N; c += C::THREADS) {
         const int q = c / G, hh = c % G;
         const int i = a.i_begin + q0 + q;
         l2s[c] = (q < nq_here) ? a.lse[(int64_t)(b * p.hq + g * G + hh) * p.nq + i] * kLog2e : INFINITY;
     }
     if (tid == 0) {
         for (int i = 0; i < SB_COUNT; ++i)
-            tc::mbar_init(bar(i), (i >= SB_SEMPTY && i < SB_SEMPTY + 2) ? 32 * SL_EPI_WARPS : 1);
+            tc::mbar_init(bar(i), (i >= SB_SEMPTY && i < SB_SEMPTY + 2) ? 32 * C::EPI_WARPS : 1);
         ab->flag = 0;
         tc::fence_mbar_init();
     }
-    if (warp == SL_MMA_WARP) tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    if (warp == C::MMA_WARP) tc::tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp == SL_TMA_WARP) {
+    if (warp == C::TMA_WARP) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0 && n_tiles > 0) {
             tc::mbar_expect_tx(bar(SB_Q), C::KB * C::QBLK);
@@ -335,7 +472,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     tc::mbar_wait(bar(SB_KFULL + it % SL_NS), (it / SL_NS) & 1, &none, nullptr, 0, 0);
             }
         }
-    } else if (warp == SL_MMA_WARP) {
+    } else if (warp == C::MMA_WARP) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0 && n_tiles > 0) {
             constexpr uint32_t ID = tc::idesc_bf16(SL_BN, N, 0, 0);
@@ -366,7 +503,6 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
         const int wg = warp >> 2, kq = warp & 3;
         const int et = tid & 127;  // key lane within the tile
         const uint32_t lane_off = (uint32_t)(kq * 32) << 16;
-        const uint32_t lt = (1u << lane) - 1u;
         const int barid = 1 + wg;
         bool ok = true;
         float lo[QH];
@@ -390,29 +526,34 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
             }
             tc::fence_after_sync();
             if constexpr (MODE == MODE_FILTER || MODE == MODE_RETRY) {
-                // rare: a list that could overflow on this tile is first cut to its exact
-                // top K; later keys (larger j) then need a score strictly above its K-th entry
-                // every warp reads the counts before any of them changes (uniform decision)
-                uint32_t need = 0;
+                // rare: a row whose list could overflow on this tile is first cut to its
+                // exact top K; later keys (larger j) then need a score strictly above its
+                // K-th entry.  The four warps of a warpgroup take the same decision:
+                //   ORDERED  from this tile's counts, which no warp changes before the
+                //            warpgroup's next barrier (the next tile's go to the other slot);
+                //   COUNTER  from the warpgroup's mark, written before this tile's barrier
+                //            and changed by no warp of the warpgroup before it decides.
+                int32_t* cnt_now = r_cnt + (L == ORDERED ? (it & 1) * QT : 0);
+                bool need = false;
+                if constexpr (L == ORDERED) {
 #pragma unroll
-                for (int qq = 0; qq < QH; ++qq) {
-                    const int c = r_cnt[(it & 1) * SL_QT + wg * QH + qq];
-                    if (c > cmax - SL_BN && c > p.topk) need |= 1u << qq;
+                    for (int qq = 0; qq < QH; ++qq) need |= cnt_now[wg * QH + qq] > thr;
+                } else {
+                    need = r_ovf[wg] == it - 1;
                 }
                 if (need) {
                     named_sync(barid, 128);
 #pragma unroll 1
                     for (int qq = kq; qq < QH; qq += 4) {
-                        if (!((need >> qq) & 1u)) continue;
                         const int q = wg * QH + qq;
+                        const int cnt = min(cnt_now[q], cmax);  // only this warp changes it now
+                        if (cnt <= thr) continue;
                         uint2* lst = lists + (int64_t)q * cmax;
-                        const int cnt = min(r_cnt[(it & 1) * SL_QT + q], cmax);  // only this warp changes it
-                        uint32_t kth, need_eq;
-                        warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)p.topk, hist + warp * 256,
-                                 kth, need_eq);
-                        const int kept = warp_keep(lst, cnt, kth, need_eq, nullptr, true);
+                        uint32_t kth, jth;
+                        list_topk_bound(lst, cnt, (uint32_t)p.topk, hist + warp * 256, kth, jth);
+                        const int kept = warp_compact(lst, cnt, kth, jth);
                         if (lane == 0) {
-                            r_cnt[(it & 1) * SL_QT + q] = kept;
+                            cnt_now[q] = kept;
                             r_lo[q] = nextafterf(__uint_as_float(kth), INFINITY);
                         }
                     }
@@ -486,11 +627,12 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                         a.samples[(row0 + q) * SL_SPR + it * SL_BN + et] = (j <= last_cand(p, t)) ? sc[qq] : 0.f;
                     }
                 }
-            } else {
-                // FILTER / RETRY: ordered append (ascending j) of the candidates at or
+            } else if constexpr (L == ORDERED) {
+                // FILTER / RETRY, ORDERED: append in ascending j of the candidates at or
                 // above each row's bound; key quarter kq's entries follow quarters < kq.
                 // Tiles entirely below every row's candidate limit skip the per-row test.
                 const bool all_valid = (int64_t)jb + SL_BN - 1 <= last_cand(p, pos0 + q0);
+                const uint32_t lt = (1u << lane) - 1u;
                 uint32_t bal[QH];
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
@@ -502,7 +644,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                     uint32_t mine = 0;
 #pragma unroll
                     for (int qq = 0; qq < QH; ++qq) mine = (lane == qq) ? bal[qq] : mine;
-                    wcnt[kq * SL_QT + wg * QH + lane] = __popc(mine);
+                    wcnt[kq * QT + wg * QH + lane] = __popc(mine);
                 }
                 named_sync(barid, 128);
                 // lane qq: base position of row (wg, qq) for this warp's key quarter; the
@@ -510,15 +652,36 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 int mybase = 0;
                 if (lane < QH) {
                     const int q = wg * QH + lane;
-                    mybase = r_cnt[(it & 1) * SL_QT + q];
-                    for (int w = 0; w < kq; ++w) mybase += wcnt[w * SL_QT + q];
-                    if (kq == 3) r_cnt[((it + 1) & 1) * SL_QT + q] = mybase + wcnt[3 * SL_QT + q];
+                    mybase = r_cnt[(it & 1) * QT + q];
+                    for (int w = 0; w < kq; ++w) mybase += wcnt[w * QT + q];
+                    if (kq == 3) r_cnt[((it + 1) & 1) * QT + q] = mybase + wcnt[3 * QT + q];
                 }
 #pragma unroll
                 for (int qq = 0; qq < QH; ++qq) {
                     const int pos = __shfl_sync(0xffffffffu, mybase, qq) + __popc(bal[qq] & lt);
                     if (((bal[qq] >> lane) & 1u) && pos < cmax)
                         lists[(wg * QH + qq) * cmax + pos] = make_uint2(__float_as_uint(sc[qq]), (uint32_t)j);
+                }
+            } else {
+                // FILTER / RETRY, COUNTER: a candidate at or above its row's bound takes
+                // the next position of the row's list from the row's shared counter (a
+                // tile's entries in any order, tiles in ascending order); a row that passes
+                // thr marks the warpgroup, and the next tile starts by compacting it.
+                const bool all_valid = (int64_t)jb + SL_BN - 1 <= last_cand(p, pos0 + q0);
+                bool keep[QH];
+                int pos[QH];
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    keep[qq] = sc[qq] >= lo[qq];
+                    if (!all_valid) keep[qq] = keep[qq] && (int32_t)j <= tlim[qq];
+                    pos[qq] = keep[qq] ? atomicAdd(&r_cnt[wg * QH + qq], 1) : cmax;
+                }
+#pragma unroll
+                for (int qq = 0; qq < QH; ++qq) {
+                    if (pos[qq] < cmax)
+                        lists[(int64_t)(wg * QH + qq) * cmax + pos[qq]] =
+                            make_uint2(__float_as_uint(sc[qq]), (uint32_t)j);
+                    if (keep[qq] && pos[qq] >= thr) r_ovf[wg] = it;
                 }
             }
         }
@@ -562,26 +725,30 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
                 const int64_t t = pos0 + q0 + q;
                 const int64_t n = last_cand(p, t) + 1;
                 const int n_sel = (int)(n < p.topk ? n : p.topk);
-                const int cnt = min(r_cnt[(n_tiles & 1) * SL_QT + q], cmax);
+                const int cnt = min(r_cnt[(L == ORDERED ? (n_tiles & 1) * QT : 0) + q], cmax);
                 uint2* lst = lists + (int64_t)q * cmax;
                 if (cnt < n_sel) {
                     if (lane == 0) a.status[row0 + q] = 1;  // the estimate was too high: retry
                     continue;
                 }
+                // the exact top n_sel (kth = 0 with every score >= 0 keeps them all)
+                uint32_t kth = 0, jth = 0xffffffffu;
+                if (cnt > n_sel) list_topk_bound(lst, cnt, (uint32_t)n_sel, hist + warp * 256, kth, jth);
                 int written;
-                if (cnt == n_sel) {
-                    for (int u = lane; u < cnt; u += 32) {
-                        const uint2 e = lst[u];
-                        orow[u] = (int32_t)e.y;
-                        if (srow) srow[u] = __uint_as_float(e.x);
-                    }
-                    written = cnt;
+                if constexpr (L == ORDERED) {
+                    written = warp_take(lst, cnt, kth, jth, orow, srow);  // the list is ascending in j
+                } else if (n_sel <= SL_STAGE) {
+                    // kept entries compacted in list order, their j staged over the dead Q
+                    // tile and K ring (every MMA that read them has completed), then
+                    // emitted ascending by j
+                    int32_t* stage = reinterpret_cast<int32_t*>(sgen) + warp * SL_STAGE;
+                    written = warp_compact(lst, cnt, kth, jth, stage);
+                    warp_emit_sorted(lst, written, [&](int i) { return stage[i]; }, orow, srow);
                 } else {
-                    uint32_t kth, need_eq;
-                    warp_kth(reinterpret_cast<const uint32_t*>(lst), 2, cnt, (uint32_t)n_sel, hist + warp * 256, kth,
-                             need_eq);
-                    written = warp_keep(lst, cnt, kth, need_eq, orow, false, srow);
+                    written = warp_compact(lst, cnt, kth, jth);
+                    warp_emit_sorted(lst, written, [&](int i) { return (int32_t)lst[i].y; }, orow, srow);
                 }
+                __syncwarp();
                 for (int u = written + lane; u < p.topk; u += 32) {
                     orow[u] = -1;
                     if (srow) srow[u] = -1.f;
@@ -595,7 +762,7 @@ __global__ void __launch_bounds__(SL_THREADS, 1) k2_select_tc_kernel(const __gri
 
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == SL_MMA_WARP) {
+    if (warp == C::MMA_WARP) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -696,14 +863,14 @@ __global__ void __launch_bounds__(128) k2_block_topk_kernel(Problem p, SelArgs a
     }
 }
 
-// [B][H_q][n_q][D] bf16 seen as (D, H_q, n_q, B) with box (64, G, 32, 1): the
+// [B][H_q][n_q][D] bf16 seen as (D, H_q, n_q, B) with box (64, G, qt, 1): the
 // shared-memory tile rows come out ordered (query, head), 128 bytes each.
-bool make_q_map(CUtensorMap* m, const void* base, int D, int hq, int nq, int B, int G) {
+bool make_q_map(CUtensorMap* m, const void* base, int D, int hq, int nq, int B, int G, int qt) {
     auto fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)hq, (cuuint64_t)nq, (cuuint64_t)B};
     cuuint64_t strides[3] = {(cuuint64_t)nq * D * 2, (cuuint64_t)D * 2, (cuuint64_t)hq * nq * D * 2};
-    cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)SL_QT, 1};
+    cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)qt, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -711,20 +878,20 @@ bool make_q_map(CUtensorMap* m, const void* base, int D, int hq, int nq, int B, 
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int G, int MODE>
+template <int D, int G, int MODE, int L>
 cudaError_t launch_mode(const Problem& p, const CUtensorMap& mq, const CUtensorMap& mk, const SelArgs& a,
                         cudaStream_t st) {
-    using C = SlCfg<D, G>;
-    auto kern = k2_select_tc_kernel<D, G, MODE>;
+    using C = SlCfg<D, G, L>;
+    auto kern = k2_select_tc_kernel<D, G, MODE, L>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    dim3 grid((a.i_count + SL_QT - 1) / SL_QT, p.hkv, p.B);
+    dim3 grid((a.i_count + C::QT - 1) / C::QT, p.hkv, p.B);
     prof_begin(MODE == MODE_SAMPLE   ? KID_SCORE
                : MODE == MODE_FILTER ? KID_FILTER
                : MODE == MODE_RETRY  ? KID_RETRY
                                      : KID_BLOCK_SWEEP,
                st);
-    kern<<<grid, SL_THREADS, C::SMEM, st>>>(mq, mk, p, a);
+    kern<<<grid, C::THREADS, C::SMEM, st>>>(mq, mk, p, a);
     prof_end(st);
     count_launch();
     return cudaGetLastError();
@@ -744,13 +911,14 @@ bool make_strided_map(CUtensorMap* m, const void* base, int D, int64_t kv_len, i
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int G>
-cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+template <int D, int G, int L>
+cudaError_t launch_select_dgl(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
     CUtensorMap mq, mk, mks;
-    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128) ||
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G, Lay<L>::QT) ||
+        !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128) ||
         !make_strided_map(&mks, k, D, p.kv_len, a.sample_stride, (int64_t)p.B * p.hkv))
         return cudaErrorInvalidValue;
-    cudaError_t e = launch_mode<D, G, MODE_SAMPLE>(p, mq, mks, a, st);
+    cudaError_t e = launch_mode<D, G, MODE_SAMPLE, L>(p, mq, mks, a, st);
     if (e != cudaSuccess) return e;
     const int64_t rows = (int64_t)p.B * p.hkv * a.i_count;
     prof_begin(KID_THRESH, st);
@@ -758,16 +926,24 @@ cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, con
     prof_end(st);
     count_launch();
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = launch_mode<D, G, MODE_FILTER>(p, mq, mk, a, st)) != cudaSuccess) return e;
-    return launch_mode<D, G, MODE_RETRY>(p, mq, mk, a, st);
+    if ((e = launch_mode<D, G, MODE_FILTER, L>(p, mq, mk, a, st)) != cudaSuccess) return e;
+    return launch_mode<D, G, MODE_RETRY, L>(p, mq, mk, a, st);
+}
+
+template <int D, int G>
+cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
+                             cudaStream_t st) {
+    return layout == COUNTER ? launch_select_dgl<D, G, COUNTER>(p, q, k, a, st)
+                             : launch_select_dgl<D, G, ORDERED>(p, q, k, a, st);
 }
 
 template <int D, int G>
 cudaError_t launch_block_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
     CUtensorMap mq, mk;
-    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G) || !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G, Lay<ORDERED>::QT) ||
+        !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
         return cudaErrorInvalidValue;
-    return launch_mode<D, G, MODE_BLOCK>(p, mq, mk, a, st);
+    return launch_mode<D, G, MODE_BLOCK, ORDERED>(p, mq, mk, a, st);
 }
 
 template <int D>
@@ -781,41 +957,47 @@ cudaError_t launch_block_d(const Problem& p, const void* q, const void* k, const
 }
 
 template <int D>
-cudaError_t launch_select_d(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+cudaError_t launch_select_d(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
+                            cudaStream_t st) {
     switch (p.hq / p.hkv) {
-        case 1: return launch_select_dg<D, 1>(p, q, k, a, st);
-        case 2: return launch_select_dg<D, 2>(p, q, k, a, st);
-        case 4: return launch_select_dg<D, 4>(p, q, k, a, st);
-        default: return launch_select_dg<D, 8>(p, q, k, a, st);
+        case 1: return launch_select_dg<D, 1>(p, q, k, a, layout, st);
+        case 2: return launch_select_dg<D, 2>(p, q, k, a, layout, st);
+        case 4: return launch_select_dg<D, 4>(p, q, k, a, layout, st);
+        default: return launch_select_dg<D, 8>(p, q, k, a, layout, st);
     }
 }
 
 }  // namespace
 
-// Survivor list capacity and slot count of a call over queries with up to
-// n_cand_max candidates, in CTAs of 32 queries.
-static void select_tc_geometry(const Problem& p, int i_count, int64_t n_cand_max, int& cmax, int& n_slots,
-                               int& by_block) {
+// The epilogue layout of a call whose longest row has n_cand_max candidates.
+static int select_tc_layout(int64_t n_cand_max) { return n_cand_max >= SL_COUNTER_MIN_CAND ? COUNTER : ORDERED; }
+
+// Layout, survivor list capacity and slot count of a call over queries with up
+// to n_cand_max candidates, in CTAs of the layout's qt queries.
+static void select_tc_geometry(const Problem& p, int i_count, int64_t n_cand_max, int& layout, int& qt, int& cmax,
+                               int& n_slots, int& by_block) {
+    layout = select_tc_layout(n_cand_max);
+    qt = layout == COUNTER ? Lay<COUNTER>::QT : Lay<ORDERED>::QT;
     cmax = n_cand_max <= SL_CMAX ? (int)((n_cand_max + 31) / 32 * 32) : SL_CMAX;
     if (cmax < 32) cmax = 32;
-    const int64_t grid = (int64_t)((i_count + SL_QT - 1) / SL_QT) * p.hkv * p.B;
+    const int64_t grid = (int64_t)((i_count + qt - 1) / qt) * p.hkv * p.B;
     by_block = grid <= SL_SLOTS;
     n_slots = by_block ? (int)grid : SL_SLOTS;
 }
 
 size_t select_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max) {
-    int cmax, n_slots, by_block;
-    select_tc_geometry(p, i_count, n_cand_max, cmax, n_slots, by_block);
+    int layout, qt, cmax, n_slots, by_block;
+    select_tc_geometry(p, i_count, n_cand_max, layout, qt, cmax, n_slots, by_block);
     const int64_t rows = (int64_t)p.B * p.hkv * i_count;
     const size_t per_row = SL_SPR * 4 + 3 * 4;
-    return (size_t)n_slots * SL_QT * cmax * sizeof(uint2) + (size_t)rows * per_row;
+    return (size_t)n_slots * qt * cmax * sizeof(uint2) + (size_t)rows * per_row;
 }
 
 size_t select_tc_status_offset(const Problem& p, int i_count, int64_t n_cand_max) {
-    int cmax, n_slots, by_block;
-    select_tc_geometry(p, i_count, n_cand_max, cmax, n_slots, by_block);
+    int layout, qt, cmax, n_slots, by_block;
+    select_tc_geometry(p, i_count, n_cand_max, layout, qt, cmax, n_slots, by_block);
     const int64_t rows = (int64_t)p.B * p.hkv * i_count;
-    return (size_t)n_slots * SL_QT * cmax * sizeof(uint2) + (size_t)rows * (SL_SPR * 4 + 2 * 4);
+    return (size_t)n_slots * qt * cmax * sizeof(uint2) + (size_t)rows * (SL_SPR * 4 + 2 * 4);
 }
 
 cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
@@ -824,14 +1006,14 @@ cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, con
     const int64_t rows = (int64_t)p.B * p.hkv * i_count;
     uint8_t* base = reinterpret_cast<uint8_t*>(scratch);
     SelArgs a{};
-    int n_slots;
-    select_tc_geometry(p, i_count, n_cand_max, a.cmax, n_slots, a.slot_by_block);
+    int layout, qt, n_slots;
+    select_tc_geometry(p, i_count, n_cand_max, layout, qt, a.cmax, n_slots, a.slot_by_block);
     a.sample_stride = p.kv_len / (SL_SAMPLE_TILES * SL_BN) > 1 ? p.kv_len / (SL_SAMPLE_TILES * SL_BN) : 1;
     a.lse = lse;
     a.idx = idx;
     a.sel_score = sel_score;
     a.slots = reinterpret_cast<uint2*>(base);
-    base += (size_t)n_slots * SL_QT * a.cmax * sizeof(uint2);
+    base += (size_t)n_slots * qt * a.cmax * sizeof(uint2);
     a.samples = reinterpret_cast<float*>(base);
     base += (size_t)rows * SL_SPR * 4;
     a.s_valid = reinterpret_cast<int32_t*>(base);
@@ -841,8 +1023,8 @@ cudaError_t launch_select_tc(const Problem& p, const void* q, const void* k, con
     a.status = reinterpret_cast<int32_t*>(base);
     a.i_begin = i_begin;
     a.i_count = i_count;
-    if (p.D == 64) return launch_select_d<64>(p, q, k, a, st);
-    return launch_select_d<128>(p, q, k, a, st);
+    if (p.D == 64) return launch_select_d<64>(p, q, k, a, layout, st);
+    return launch_select_d<128>(p, q, k, a, layout, st);
 }
 
 // Chunk sums: one float per 32 keys of every candidate tile, rows of cstride.

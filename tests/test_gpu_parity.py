@@ -377,3 +377,68 @@ def test_kv_head_halves_match_the_whole_call():
         assert torch.equal(half["lse"], whole["lse"][:, h0:h1])
         assert torch.equal(half["sparse"][0], whole["sparse"][0][:, h0:h1])
         P.compare_rows(w_r, share, half, 0, np.array([0, 1, 255, 511]))
+
+
+# The selection sweep has two epilogue layouts (ORDERED for calls whose longest
+# row has fewer than 2^18 candidates, COUNTER from 2^18 on).  The small shapes
+# above exercise ORDERED; these put every row of a COUNTER call next to the
+# oracle: ragged tails of 28-query CTAs, exact ties (list compaction, the j
+# tie-break and the run-ranked output), the retry pass, and a budget above the
+# shared-memory staging of the final select.
+COUNTER_MIN_CAND = 1 << 18
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("counter_segments", dict(n_q=60, q_pos0=280000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                              keys="segments", needles=16)),
+    ("counter_d64_g4", dict(n_q=33, q_pos0=270000, h_q=16, h_kv=4, head_dim=64, window=64, topk=512)),
+    ("counter_topk2048", dict(n_q=30, q_pos0=265000, h_q=16, h_kv=2, head_dim=128, window=128, topk=2048)),
+], ids=["segments", "d64_g4", "topk2048"])
+def test_counter_layout_every_row(name, kw):
+    w = wl.custom(name, n_sparse=1, seed=15, **kw)
+    assert w.q_pos0 + w.n_q - w.window >= COUNTER_MIN_CAND
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+    _row_properties(gpu["idx"], w)
+
+
+def test_counter_layout_exact_ties():
+    """q = 0 over 270K candidates: every score is G/(t+1), every candidate passes
+    the bound, the lists overflow and are compacted with the lower-j tie-break,
+    and the selection must be exactly 0..K-1 (eight full key tiles, ranked
+    inside their runs)."""
+    w = wl.custom("counter_ties", n_q=56, q_pos0=270000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=1, seed=16)
+    inp = wl.make_inputs(w, "cuda")
+    inp["q"].zero_()
+    gpu = P.run_gpu(w, inp)
+    want = torch.arange(w.topk, dtype=torch.int32, device="cuda")
+    assert torch.equal(gpu["idx"], want.expand_as(gpu["idx"]))
+    P.compare_rows(w, inp, gpu, 0, np.array([0, 27, 28, 55]))
+
+
+def test_counter_layout_forced_retry():
+    """The retry pass of the COUNTER layout: strong plants at the sampling stride
+    make the estimated bound overshoot on every row."""
+    w = wl.custom("counter_retry", n_q=40, q_pos0=270000, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024,
+                  n_sparse=1, seed=17)
+    inp = wl.make_inputs(w, "cuda")
+    q, k = inp["q"], inp["k"]
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(78)
+    u = torch.randn(w.h_kv, w.head_dim, generator=gen, device="cuda")
+    u = u / u.norm(dim=-1, keepdim=True)
+    q_f = q.float().view(1, w.h_kv, w.group, w.n_q, w.head_dim) + 2.0 * u.view(1, w.h_kv, 1, 1, w.head_dim)
+    q.copy_(q_f.view_as(q).to(torch.bfloat16))
+    S = w.kv_len // 1024
+    pos = torch.arange(0, w.kv_len, S, device="cuda")
+    noise = torch.randn(w.h_kv, pos.numel(), w.head_dim, generator=gen, device="cuda")
+    k[0][:, pos, :] = (8.0 * u[:, None, :] + 0.1 * noise).to(torch.bfloat16)
+    shape = nv.shape_of(q, k, window=w.window, topk=w.topk, q_pos0=w.q_pos0)
+    ws = nv.alloc_workspace(shape, nv.HS2_ENTRY_FULL_SELECT)
+    out, lse, idx = nv.full_attn_select(q, k, inp["v"], window=w.window, topk=w.topk, q_pos0=w.q_pos0, ws=ws)
+    assert nv.hs2_select_retry_rows(shape, ws) == w.h_kv * w.n_q
+    sp = [nv.sparse_attn(qs, k, inp["v"], idx, window=w.window, q_pos0=w.q_pos0) for qs in inp["q_sparse"]]
+    torch.cuda.synchronize()
+    P.compare_rows(w, inp, dict(out=out, lse=lse, idx=idx, sparse=sp), 0, np.arange(w.n_q))
