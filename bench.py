@@ -124,16 +124,24 @@ def unique_kv_rows(w: wl.Workload, idx: torch.Tensor) -> float:
     return float(total)
 
 
+# the selection sweep's CTAs hold 32 queries below this many candidates in the
+# call's longest row (the ORDERED layout) and 28 from it on (COUNTER)
+SELECT_COUNTER_MIN_CAND = 1 << 18
+
+
 def select_stream_bytes(w: wl.Workload) -> float:
     """Bytes the filtered sweep streams per call: every CTA (32 queries of one KV
-    group) reads the K rows of its candidate tiles (128 keys each) once, plus the
-    queries, the LSE and the written selection.  The fraction of HBM bandwidth
-    this gives is the one usually quoted for a select pass; most of
-    the K reads are L2 hits, and the binding unit is the ex2 rate."""
+    group, or 28 in the layout used for long rows) reads the K rows of its
+    candidate tiles (128 keys each) once, plus the queries, the LSE and the
+    written selection.  The fraction of HBM bandwidth this gives is the one
+    usually quoted for a select pass; most of the K reads are L2 hits, and the
+    binding unit is the ex2 rate."""
     D = w.head_dim
+    longest = w.q_pos0 + w.n_q - w.window
+    qt = 28 if longest >= SELECT_COUNTER_MIN_CAND else 32
     tiles = 0
-    for q0 in range(0, w.n_q, 32):
-        t_max = w.q_pos0 + min(q0 + 32, w.n_q) - 1
+    for q0 in range(0, w.n_q, qt):
+        t_max = w.q_pos0 + min(q0 + qt, w.n_q) - 1
         cand_end = t_max - w.window + 1
         tiles += max(0, -(-cand_end // 128))
     k_bytes = tiles * 128 * D * 2 * w.h_kv * w.batch

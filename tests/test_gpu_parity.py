@@ -290,12 +290,16 @@ def _check_selection_and_scores(g_idx, g_score, ores, ts, w, what):
             assert np.all(np.abs(got - want) <= 1e-9 + 1e-4 * np.abs(want)), f"{what} row t={t} g={g}: scores"
 
 
-def test_selection_pass_fed_the_oracle_lse():
+@pytest.mark.parametrize("n_q,q_pos0,topk", [(600, 1400, 256), (64, 270000, 1024)], ids=["ordered", "counter"])
+def test_selection_pass_fed_the_oracle_lse(n_q, q_pos0, topk):
     """The selection pass alone (the slice step of context parallelism over the
     whole cache), fed the oracle's LSE instead of the full-attention kernel's:
-    isolates the selection kernel from the LSE the first kernel computes."""
+    isolates the selection kernel from the LSE the first kernel computes.  It
+    also returns each selected key's score, checked against the oracle's.  The
+    second case has more than 2^18 candidates per row (the COUNTER layout, as
+    each slice of a 1M context split four ways has)."""
     from long_context_sparse_flash_b200 import cp
-    w = wl.custom("k2_oracle_lse", n_q=600, q_pos0=1400, h_q=16, h_kv=2, head_dim=128, window=128, topk=256,
+    w = wl.custom("k2_oracle_lse", n_q=n_q, q_pos0=q_pos0, h_q=16, h_kv=2, head_dim=128, window=128, topk=topk,
                   n_sparse=0, seed=9)
     inp = wl.make_inputs(w, "cuda", with_sparse=False)
     ts = w.q_pos0 + np.arange(w.n_q)
@@ -393,13 +397,15 @@ COUNTER_MIN_CAND = 1 << 18
                               keys="segments", needles=16)),
     ("counter_d64_g4", dict(n_q=33, q_pos0=270000, h_q=16, h_kv=4, head_dim=64, window=64, topk=512)),
     ("counter_topk2048", dict(n_q=30, q_pos0=265000, h_q=16, h_kv=2, head_dim=128, window=128, topk=2048)),
-], ids=["segments", "d64_g4", "topk2048"])
+    ("counter_batch2", dict(batch=2, n_q=31, q_pos0=263000, h_q=8, h_kv=2, head_dim=128, window=128, topk=1024)),
+], ids=["segments", "d64_g4", "topk2048", "batch2"])
 def test_counter_layout_every_row(name, kw):
     w = wl.custom(name, n_sparse=1, seed=15, **kw)
     assert w.q_pos0 + w.n_q - w.window >= COUNTER_MIN_CAND
     inp = wl.make_inputs(w, "cuda")
     gpu = P.run_gpu(w, inp)
-    P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+    for b in range(w.batch):
+        P.compare_rows(w, inp, gpu, b, np.arange(w.n_q))
     _row_properties(gpu["idx"], w)
 
 
