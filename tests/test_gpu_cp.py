@@ -124,3 +124,37 @@ def test_slice_steps_report_timeouts_and_checks_through_their_workspace():
     first = offs[1] - w.q_pos0
     assert torch.all(torch.isneginf(lse[:, :, :first])) and torch.all(out[:, :, :first] == 0)
     assert torch.all(torch.isfinite(lse[:, :, first:]))
+
+
+def test_context_parallel_class_over_nccl_one_rank():
+    """The ContextParallel class as each rank of a multi-GPU run drives it: the
+    library's kernels for the slice steps and merges, and the NCCL all-gather
+    (dist_gather) to stack the per-slice results, here as rank 0 of a one-rank
+    process group on this GPU (the collective runs on the device but exchanges
+    nothing).  Its results equal those of the one-process path over the same
+    single slice bit for bit, and match the oracle on every row."""
+    import datetime
+    import socket
+    import torch.distributed as dist
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        w = wl.custom("cp_nccl", n_q=300, q_pos0=500, h_q=8, h_kv=2, head_dim=64, window=64, topk=128, n_sparse=1,
+                      seed=23)
+        inp = wl.make_inputs(w, "cuda")
+        rank = cp.ContextParallel(inp["k"], inp["v"], rank=0, kv_offs=[0], kv_len=w.kv_len, window=w.window,
+                                  topk=w.topk)
+        before = nv.hs2_launch_count()
+        out, lse, idx = rank.full_attn_select(inp["q"], w.q_pos0)
+        sp = [rank.sparse_attn(qs, idx, w.q_pos0) for qs in inp["q_sparse"]]
+        torch.cuda.synchronize()
+        assert nv.hs2_launch_count() > before
+        ref = _run_cp(w, inp, 1)
+        assert torch.equal(out, ref["out"]) and torch.equal(lse, ref["lse"]) and torch.equal(idx, ref["idx"])
+        assert all(torch.equal(a, b) for a, b in zip(sp, ref["sparse"]))
+        P.compare_rows(w, inp, dict(out=out, lse=lse, idx=idx, sparse=sp), 0, np.arange(w.n_q))
+    finally:
+        dist.destroy_process_group()
