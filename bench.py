@@ -557,10 +557,13 @@ class Step:
 
 
 def dist_setup(n_gpus: int):
+    """One process per GPU.  A process group (NCCL) is set up whenever the
+    launcher is torchrun, a one-rank run included, so the barrier and the max
+    over ranks take the same collective path at every N."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if ws > 1:
+    if ws > 1 or os.environ.get("TORCHELASTIC_RUN_ID"):
         import datetime
         torch.cuda.set_device(local)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
@@ -570,14 +573,18 @@ def dist_setup(n_gpus: int):
     return ws, rank, local
 
 
+def dist_on() -> bool:
+    return torch.distributed.is_available() and torch.distributed.is_initialized()
+
+
 def barrier(ws):
-    if ws > 1:
+    if dist_on():
         torch.distributed.barrier()
 
 
 def max_over_ranks(x: float, ws: int) -> float:
     """The slowest rank's time (every rank gets it)."""
-    if ws == 1:
+    if not dist_on():
         return x
     dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
     t = torch.tensor([x], dtype=torch.float64, device=dev)
@@ -940,7 +947,7 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     else:
         line = None
-    if ws > 1:
+    if dist_on():
         torch.distributed.destroy_process_group()
     return line
 
