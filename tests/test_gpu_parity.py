@@ -88,7 +88,7 @@ def test_prefill_32k_sampled():
     w = wl.WORKLOADS["prefill_32k"]
     inp = wl.make_inputs(w, "cuda")
     gpu = P.run_gpu(w, inp)
-    rows = wl.stratified_rows(w, 12)
+    rows = wl.stratified_rows(w, 32)
     res = P.compare_rows(w, inp, gpu, 0, rows)
     print("32k", res["idx"], res["out_err"], res["sparse_err"])
     _row_properties(gpu["idx"], w)
@@ -116,7 +116,7 @@ def test_chunk_256k_sampled():
     w = wl.WORKLOADS["chunk_256k"]
     inp = wl.make_inputs(w, "cuda")
     gpu = P.run_gpu(w, inp)
-    rows = wl.stratified_rows(w, 8)
+    rows = wl.stratified_rows(w, 32)
     res = P.compare_rows(w, inp, gpu, 0, rows)
     print("256k", res["idx"], res["out_err"], res["sparse_err"])
     _row_properties(gpu["idx"], w)
