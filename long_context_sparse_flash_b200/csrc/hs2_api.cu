@@ -222,9 +222,20 @@ BlockPlan block_plan(const Problem& p) {
     if (cand <= 0 || p.nq == 0 || p.B == 0 || p.topk == 0) return bp;
     bp.n_cand_max = cand;
     const size_t per_q = block_tc_scratch_bytes(p, 1, cand);
-    int64_t chunk = (int64_t)(kScoreBudget / per_q) / 32 * 32;
-    if (chunk < 32) chunk = 32;
-    if (chunk > p.nq) chunk = p.nq;
+    const int64_t fit = (int64_t)(kScoreBudget / per_q);  // queries whose sums fit the budget
+    int64_t chunk = p.nq;
+    if (fit < p.nq) {
+        // Every CTA of the sweep takes about the same time (it sweeps every
+        // candidate tile of its queries) and holds one SM, so a chunk costs whole
+        // waves of 148 CTAs: cut the queries into chunks of whole waves.  At 1M
+        // that is 4 chunks of 1036 queries (148 CTAs each) instead of 2016, 2016
+        // and 64 queries (288, 288 and 12 CTAs: 5 waves).
+        const int64_t qt = select_tc_qt(cand);
+        const int64_t groups = (int64_t)p.hkv * p.B;     // CTAs per qt queries
+        const int64_t wave_q = 148 / groups * qt;        // queries of one full wave
+        chunk = wave_q > 0 && fit >= wave_q ? fit / wave_q * wave_q : fit / qt * qt;
+        if (chunk < qt) chunk = qt;
+    }
     bp.chunk = (int)chunk;
     bp.bytes = block_tc_scratch_bytes(p, bp.chunk, cand);
     return bp;

@@ -53,7 +53,8 @@
 // The same sweep in MODE_BLOCK serves block-level selection (the design
 // token-level selection replaces, same report and section): the epilogue sums
 // each warp's 32 keys per query and writes one float per 32 candidate keys,
-// and k2_block_topk_kernel ranks whole blocks from those sums.
+// and k2_block_topk_kernel ranks whole blocks from those sums.  It takes the
+// token sweep's geometry for the same candidate count (ORDERED or COUNTER).
 //
 // The buffer may hold one slice of a longer context (context parallelism):
 // positions are then shifted by the slice's first key, and every candidate
@@ -599,24 +600,36 @@ __global__ void __launch_bounds__(SlCfg<D, G, L>::THREADS, 1)
             tc::mbar_arrive(bar(SB_SEMPTY + sb));
 
             if constexpr (MODE == MODE_BLOCK) {
-                // sum of the warp's 32 keys for each of its QH = 8 queries, as a
-                // transposing butterfly: every exchange halves the values a lane holds,
-                // so lane l ends with query l >> 2 summed over all 32 lanes (9 shuffles
-                // instead of 8 x 5)
-                static_assert(QH == 8, "the butterfly below reduces 8 query columns");
-                float h4[4], h2[2], h1;
-                const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4;
+                // sum of the warp's 32 keys for each of its QH queries, as a transposing
+                // butterfly: every exchange halves the values a lane holds, so lane l ends
+                // with query l / (32 / QH) summed over all 32 lanes.  Both layouts add the
+                // lanes in the same tree (xor 16, 8, 4, 2, 1), so their sums agree bit for bit.
+                static_assert(QH == 8 || QH == 4, "the butterflies below reduce 8 or 4 query columns");
+                float h1;
+                const bool b4 = lane & 16, b3 = lane & 8;
+                if constexpr (QH == 8) {
+                    float h4[4], h2[2];
+                    const bool b2 = lane & 4;
 #pragma unroll
-                for (int u = 0; u < 4; ++u)
-                    h4[u] = (b4 ? sc[4 + u] : sc[u]) + __shfl_xor_sync(0xffffffffu, b4 ? sc[u] : sc[4 + u], 16);
+                    for (int u = 0; u < 4; ++u)
+                        h4[u] = (b4 ? sc[4 + u] : sc[u]) + __shfl_xor_sync(0xffffffffu, b4 ? sc[u] : sc[4 + u], 16);
 #pragma unroll
-                for (int u = 0; u < 2; ++u)
-                    h2[u] = (b3 ? h4[2 + u] : h4[u]) + __shfl_xor_sync(0xffffffffu, b3 ? h4[u] : h4[2 + u], 8);
-                h1 = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h2[0] : h2[1], 4);
+                    for (int u = 0; u < 2; ++u)
+                        h2[u] = (b3 ? h4[2 + u] : h4[u]) + __shfl_xor_sync(0xffffffffu, b3 ? h4[u] : h4[2 + u], 8);
+                    h1 = (b2 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? h2[0] : h2[1], 4);
+                } else {
+                    float h2[2];
+#pragma unroll
+                    for (int u = 0; u < 2; ++u)
+                        h2[u] = (b4 ? sc[2 + u] : sc[u]) + __shfl_xor_sync(0xffffffffu, b4 ? sc[u] : sc[2 + u], 16);
+                    h1 = (b3 ? h2[1] : h2[0]) + __shfl_xor_sync(0xffffffffu, b3 ? h2[0] : h2[1], 8);
+                    h1 += __shfl_xor_sync(0xffffffffu, h1, 4);
+                }
                 h1 += __shfl_xor_sync(0xffffffffu, h1, 2);
                 h1 += __shfl_xor_sync(0xffffffffu, h1, 1);
-                const int q = wg * QH + (lane >> 2);
-                if ((lane & 3) == 0 && q < nq_here)
+                constexpr int LPQ = 32 / QH;  // lanes per query after the exchanges
+                const int q = wg * QH + lane / LPQ;
+                if (lane % LPQ == 0 && q < nq_here)
                     a.csum[(row0 + q) * a.cstride + (jb >> 5) + kq] = h1;
             } else if constexpr (MODE == MODE_SAMPLE) {
 #pragma unroll
@@ -937,22 +950,30 @@ cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, con
                              : launch_select_dgl<D, G, ORDERED>(p, q, k, a, st);
 }
 
-template <int D, int G>
-cudaError_t launch_block_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+template <int D, int G, int L>
+cudaError_t launch_block_dgl(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
     CUtensorMap mq, mk;
-    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G, Lay<ORDERED>::QT) ||
+    if (!make_q_map(&mq, q, D, p.hq, p.nq, p.B, G, Lay<L>::QT) ||
         !make_map(&mk, k, D, (uint64_t)p.kv_len, (uint64_t)p.B * p.hkv, 128))
         return cudaErrorInvalidValue;
-    return launch_mode<D, G, MODE_BLOCK, ORDERED>(p, mq, mk, a, st);
+    return launch_mode<D, G, MODE_BLOCK, L>(p, mq, mk, a, st);
+}
+
+template <int D, int G>
+cudaError_t launch_block_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
+                            cudaStream_t st) {
+    return layout == COUNTER ? launch_block_dgl<D, G, COUNTER>(p, q, k, a, st)
+                             : launch_block_dgl<D, G, ORDERED>(p, q, k, a, st);
 }
 
 template <int D>
-cudaError_t launch_block_d(const Problem& p, const void* q, const void* k, const SelArgs& a, cudaStream_t st) {
+cudaError_t launch_block_d(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
+                           cudaStream_t st) {
     switch (p.hq / p.hkv) {
-        case 1: return launch_block_dg<D, 1>(p, q, k, a, st);
-        case 2: return launch_block_dg<D, 2>(p, q, k, a, st);
-        case 4: return launch_block_dg<D, 4>(p, q, k, a, st);
-        default: return launch_block_dg<D, 8>(p, q, k, a, st);
+        case 1: return launch_block_dg<D, 1>(p, q, k, a, layout, st);
+        case 2: return launch_block_dg<D, 2>(p, q, k, a, layout, st);
+        case 4: return launch_block_dg<D, 4>(p, q, k, a, layout, st);
+        default: return launch_block_dg<D, 8>(p, q, k, a, layout, st);
     }
 }
 
@@ -971,6 +992,10 @@ cudaError_t launch_select_d(const Problem& p, const void* q, const void* k, cons
 
 // The epilogue layout of a call whose longest row has n_cand_max candidates.
 static int select_tc_layout(int64_t n_cand_max) { return n_cand_max >= SL_COUNTER_MIN_CAND ? COUNTER : ORDERED; }
+
+int select_tc_qt(int64_t n_cand_max) {
+    return select_tc_layout(n_cand_max) == COUNTER ? Lay<COUNTER>::QT : Lay<ORDERED>::QT;
+}
 
 // Layout, survivor list capacity and slot count of a call over queries with up
 // to n_cand_max candidates, in CTAs of the layout's qt queries.
@@ -1047,7 +1072,11 @@ cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* 
     a.cstride = block_cstride(n_cand_max);
     // the sweep only runs when some row has more candidate blocks than the budget
     if (n_cand_max / blk > p.topk / blk && p.topk >= blk) {
-        const cudaError_t e = p.D == 64 ? launch_block_d<64>(p, q, k, a, st) : launch_block_d<128>(p, q, k, a, st);
+        // the token sweep's epilogue geometry for this candidate count (the chunk
+        // sums are the same in both)
+        const int layout = select_tc_layout(n_cand_max);
+        const cudaError_t e = p.D == 64 ? launch_block_d<64>(p, q, k, a, layout, st)
+                                        : launch_block_d<128>(p, q, k, a, layout, st);
         if (e != cudaSuccess) return e;
     }
     const int64_t rows = (int64_t)p.B * p.hkv * i_count;

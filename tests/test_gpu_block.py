@@ -76,6 +76,8 @@ BLOCK_SHAPES = [
                                         window=64, topk=192)),
     ("b32_topk_below_block", 32, dict(n_q=64, q_pos0=200, h_q=8, h_kv=2, head_dim=64, window=8, topk=20)),
     ("b128_topk_2048", 128, dict(n_q=64, q_pos0=3000, h_q=16, h_kv=2, head_dim=64, window=128, topk=2048)),
+    # more than 2^18 candidates per row: the sweep's 28-query geometry (COUNTER)
+    ("b64_counter_270k", 64, dict(n_q=64, q_pos0=270000, h_q=16, h_kv=2, head_dim=128, window=128, topk=1024)),
 ]
 
 
@@ -123,11 +125,14 @@ def test_prefill_32k_block64_sampled():
 
 def test_chunk_1m_block64_sampled():
     """1M-token cache, 4096 new queries: the chunk sums (one float per 32 keys per
-    row, 1 GiB budget) take three query chunks of 2016, 2016 and 64 queries."""
+    row, 1 GiB budget) take query chunks of whole waves of CTAs, 1036 queries
+    each (148 CTAs of 28 queries) and 988 last; rows on both sides of every
+    chunk boundary, and seeded random ones."""
     w = wl.WORKLOADS["chunk_1m"]
     inp = wl.make_inputs(w, "cuda")
     gpu = run_block(w, inp, 64)
-    rows = np.array([0, 2015, 2016, 4031, 4032, 4095])
+    edges = np.array([0, 1035, 1036, 2071, 2072, 3107, 3108, 4095])
+    rows = np.union1d(edges, np.random.default_rng(7).integers(0, w.n_q, size=8))
     res = compare_block_rows(w, inp, gpu, 0, rows, 64)
     print("1m block 64", res["idx"], res["out_err"])
     _block_row_properties(gpu["idx"], w, 64)
