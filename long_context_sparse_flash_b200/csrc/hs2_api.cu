@@ -230,7 +230,7 @@ BlockPlan block_plan(const Problem& p) {
         // waves of 148 CTAs: cut the queries into chunks of whole waves.  At 1M
         // that is 4 chunks of 1036 queries (148 CTAs each) instead of 2016, 2016
         // and 64 queries (288, 288 and 12 CTAs: 5 waves).
-        const int64_t qt = select_tc_qt(cand);
+        const int64_t qt = select_tc_qt(cand, p.hq / p.hkv);
         const int64_t groups = (int64_t)p.hkv * p.B;     // CTAs per qt queries
         const int64_t wave_q = 148 / groups * qt;        // queries of one full wave
         chunk = wave_q > 0 && fit >= wave_q ? fit / wave_q * wave_q : fit / qt * qt;

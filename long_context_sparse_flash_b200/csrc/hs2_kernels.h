@@ -77,8 +77,9 @@ cudaError_t launch_topk_decode(const Problem& p, const float* scores, int64_t ss
 // chunk sums, block_tc_scratch_bytes(p, i_count, n_cand_max) bytes.
 size_t block_tc_scratch_bytes(const Problem& p, int i_count, int64_t n_cand_max);
 // Queries per CTA of the tensor-core sweeps (token and block) over rows of up
-// to n_cand_max candidates; the sweeps run one CTA per SM.
-int select_tc_qt(int64_t n_cand_max);
+// to n_cand_max candidates with G query heads per KV head; the sweeps run one
+// CTA per SM.
+int select_tc_qt(int64_t n_cand_max, int G);
 cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* k, const float* lse, int32_t* idx,
                                    void* scratch, int i_begin, int i_count, int64_t n_cand_max, int blk,
                                    cudaStream_t st);

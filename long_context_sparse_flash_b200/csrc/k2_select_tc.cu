@@ -96,6 +96,12 @@ struct Lay<COUNTER> {
     static constexpr int QT = 28, EPI_WARPS = 28;
 };
 
+// COUNTER's MMA has N = 28 G columns: a valid M = 128 shape (a multiple of 16)
+// only for G of 4 and 8.  Calls with G of 1 or 2 keep ORDERED (N = 32 G) at
+// every length.
+template <int G>
+constexpr bool kCounterFits = (Lay<COUNTER>::QT * G) % 16 == 0;
+
 template <int D, int G, int L>
 struct SlCfg {
     static constexpr int QT = Lay<L>::QT;               // queries per CTA
@@ -128,6 +134,8 @@ struct SlCfg {
     static constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : (2 * N <= 256) ? 256 : 512;
     static_assert(NWG <= 8, "named barriers 1..NWG");
     static_assert(QT % NWG == 0, "whole queries per warpgroup");
+    static_assert(N % 16 == 0 && N <= 256, "MMA N of an M = 128 tcgen05.mma: a multiple of 16, at most 256");
+    static_assert(N / NWG >= 8, "a warpgroup's columns fill one tensor-memory load of at least 8 columns");
 };
 
 enum : int { SB_Q = 0, SB_KFULL = 1, SB_KEMPTY = SB_KFULL + SL_NS, SB_SFULL = SB_KEMPTY + SL_NS,
@@ -946,8 +954,10 @@ cudaError_t launch_select_dgl(const Problem& p, const void* q, const void* k, co
 template <int D, int G>
 cudaError_t launch_select_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
                              cudaStream_t st) {
-    return layout == COUNTER ? launch_select_dgl<D, G, COUNTER>(p, q, k, a, st)
-                             : launch_select_dgl<D, G, ORDERED>(p, q, k, a, st);
+    if constexpr (kCounterFits<G>) {
+        if (layout == COUNTER) return launch_select_dgl<D, G, COUNTER>(p, q, k, a, st);
+    }
+    return launch_select_dgl<D, G, ORDERED>(p, q, k, a, st);
 }
 
 template <int D, int G, int L>
@@ -962,8 +972,10 @@ cudaError_t launch_block_dgl(const Problem& p, const void* q, const void* k, con
 template <int D, int G>
 cudaError_t launch_block_dg(const Problem& p, const void* q, const void* k, const SelArgs& a, int layout,
                             cudaStream_t st) {
-    return layout == COUNTER ? launch_block_dgl<D, G, COUNTER>(p, q, k, a, st)
-                             : launch_block_dgl<D, G, ORDERED>(p, q, k, a, st);
+    if constexpr (kCounterFits<G>) {
+        if (layout == COUNTER) return launch_block_dgl<D, G, COUNTER>(p, q, k, a, st);
+    }
+    return launch_block_dgl<D, G, ORDERED>(p, q, k, a, st);
 }
 
 template <int D>
@@ -991,17 +1003,20 @@ cudaError_t launch_select_d(const Problem& p, const void* q, const void* k, cons
 }  // namespace
 
 // The epilogue layout of a call whose longest row has n_cand_max candidates.
-static int select_tc_layout(int64_t n_cand_max) { return n_cand_max >= SL_COUNTER_MIN_CAND ? COUNTER : ORDERED; }
+static int select_tc_layout(int64_t n_cand_max, int G) {
+    const bool fits = G == 4 ? kCounterFits<4> : G == 8 ? kCounterFits<8> : false;
+    return n_cand_max >= SL_COUNTER_MIN_CAND && fits ? COUNTER : ORDERED;
+}
 
-int select_tc_qt(int64_t n_cand_max) {
-    return select_tc_layout(n_cand_max) == COUNTER ? Lay<COUNTER>::QT : Lay<ORDERED>::QT;
+int select_tc_qt(int64_t n_cand_max, int G) {
+    return select_tc_layout(n_cand_max, G) == COUNTER ? Lay<COUNTER>::QT : Lay<ORDERED>::QT;
 }
 
 // Layout, survivor list capacity and slot count of a call over queries with up
 // to n_cand_max candidates, in CTAs of the layout's qt queries.
 static void select_tc_geometry(const Problem& p, int i_count, int64_t n_cand_max, int& layout, int& qt, int& cmax,
                                int& n_slots, int& by_block) {
-    layout = select_tc_layout(n_cand_max);
+    layout = select_tc_layout(n_cand_max, p.hq / p.hkv);
     qt = layout == COUNTER ? Lay<COUNTER>::QT : Lay<ORDERED>::QT;
     cmax = n_cand_max <= SL_CMAX ? (int)((n_cand_max + 31) / 32 * 32) : SL_CMAX;
     if (cmax < 32) cmax = 32;
@@ -1074,7 +1089,7 @@ cudaError_t launch_block_select_tc(const Problem& p, const void* q, const void* 
     if (n_cand_max / blk > p.topk / blk && p.topk >= blk) {
         // the token sweep's epilogue geometry for this candidate count (the chunk
         // sums are the same in both)
-        const int layout = select_tc_layout(n_cand_max);
+        const int layout = select_tc_layout(n_cand_max, p.hq / p.hkv);
         const cudaError_t e = p.D == 64 ? launch_block_d<64>(p, q, k, a, layout, st)
                                         : launch_block_d<128>(p, q, k, a, layout, st);
         if (e != cudaSuccess) return e;

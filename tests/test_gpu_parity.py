@@ -409,6 +409,22 @@ def test_counter_layout_every_row(name, kw):
     _row_properties(gpu["idx"], w)
 
 
+@pytest.mark.parametrize("name,kw", [
+    ("long_g1", dict(n_q=40, q_pos0=270000, h_q=2, h_kv=2, head_dim=128, window=128, topk=1024)),
+    ("long_g2", dict(n_q=40, q_pos0=270000, h_q=4, h_kv=2, head_dim=64, window=64, topk=512)),
+], ids=["g1", "g2"])
+def test_long_rows_with_one_or_two_heads_per_group(name, kw):
+    """More than 2^18 candidates per row with G = 1 or 2 query heads per KV head:
+    the COUNTER layout's MMA (N = 28 G columns) is not a valid tcgen05 shape for
+    these G, so the sweep keeps ORDERED (N = 32 G); every row against the oracle."""
+    w = wl.custom(name, n_sparse=1, seed=16, **kw)
+    assert w.q_pos0 + w.n_q - w.window >= COUNTER_MIN_CAND
+    inp = wl.make_inputs(w, "cuda")
+    gpu = P.run_gpu(w, inp)
+    P.compare_rows(w, inp, gpu, 0, np.arange(w.n_q))
+    _row_properties(gpu["idx"], w)
+
+
 def test_counter_layout_exact_ties():
     """q = 0 over 270K candidates: every score is G/(t+1), every candidate passes
     the bound, the lists overflow and are compacted with the lower-j tie-break,
