@@ -82,11 +82,15 @@ template <int D>
 struct PpCfg {
     static constexpr int KB = D / 64;                  // 64-element (128-byte) column blocks
     static constexpr int BLK = 128 * 128;              // one block: 128 rows x 128 B
-    static constexpr int NS = D == 64 ? 4 : 2;         // K/V ring stages
+    // ring stages of K and V tiles: K(j+1) and V(j) may only load once the MMAs
+    // of tile j-NS have freed their slots, and a 64 KB tile pair from L2 takes
+    // about one tile period to land; at D = 128 shared memory holds one more
+    // 32 KB stage, which goes to K (2-3% faster at a 1M context)
+    static constexpr int NSK = D == 64 ? 4 : 3, NSV = D == 64 ? 4 : 2;
     static constexpr int Q_OFF = 0;                    // [tile][kb] BLK
     static constexpr int K_OFF = Q_OFF + PP_QT * KB * BLK;
-    static constexpr int V_OFF = K_OFF + NS * KB * BLK;
-    static constexpr int BAR_OFF = V_OFF + NS * KB * BLK;
+    static constexpr int V_OFF = K_OFF + NSK * KB * BLK;
+    static constexpr int BAR_OFF = V_OFF + NSV * KB * BLK;
     static constexpr int SMEM = BAR_OFF + 256 + 1024;
     // TMEM columns: S[tile] 128 each at 0 and 128 (P[tile], 128 bf16 keys =
     // 64 columns, overwrites the first half of S[tile] once it has been read),
@@ -171,7 +175,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                                                                   float* __restrict__ part_o,
                                                                   float* __restrict__ part_l) {
     using C = PpCfg<D>;
-    constexpr int NS = C::NS;
+    constexpr int NSK = C::NSK, NSV = C::NSV;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     uint8_t* sgen = smem_raw + (sbase - smem_u32(smem_raw));
@@ -226,8 +230,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             bool ok = true;
             for (int j = 0; ok && j <= n_tiles; ++j) {
                 if (j < n_tiles) {
-                    const int s = j % NS;
-                    if (j >= NS) ok = tc::mbar_wait(bar(PB_KEMPTY + s), ((j - NS) / NS) & 1, ab, p.err, KID_FULL, 1);
+                    const int s = j % NSK;
+                    if (j >= NSK) ok = tc::mbar_wait(bar(PB_KEMPTY + s), ((j - NSK) / NSK) & 1, ab, p.err, KID_FULL, 1);
                     if (!ok) break;
                     tc::mbar_expect_tx(bar(PB_KFULL + s), C::KB * C::BLK);
                     for (int kb = 0; kb < C::KB; ++kb)
@@ -236,8 +240,8 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
                     k_issued = j + 1;
                 }
                 if (j >= 1) {
-                    const int jv = j - 1, s = jv % NS;
-                    if (jv >= NS) ok = tc::mbar_wait(bar(PB_VEMPTY + s), ((jv - NS) / NS) & 1, ab, p.err, KID_FULL, 2);
+                    const int jv = j - 1, s = jv % NSV;
+                    if (jv >= NSV) ok = tc::mbar_wait(bar(PB_VEMPTY + s), ((jv - NSV) / NSV) & 1, ab, p.err, KID_FULL, 2);
                     if (!ok) break;
                     tc::mbar_expect_tx(bar(PB_VFULL + s), C::KB * C::BLK);
                     for (int kb = 0; kb < C::KB; ++kb)
@@ -249,10 +253,10 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             if (!ok || ab->flag) {  // drain: every issued load lands before the CTA exits
                 tc::Abort none{0};
                 tc::mbar_wait(bar(PB_Q), 0, &none, nullptr, 0, 0);
-                for (int j = (k_issued > NS ? k_issued - NS : 0); j < k_issued; ++j)
-                    tc::mbar_wait(bar(PB_KFULL + j % NS), (j / NS) & 1, &none, nullptr, 0, 0);
-                for (int j = (v_issued > NS ? v_issued - NS : 0); j < v_issued; ++j)
-                    tc::mbar_wait(bar(PB_VFULL + j % NS), (j / NS) & 1, &none, nullptr, 0, 0);
+                for (int j = (k_issued > NSK ? k_issued - NSK : 0); j < k_issued; ++j)
+                    tc::mbar_wait(bar(PB_KFULL + j % NSK), (j / NSK) & 1, &none, nullptr, 0, 0);
+                for (int j = (v_issued > NSV ? v_issued - NSV : 0); j < v_issued; ++j)
+                    tc::mbar_wait(bar(PB_VFULL + j % NSV), (j / NSV) & 1, &none, nullptr, 0, 0);
             }
         }
       } else if (warp == PP_MMA_WARP) {
@@ -270,7 +274,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
         const uint64_t dq0 = tc::sdesc_sw128(sQ, 16, 1024), dk0 = tc::sdesc_sw128(sK, 16, 1024);
         const uint64_t dv0 = tc::sdesc_sw128(sV, C::BLK, 1024);
         auto issue_s = [&](int x, int j) {
-            const int s = j % NS;
+            const int s = j % NSK;
             if (tc::elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
@@ -283,7 +287,7 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             __syncwarp();
         };
         auto issue_pv = [&](int x, int j) {
-            const int s = j % NS;
+            const int s = j % NSV;
             if (tc::elect_one()) {
 #pragma unroll
                 for (int kk = 0; kk < PP_BN / 16; ++kk) {
@@ -306,11 +310,11 @@ __global__ void __launch_bounds__(PP_THREADS, 1) k1_full_tc_kernel(const __grid_
             commit(PB_KEMPTY);
         }
         for (int j = 0; ok && j < n_tiles; ++j) {
-            const int s = j % NS, s1 = (j + 1) % NS;
+            const int s = j % NSV, s1 = (j + 1) % NSK;
             const bool more = j + 1 < n_tiles;
-            ok = __all_sync(~0u, tc::mbar_wait(bar(PB_VFULL + s), (j / NS) & 1, ab, p.err, KID_FULL, 5));
+            ok = __all_sync(~0u, tc::mbar_wait(bar(PB_VFULL + s), (j / NSV) & 1, ab, p.err, KID_FULL, 5));
             if (ok && more)
-                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL + s1), ((j + 1) / NS) & 1, ab, p.err, KID_FULL, 6));
+                ok = __all_sync(~0u, tc::mbar_wait(bar(PB_KFULL + s1), ((j + 1) / NSK) & 1, ab, p.err, KID_FULL, 6));
             for (int x = 0; ok && x < PP_QT; ++x) {
                 ok = __all_sync(~0u, tc::mbar_wait(bar(PB_PFULL + x), j & 1, ab, p.err, KID_FULL, 7));
                 if (!ok) break;
