@@ -44,7 +44,9 @@ def slice_offsets(kv_len: int, n_slices: int) -> List[int]:
 def _ws(shape, kv_off: int, entry: int, device, stream=None) -> torch.Tensor:
     n = nv.hs2_cp_workspace_size(shape, kv_off, entry)
     if n == 0:
-        raise nv.HS2Error(1, "hs2_cp_workspace_size")
+        # 0: the shape is invalid or not supported by the slice calls (n_q >= 64,
+        # head_dim in {64, 128}, G in {1, 2, 4, 8}, ...)
+        raise nv.HS2Error(1, "hs2_cp_workspace_size (shape not accepted by the slice calls)")
     ws = torch.empty(n, dtype=torch.uint8, device=device)
     nv.hs2_workspace_init(ws, stream=stream)
     return ws
