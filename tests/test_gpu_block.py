@@ -79,6 +79,7 @@ BLOCK_SHAPES = [
     # more than 2^18 candidates per row: the sweep's 28-query geometry (COUNTER)
     ("b64_counter_270k", 64, dict(n_q=64, q_pos0=270000, h_q=16, h_kv=2, head_dim=128, window=128, topk=1024)),
     ("b32_counter_g4_d64", 32, dict(n_q=40, q_pos0=270000, h_q=8, h_kv=2, head_dim=64, window=64, topk=512)),
+    ("b64_counter_g8_d64", 64, dict(n_q=36, q_pos0=262300, h_q=16, h_kv=2, head_dim=64, window=128, topk=1024)),
     # G = 2 above 2^18 candidates keeps the 32-query geometry
     ("b128_long_g2", 128, dict(n_q=40, q_pos0=270000, h_q=4, h_kv=2, head_dim=64, window=64, topk=1024)),
 ]

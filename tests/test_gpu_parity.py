@@ -398,7 +398,8 @@ COUNTER_MIN_CAND = 1 << 18
     ("counter_d64_g4", dict(n_q=33, q_pos0=270000, h_q=16, h_kv=4, head_dim=64, window=64, topk=512)),
     ("counter_topk2048", dict(n_q=30, q_pos0=265000, h_q=16, h_kv=2, head_dim=128, window=128, topk=2048)),
     ("counter_batch2", dict(batch=2, n_q=31, q_pos0=263000, h_q=8, h_kv=2, head_dim=128, window=128, topk=1024)),
-], ids=["segments", "d64_g4", "topk2048", "batch2"])
+    ("counter_d64_g8", dict(n_q=30, q_pos0=262300, h_q=16, h_kv=2, head_dim=64, window=128, topk=1024)),
+], ids=["segments", "d64_g4", "topk2048", "batch2", "d64_g8"])
 def test_counter_layout_every_row(name, kw):
     w = wl.custom(name, n_sparse=1, seed=15, **kw)
     assert w.q_pos0 + w.n_q - w.window >= COUNTER_MIN_CAND
