@@ -235,6 +235,31 @@ def test_block_select_validation_without_launch():
     assert nv.hs2_launch_count() == before
 
 
+def test_block_select_chunks_in_whole_waves():
+    """At the 1M chunk the chunk sums of all 4096 queries exceed the 1 GiB budget,
+    so the sweep runs over chunks of queries; each chunk is a whole number of
+    waves of one-CTA-per-SM sweeps (148 CTAs of 28 queries for G = 8 above 2^18
+    candidates, 32 queries for G = 2), and the workspace holds one chunk."""
+    def expected(s_kw, qt):
+        s = shape(**s_kw)
+        B, hkv, nq, D, hq = s_kw["batch"], s_kw["h_kv"], s_kw["n_q"], s_kw["head_dim"], s_kw["h_q"]
+        cand = s_kw["q_pos0"] + nq - s_kw["window"]
+        per_q = B * hkv * (-(-cand // 128) * 4) * 4
+        fit = (1 << 30) // per_q
+        wave_q = 148 // (hkv * B) * qt
+        chunk = fit // wave_q * wave_q
+        # the full layer's split parts (2 key ranges at this shape) share the body with the sums
+        split = 2 * B * hq * nq * (D * 4 + 4) + 256
+        return nv.hs2_workspace_size(s, nv.HS2_ENTRY_BLOCK_SELECT), 256 + max(split, chunk * per_q), chunk
+    kw = dict(batch=1, n_q=4096, h_q=32, h_kv=4, head_dim=128, window=128, topk=1024, q_pos0=1048576,
+              kv_len=1052672)
+    got, want, chunk = expected(kw, 28)
+    assert chunk == 1036 and got == want
+    kw2 = dict(kw, h_q=8)  # G = 2: the 32-query geometry
+    got, want, chunk = expected(kw2, 32)
+    assert chunk == 1184 and got == want
+
+
 def test_swa_branches_validation_without_launch():
     """The two-branch comparator entry: shape, pointers, alignment, workspace, empty calls."""
     L = nv.load()
